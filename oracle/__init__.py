@@ -1,0 +1,270 @@
+"""CPU oracle for the activation-sparse linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (``sparse_input_gemv_threshold_b200``) never imports
+it, and it never imports the product: the two share no code.  The only module
+both sides use is ``workloads`` (seeded random inputs, no method arithmetic).
+
+It is a plain, slow, obviously correct restatement in numpy float64 of what the
+pages define.  Library primitives (a stable sort, a float64 matrix product,
+``exp``, the fp64 -> fp16 cast) serve as single steps; nothing is blocked, fused
+or reordered.
+
+Sources, cited by page title and section:
+
+* [QS]   "Q-Sparse: All Large Language Models can be Fully Sparsely-Activated"
+         (OpenReview rebuttal).  A1 to the second reviewer defines activation
+         sparsity as the share of zero entries of X in WX; A3 (FLOPs) counts
+         2 d^2 for a d x d by d x 1 product; A1 on MoE says Q-Sparse keeps, per
+         token, the entries of largest magnitude; A2 (batched inference) brings
+         in Block Q-Sparse with N:M activation sparsity.
+* [TEAL] "Training-Free Activation Sparsity in Large Language Models" (TEAL
+         README), Abstract: magnitude-based activation sparsity of the hidden
+         states that feed each matrix multiplication.
+* [RaNA] "Adaptive Rank Allocation: Speeding Up Modern Transformers with RaNA
+         Adapters" (OpenReview rebuttal): Q3, Eqn. 12 (RaNA neuron masker) and
+         the CATS masker beside it; Q5.1, the masked product A(m(x) . Bx) that
+         skips the columns whose mask entry is 0.
+* [NM]   "Motivating Next-Gen Accelerators with Flexible (N:M) Activation
+         Sparsity ..." (summary), Methodology: in blocks of size M, N non-zero
+         elements are kept; selection criterion ACT = absolute activation size.
+
+Readings where the pages are silent or disagree (each one is a choice):
+
+* Threshold comparison is ``|x_i| >= t`` ([RaNA] Eqn. 12 writes ``>= t``; TEAL
+  gives no operator).  A NaN is never kept by a threshold.
+* Ranking by magnitude (top-k, N:M): larger |x| first, equal |x| by lower index
+  first; +v and -v tie, +0 and -0 tie; a NaN ranks below every number.
+* N:M keeps the N largest of each M consecutive elements ([NM] Methodology;
+  [QS] A2 words it as "N ... to be zero", which the 50 % patterns do not tell
+  apart; 1:4 read as keep one of four, 75 % sparsity).
+* ||W^down_i||_F in Eqn. 12 is the l2 norm of the weights that multiply neuron
+  i, i.e. row i of the transposed down weight, computed in float64 and rounded
+  once to float32.
+* Eqn. 12 precision: g and u in float64 from the fp16 inputs, h rounded once to
+  fp16, ``s_i = float32(|h_i|) * norm_i`` as one float32 multiply, ``s_i >= t``.
+* Outputs: y in float64 (used for the error bound) and rounded once to fp16.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, hand-derived fixtures under ``tests/golden/``, brute force on
+tiny inputs, reductions to the dense product).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "fp16", "magnitude_order", "threshold_mask", "topk_mask", "nm_mask",
+    "compact", "pack_bits", "unpack_bits", "sparsity", "flops",
+    "masked_matvec", "sparse_linear", "silu", "row_norms", "rana_hidden",
+    "rana_scores", "rana_mask", "gated_mlp", "nm_gemm",
+]
+
+
+# ---------------------------------------------------------------------------
+# Rounding
+# ---------------------------------------------------------------------------
+
+def fp16(v) -> np.ndarray:
+    """Round float64 values once to IEEE binary16, round-to-nearest-even.
+
+    numpy's float64 -> float16 cast rounds directly from the 52-bit mantissa
+    (no detour through float32); the pins check this against exact rational
+    arithmetic, including values just off a halfway point.
+    """
+    with np.errstate(over="ignore"):
+        return np.asarray(v, dtype=np.float64).astype(np.float16)
+
+
+# ---------------------------------------------------------------------------
+# Masks
+# ---------------------------------------------------------------------------
+
+def _magnitude_key(x) -> np.ndarray:
+    """|x| in float64 with NaN mapped below every magnitude (to -1)."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    return np.where(np.isnan(a), -1.0, a)
+
+
+def magnitude_order(x) -> np.ndarray:
+    """Indices of a 1-D ``x`` by |x| descending, ties by lower index ([QS] A1 on MoE)."""
+    key = _magnitude_key(x)
+    return np.argsort(-key, kind="stable")
+
+
+def threshold_mask(x, t: float) -> np.ndarray:
+    """[TEAL] Abstract: keep x_i when |x_i| >= t (a NaN is never kept)."""
+    return np.abs(np.asarray(x, dtype=np.float64)) >= np.float64(t)
+
+
+def topk_mask(x, k: int) -> np.ndarray:
+    """[QS] A1 on MoE: per token keep the k entries of largest magnitude."""
+    x = np.asarray(x).ravel()
+    if not 0 <= k <= x.size:
+        raise ValueError("k out of range")
+    m = np.zeros(x.size, dtype=bool)
+    m[magnitude_order(x)[:k]] = True
+    return m
+
+
+def nm_mask(X, n: int, m: int) -> np.ndarray:
+    """[NM] Methodology / [QS] A2: per row, in each block of M consecutive
+    elements keep the N of largest magnitude (ties by lower index)."""
+    X = np.asarray(X)
+    squeeze = X.ndim == 1
+    X2 = X.reshape(1, -1) if squeeze else X
+    rows, d = X2.shape
+    if not (1 <= n <= m) or d % m:
+        raise ValueError("need 1 <= n <= m and m | d")
+    key = _magnitude_key(X2).reshape(rows, d // m, m)
+    order = np.argsort(-key, axis=-1, kind="stable")
+    keep = np.zeros((rows, d // m, m), dtype=bool)
+    np.put_along_axis(keep, order[..., :n], True, axis=-1)
+    keep = keep.reshape(rows, d)
+    return keep[0] if squeeze else keep
+
+
+def compact(mask) -> np.ndarray:
+    """Ascending int32 indices of the kept entries ([RaNA] Q5.1: the product
+    skips the columns whose mask entry is 0, so only these are visited)."""
+    return np.flatnonzero(np.asarray(mask).ravel()).astype(np.int32)
+
+
+def pack_bits(mask) -> np.ndarray:
+    """Bit i%32 of uint32 word i//32 is mask[i] (little-endian within a word).
+
+    A 2-D mask packs each row separately, rows padded to whole words.
+    """
+    mask = np.asarray(mask, dtype=bool)
+    if mask.ndim == 2:
+        return np.stack([pack_bits(r) for r in mask]) if len(mask) else \
+            np.zeros((0, (mask.shape[1] + 31) // 32), np.uint32)
+    d = mask.size
+    words = (d + 31) // 32
+    padded = np.zeros(words * 32, dtype=np.uint64)
+    padded[:d] = mask
+    weights = np.left_shift(np.uint64(1), np.arange(32, dtype=np.uint64))
+    return (padded.reshape(words, 32) * weights).sum(axis=1).astype(np.uint32)
+
+
+def unpack_bits(words, d: int) -> np.ndarray:
+    """Inverse of :func:`pack_bits` for one row of ``d`` entries."""
+    words = np.asarray(words, dtype=np.uint32)
+    bits = (words[:, None] >> np.arange(32, dtype=np.uint32)) & np.uint32(1)
+    return bits.ravel()[:d].astype(bool)
+
+
+def sparsity(mask) -> float:
+    """[QS] A1 to the second reviewer: share of zero entries of the masked input."""
+    mask = np.asarray(mask)
+    return float(1.0 - mask.sum() / mask.size) if mask.size else 0.0
+
+
+def flops(d_out: int, nnz: int) -> int:
+    """[QS] A3: a d_out x d_in by d_in x 1 product costs 2 d_out d_in; with
+    only nnz inputs kept it costs 2 d_out nnz (mask cost left out)."""
+    return 2 * int(d_out) * int(nnz)
+
+
+# ---------------------------------------------------------------------------
+# The sparse-input product y = W (m . x)
+# ---------------------------------------------------------------------------
+
+def masked_matvec(WT, x, mask, cols=None):
+    """y_j = sum_i WT[i, j] * (m_i ? x_i : 0) in float64 ([RaNA] Q5.1).
+
+    ``WT`` is the transposed weight (d_in, d_out): row i multiplies input i.
+    Returns ``(y64, bound)`` with ``bound_j = sum_i |WT[i, j] * m_i x_i|``,
+    the scale of the per-element error tolerance.  ``cols`` restricts the
+    output to a subset of output columns.
+    """
+    WT = np.asarray(WT)
+    if cols is not None:
+        WT = WT[:, np.asarray(cols)]
+    xm = np.where(np.asarray(mask, dtype=bool), np.asarray(x, dtype=np.float64), 0.0)
+    W64 = WT.astype(np.float64)
+    y64 = xm @ W64
+    bound = np.abs(xm) @ np.abs(W64)
+    return y64, bound
+
+
+def sparse_linear(WT, x, mask, cols=None) -> dict:
+    """Mask applied, product taken, result rounded once to fp16."""
+    y64, bound = masked_matvec(WT, x, mask, cols)
+    idx = compact(mask)
+    return {"mask": np.asarray(mask, dtype=bool), "idx": idx, "nnz": int(idx.size),
+            "y64": y64, "y16": fp16(y64), "bound": bound}
+
+
+# ---------------------------------------------------------------------------
+# RaNA gated-MLP neuron masker (Eqn. 12)
+# ---------------------------------------------------------------------------
+
+def silu(z):
+    """SiLU(z) = z * sigmoid(z) = z / (1 + exp(-z)), float64."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def row_norms(WT) -> np.ndarray:
+    """l2 norm of each row of a transposed weight, float64, rounded to float32.
+
+    For the down projection, row i of WdT holds the weights that multiply
+    neuron i: the ||W^down_i||_F of [RaNA] Eqn. 12.
+    """
+    W64 = np.asarray(WT).astype(np.float64)
+    return np.sqrt((W64 * W64).sum(axis=1)).astype(np.float32)
+
+
+def rana_hidden(x, WgT, WuT):
+    """g = GateProj(x), u = UpProj(x) in float64; h = fp16(SiLU(g) * u).
+
+    h is the input of the down projection ([RaNA] Q3, the sentence after
+    Eqn. 12).
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    g = x64 @ np.asarray(WgT).astype(np.float64)
+    u = x64 @ np.asarray(WuT).astype(np.float64)
+    return g, u, fp16(silu(g) * u)
+
+
+def rana_scores(h16, norms32) -> np.ndarray:
+    """s_i = |h_i| * ||W^down_i|| as one float32 multiply ([RaNA] Eqn. 12)."""
+    h32 = np.abs(np.asarray(h16, dtype=np.float16)).astype(np.float32)
+    return (h32 * np.asarray(norms32, dtype=np.float32)).astype(np.float32)
+
+
+def rana_mask(s32, t: float) -> np.ndarray:
+    """m_i = s_i >= t, compared in float32 ([RaNA] Eqn. 12)."""
+    return np.asarray(s32, dtype=np.float32) >= np.float32(t)
+
+
+def gated_mlp(x, WgT, WuT, WdT, norms32, t: float, cols=None) -> dict:
+    """Eqn. 12 masker then the masked down projection y = W_down (m . h)."""
+    g, u, h16 = rana_hidden(x, WgT, WuT)
+    s32 = rana_scores(h16, norms32)
+    m = rana_mask(s32, t)
+    out = sparse_linear(WdT, h16, m, cols)
+    out.update({"g": g, "u": u, "h16": h16, "s32": s32})
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Block Q-Sparse batched product Y = (M . X) WT
+# ---------------------------------------------------------------------------
+
+def nm_gemm(X, WT, mask, rows=None):
+    """Y[r, j] = sum_i (M . X)[r, i] WT[i, j] in float64 ([QS] A2, Block Q-Sparse).
+
+    Returns ``(Y64, bound)`` with ``bound[r, j] = sum_i |(M . X)[r, i] WT[i, j]|``.
+    ``rows`` restricts the output to a subset of tokens.
+    """
+    X = np.asarray(X)
+    mask = np.asarray(mask, dtype=bool)
+    if rows is not None:
+        X, mask = X[np.asarray(rows)], mask[np.asarray(rows)]
+    Xm = np.where(mask, X.astype(np.float64), 0.0)
+    W64 = np.asarray(WT).astype(np.float64)
+    return Xm @ W64, np.abs(Xm) @ np.abs(W64)

@@ -1,0 +1,471 @@
+"""Pins for the CPU oracle: checks against what the pages and mathematics fix.
+
+None of these re-types the oracle's formula or re-calls its library routine.
+They use hand-derived fixtures (tests/golden/), exact rational arithmetic,
+closed forms, brute force over all subsets on tiny inputs, pure-Python loops,
+and reductions to the plain dense product.
+"""
+import itertools
+import math
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests.conftest import golden_path
+
+
+# ---------------------------------------------------------------------------
+# fixtures readers
+# ---------------------------------------------------------------------------
+
+def _floats(s):
+    return [float(v) for v in s.split()]
+
+
+def _read_lines(name):
+    with open(golden_path(name)) as f:
+        return [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ---------------------------------------------------------------------------
+# fp16 round-to-nearest-even
+# ---------------------------------------------------------------------------
+
+def _fp16_exact(v: Fraction) -> Fraction:
+    """Binary16 RNE by exact rational arithmetic (finite results only)."""
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = math.floor(math.log2(a))
+    # adjust for log2 rounding
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -14)                      # subnormals share the 2^-14 binade spacing
+    ulp = Fraction(2) ** (e - 10)
+    q, r = divmod(a, ulp)
+    if r * 2 > ulp or (r * 2 == ulp and q % 2 == 1):
+        q += 1
+    return sign * q * ulp
+
+
+def test_fp16_roundtrips_every_bit_pattern():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    h = bits.view(np.float16)
+    back = oracle.fp16(h.astype(np.float64))
+    nan = np.isnan(h)
+    assert np.array_equal(back.view(np.uint16)[~nan], bits[~nan])
+    assert np.isnan(back[nan]).all()
+
+
+def test_fp16_halfway_and_off_halfway_against_exact_rationals():
+    rng = np.random.default_rng(1)
+    pos = np.arange(1, 0x7BFF, dtype=np.uint16)   # finite positives, a < b pairs
+    pick = rng.choice(pos, 400, replace=False)
+    picks = np.concatenate([pick, [1, 2, 0x3FF, 0x400, 0x401, 0x3BFF, 0x3C00, 0x7BFE]]).astype(np.uint16)
+    for b in picks:
+        a = np.array([b], dtype=np.uint16).view(np.float16)[0]
+        c = np.array([b + 1], dtype=np.uint16).view(np.float16)[0]
+        mid = (float(a) + float(c)) / 2.0           # exact in float64
+        for v in (mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf)):
+            want = _fp16_exact(Fraction(float(v)))
+            got = Fraction(float(oracle.fp16(v)))
+            assert got == want, (float(a), float(c), float(v))
+            # and for the negative side
+            assert Fraction(float(oracle.fp16(-v))) == -want
+
+
+def test_fp16_overflow_and_underflow_edges():
+    assert float(oracle.fp16(65504.0)) == 65504.0
+    assert float(oracle.fp16(65519.99)) == 65504.0
+    assert math.isinf(float(oracle.fp16(65520.0)))      # tie goes to even = 2^16 = inf
+    assert float(oracle.fp16(2.0 ** -25)) == 0.0         # tie to even (0)
+    assert float(oracle.fp16(np.nextafter(2.0 ** -25, 1.0))) == 2.0 ** -24
+
+
+# ---------------------------------------------------------------------------
+# masks
+# ---------------------------------------------------------------------------
+
+def test_threshold_golden():
+    lines = _read_lines("threshold_small.txt")
+    x = np.array(_floats(lines[0].split(":", 1)[1]), dtype=np.float16)
+    n = 0
+    for ln in lines[1:]:
+        t, m = ln.split(":", 1)[1].split("|")
+        want = np.array([int(v) for v in m.split()], dtype=bool)
+        assert np.array_equal(oracle.threshold_mask(x, float(t)), want), ln
+        n += 1
+    assert n == 5
+
+
+def test_threshold_matches_brute_force_loop_and_sorted_count():
+    rng = np.random.default_rng(2)
+    x = workloads.draw_vector(rng, 3001, "laplace")
+    for s in (0.0, 0.25, 0.5, 0.65, 0.99):
+        t = workloads.quantile_threshold(x, s)
+        m = oracle.threshold_mask(x, t)
+        loop = [abs(float(v)) >= t for v in x]
+        assert m.tolist() == loop
+        mags = sorted(abs(float(v)) for v in x)
+        first = next(i for i, v in enumerate(mags) if v >= t)
+        assert int(m.sum()) == len(mags) - first
+        assert int(m.sum()) >= x.size - math.floor(s * x.size)
+
+
+def test_threshold_never_keeps_nan_and_keeps_inf():
+    x = np.array([np.nan, np.inf, -np.inf, 1.0], dtype=np.float16)
+    assert oracle.threshold_mask(x, 0.0).tolist() == [False, True, True, True]
+
+
+def test_topk_golden():
+    lines = _read_lines("topk_small.txt")
+    x = np.array(_floats(lines[0].split(":", 1)[1]), dtype=np.float16)
+    for ln in lines[1:]:
+        k, idx = ln.split(":", 1)[1].split("|")
+        want = [int(v) for v in idx.split()]
+        assert oracle.compact(oracle.topk_mask(x, int(k))).tolist() == want, ln
+
+
+def _lexmin_maxsum_subset(vals, k):
+    """All k-subsets; the max sum of |v| (exact in float64 for fp16 data),
+    the lexicographically smallest sorted index tuple among the maxima."""
+    best, best_set = None, None
+    for sub in itertools.combinations(range(len(vals)), k):  # lexicographic order
+        s = sum(abs(float(vals[i])) for i in sub)
+        if best is None or s > best:
+            best, best_set = s, sub
+    return list(best_set) if best_set is not None else []
+
+
+def test_topk_brute_force_tiny():
+    rng = np.random.default_rng(3)
+    for trial in range(60):
+        d = int(rng.integers(1, 10))
+        # few distinct magnitudes to force ties, random signs and signed zeros
+        vals = rng.choice([0.0, -0.0, 0.5, -0.5, 1.0, -1.0, 2.0, 3.0, -3.0], size=d)
+        x = np.array(vals, dtype=np.float16)
+        for k in range(d + 1):
+            got = oracle.compact(oracle.topk_mask(x, k)).tolist()
+            assert got == _lexmin_maxsum_subset(x, k), (x, k)
+
+
+def test_topk_invariants_large():
+    rng = np.random.default_rng(4)
+    x = workloads.draw_vector(rng, 28672, "student_t4")
+    mags = np.abs(x.astype(np.float64))
+    for f in workloads.QSPARSE_KEEP_FRACTIONS:
+        k = workloads.topk_count(f, x.size)
+        m = oracle.topk_mask(x, k)
+        assert int(m.sum()) == k
+        assert mags[m].min() >= mags[~m].max()
+        kstar = mags[m].min()
+        tie_kept = np.flatnonzero(m & (mags == kstar))
+        tie_drop = np.flatnonzero(~m & (mags == kstar))
+        if tie_drop.size:
+            assert tie_kept.max() < tie_drop.min()
+    assert workloads.topk_count(0.6, 8192) == 4915
+    assert workloads.topk_count(0.4, 28672) == 11469
+
+
+def test_topk_nan_ranks_last():
+    x = np.array([np.nan, 0.0, np.inf, -1.0, np.nan], dtype=np.float16)
+    assert oracle.compact(oracle.topk_mask(x, 3)).tolist() == [1, 2, 3]
+    assert oracle.compact(oracle.topk_mask(x, 4)).tolist() == [0, 1, 2, 3]
+
+
+def test_nm_golden():
+    lines = _read_lines("nm_small.txt")
+    row, checked = None, 0
+    for ln in lines:
+        if ln.startswith("row:"):
+            row = np.array(_floats(ln[4:]), dtype=np.float16)
+            continue
+        nm, m = ln.split("|")
+        n, mm = (int(v) for v in nm.split())
+        want = np.array([int(v) for v in m.split()], dtype=bool)
+        assert np.array_equal(oracle.nm_mask(row, n, mm), want), ln
+        checked += 1
+    assert checked == 8
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (3, 4), (4, 8), (8, 16)])
+def test_nm_brute_force_blocks(n, m):
+    rng = np.random.default_rng(5 + n + m)
+    rows = []
+    for _ in range(3):
+        rows.append(rng.choice([0.0, -0.0, 0.25, -0.25, 1.0, -1.0, 2.0], size=m))
+    rows.append(rng.laplace(0, 1, m))
+    X = np.array(rows, dtype=np.float16)
+    M = oracle.nm_mask(X, n, m)
+    for r in range(X.shape[0]):
+        assert int(M[r].sum()) == n
+        assert oracle.compact(M[r]).tolist() == _lexmin_maxsum_subset(X[r], n)
+
+
+def test_nm_exact_count_per_block_large():
+    WT, X = workloads.nm_tokens(seed=0, rows=64, d=1024, d_out=8)
+    for n, m in workloads.NM_PATTERNS:
+        M = oracle.nm_mask(X, n, m)
+        assert (M.reshape(64, -1, m).sum(-1) == n).all()
+        assert abs(oracle.sparsity(M) - (1 - n / m)) < 1e-12
+
+
+def test_nm_equals_topk_per_block():
+    """An N:M mask is top-N applied to each block on its own."""
+    rng = np.random.default_rng(6)
+    X = rng.laplace(0, 1, (5, 64)).astype(np.float16)
+    M = oracle.nm_mask(X, 8, 16)
+    for r in range(5):
+        for b in range(4):
+            blk = X[r, 16 * b:16 * (b + 1)]
+            assert np.array_equal(M[r, 16 * b:16 * (b + 1)], oracle.topk_mask(blk, 8))
+
+
+def test_pack_bits_known_words():
+    m = np.zeros(70, dtype=bool)
+    m[[0, 31, 32, 69]] = True
+    w = oracle.pack_bits(m)
+    assert w.tolist() == [0x80000001, 0x1, 0x20]
+    assert np.array_equal(oracle.unpack_bits(w, 70), m)
+
+
+def test_compact_is_ascending_and_complete():
+    m = np.array([0, 1, 1, 0, 0, 1], dtype=bool)
+    assert oracle.compact(m).tolist() == [1, 2, 5]
+    assert oracle.compact(np.zeros(4, bool)).tolist() == []
+
+
+# ---------------------------------------------------------------------------
+# product
+# ---------------------------------------------------------------------------
+
+def _triple_loop(W_rows, x, mask):
+    """y_j = sum_i W[j][i] * m_i x_i with W in its natural (d_out, d_in)
+    orientation, as the pages write W X ("Q-Sparse ...", A3)."""
+    d_out, d_in = len(W_rows), len(x)
+    y = []
+    for j in range(d_out):
+        acc = Fraction(0)
+        for i in range(d_in):
+            if mask[i]:
+                acc += Fraction(float(W_rows[j][i])) * Fraction(float(x[i]))
+        y.append(acc)
+    return y
+
+
+def test_product_matches_exact_triple_loop_nonsquare():
+    rng = np.random.default_rng(7)
+    d_in, d_out = 37, 23
+    W = rng.normal(0, 0.02, (d_out, d_in)).astype(np.float16)      # natural orientation
+    x = rng.laplace(0, 1, d_in).astype(np.float16)
+    mask = oracle.threshold_mask(x, workloads.quantile_threshold(x, 0.4))
+    y64, bound = oracle.masked_matvec(W.T.copy(), x, mask)
+    exact = _triple_loop(W, x, mask)
+    for j in range(d_out):
+        assert abs(Fraction(float(y64[j])) - exact[j]) <= Fraction(1, 10 ** 12) * (1 + abs(exact[j]))
+        b = sum(abs(Fraction(float(W[j, i])) * Fraction(float(x[i]))) for i in range(d_in) if mask[i])
+        assert abs(Fraction(float(bound[j])) - b) <= Fraction(1, 10 ** 12) * (1 + b)
+
+
+def test_product_identity_and_permutation():
+    rng = np.random.default_rng(8)
+    d = 64
+    x = rng.laplace(0, 1, d).astype(np.float16)
+    mask = oracle.topk_mask(x, 20)
+    out = oracle.sparse_linear(np.eye(d, dtype=np.float16), x, mask)
+    assert np.array_equal(out["y16"], np.where(mask, x, np.float16(0)))
+    perm = rng.permutation(d)
+    P = np.zeros((d, d), dtype=np.float16)          # y_j = x_{perm[j]}, so WT[perm[j], j] = 1
+    P[perm, np.arange(d)] = 1
+    out = oracle.sparse_linear(P, x, mask)
+    assert np.array_equal(out["y16"], np.where(mask[perm], x[perm], np.float16(0)))
+
+
+def test_zero_sparsity_reduces_to_dense_product():
+    rng = np.random.default_rng(9)
+    p = workloads.projection("t", 48, 40, sigma=0.02, dist="laplace", seed=9, sparsities=(0.0,))
+    for mask in (oracle.threshold_mask(p.x, p.thresholds[0.0]),
+                 oracle.topk_mask(p.x, p.d_in),
+                 oracle.nm_mask(p.x, 4, 4)):
+        assert mask.all()
+        y64, _ = oracle.masked_matvec(p.WT, p.x, mask)
+        exact = _triple_loop(p.WT.T, p.x, np.ones(p.d_in, bool))
+        assert all(abs(Fraction(float(a)) - b) <= Fraction(1, 10 ** 12) for a, b in zip(y64, exact))
+
+
+def test_empty_mask_gives_zero_output():
+    p = workloads.projection("t", 16, 8, sigma=0.02, dist="laplace", seed=1)
+    out = oracle.sparse_linear(p.WT, p.x, np.zeros(16, bool))
+    assert out["nnz"] == 0 and not out["y64"].any() and not out["bound"].any()
+
+
+def test_cols_subset_equals_full_columns():
+    p = workloads.projection("t", 32, 24, sigma=0.02, dist="laplace", seed=2)
+    m = oracle.topk_mask(p.x, 10)
+    full, _ = oracle.masked_matvec(p.WT, p.x, m)
+    cols = [3, 0, 23, 7]
+    sub, _ = oracle.masked_matvec(p.WT, p.x, m, cols=cols)
+    assert np.array_equal(sub, full[cols])
+
+
+def test_flops_and_sparsity_definitions():
+    # "Q-Sparse ...", A3: 2 d^2 for a d x d weight and a d x 1 input.
+    assert oracle.flops(4096, 4096) == 2 * 4096 ** 2
+    x = workloads.draw_vector(np.random.default_rng(3), 4096, "laplace")
+    for s in workloads.LLAMA2_SPARSITIES:
+        m = oracle.threshold_mask(x, workloads.quantile_threshold(x, s))
+        # the Laplace draw has ties in fp16, so sparsity is at most the target
+        assert oracle.sparsity(m) <= s + 1e-12
+        assert oracle.flops(4096, int(m.sum())) == 2 * 4096 * int(m.sum())
+
+
+# ---------------------------------------------------------------------------
+# RaNA Eqn. 12
+# ---------------------------------------------------------------------------
+
+def _silu_decimal(z: float) -> Decimal:
+    getcontext().prec = 40
+    z = Decimal(z)
+    return z / (1 + (-z).exp())
+
+
+def test_silu_closed_forms():
+    assert float(oracle.silu(0.0)) == 0.0
+    ln3 = math.log(3.0)
+    # sigmoid(ln 3) = 3/4 and sigmoid(-ln 3) = 1/4
+    assert abs(float(oracle.silu(ln3)) - 0.75 * ln3) < 1e-15
+    assert abs(float(oracle.silu(-ln3)) + 0.25 * ln3) < 1e-15
+    zs = np.linspace(-30, 30, 241)
+    # SiLU(z) - SiLU(-z) = z
+    assert np.allclose(oracle.silu(zs) - oracle.silu(-zs), zs, atol=1e-13, rtol=0)
+    for z in (-20.0, -3.5, -0.1, 0.7, 5.0, 30.0):
+        assert abs(Decimal(float(oracle.silu(z))) - _silu_decimal(z)) <= Decimal(1e-15) * (1 + abs(_silu_decimal(z)))
+    assert float(oracle.silu(-1000.0)) == 0.0
+
+
+def _rana_fixture():
+    lines = dict(ln.split(":", 1) for ln in _read_lines("rana_eqn12.txt"))
+    return ({k: np.array(_floats(v)) for k, v in lines.items() if k in ("g", "u", "norm")},
+            float(lines["t"]), [int(v) for v in lines["rana"].split()],
+            [int(v) for v in lines["cats"].split()])
+
+
+def test_rana_eqn12_golden_and_cats():
+    vals, t, want_rana, want_cats = _rana_fixture()
+    d_ff = vals["g"].size
+    x = np.array([1.0], dtype=np.float16)
+    WgT = vals["g"].astype(np.float16).reshape(1, d_ff)
+    WuT = vals["u"].astype(np.float16).reshape(1, d_ff)
+    norms = vals["norm"].astype(np.float32)
+    g, u, h16 = oracle.rana_hidden(x, WgT, WuT)
+    assert np.array_equal(g, vals["g"]) and np.array_equal(u, vals["u"])
+    s = oracle.rana_scores(h16, norms)
+    for i in range(d_ff):
+        exact = abs(_silu_decimal(vals["g"][i]) * Decimal(vals["u"][i])) * Decimal(float(norms[i]))
+        # h is rounded once to fp16 (rel. 2^-11) and s once more to fp32
+        assert abs(Decimal(float(s[i])) - exact) <= exact * Decimal(2.0 ** -11 + 2.0 ** -23)
+    assert oracle.rana_mask(s, t).astype(int).tolist() == want_rana
+    # CATS ("RaNA ...", Q3) is Eqn. 12 with u = 1 and unit norms
+    ones = np.ones((1, d_ff), np.float16)
+    _, _, h_c = oracle.rana_hidden(x, WgT, ones)
+    s_c = oracle.rana_scores(h_c, np.ones(d_ff, np.float32))
+    assert oracle.rana_mask(s_c, t).astype(int).tolist() == want_cats
+    for i in range(d_ff):
+        assert abs(float(s_c[i]) - abs(float(_silu_decimal(vals["g"][i])))) <= 2.0 ** -11 * abs(float(s_c[i])) + 1e-30
+
+
+def test_rana_cats_special_case_random():
+    """u = 1 and norm = 1: the RaNA mask is |fp16(SiLU(g))| >= t, computed here
+    with scalar math.exp, independent of numpy."""
+    rng = np.random.default_rng(10)
+    d_model, d_ff = 8, 300
+    x = rng.normal(0, 1, d_model).astype(np.float16)
+    WgT = rng.normal(0, 0.5, (d_model, d_ff)).astype(np.float16)
+    WuT_ones = np.zeros((d_model, d_ff), np.float16)
+    # u = 1: put 1/x_0 ... simpler: x_0 = 1 and the u weights only on row 0
+    x[0] = 1.0
+    WuT_ones[0, :] = 1.0
+    g, u, h16 = oracle.rana_hidden(x, WgT, WuT_ones)
+    assert (u == 1.0).all()
+    s = oracle.rana_scores(h16, np.ones(d_ff, np.float32))
+    t = 0.3
+    m = oracle.rana_mask(s, t)
+    for i in range(d_ff):
+        gi = sum(float(x[k]) * float(WgT[k, i]) for k in range(d_model))
+        silu = gi / (1.0 + math.exp(-gi))
+        h = float(np.float16(silu))   # fp16 rounding; decision compared away from ties
+        if abs(abs(silu) - t) > 1e-3:
+            assert m[i] == (abs(h) >= t) == (abs(silu) >= t)
+
+
+def test_rana_scale_invariance():
+    """Doubling every norm and t leaves the mask unchanged (exact in fp32)."""
+    rng = np.random.default_rng(11)
+    h = rng.normal(0, 1, 500).astype(np.float16)
+    norms = np.abs(rng.normal(1, 0.2, 500)).astype(np.float32)
+    s1 = oracle.rana_scores(h, norms)
+    s2 = oracle.rana_scores(h, norms * np.float32(2))
+    assert np.array_equal(oracle.rana_mask(s1, 0.7), oracle.rana_mask(s2, 1.4))
+
+
+def test_row_norms_pythagorean():
+    WT = np.array([[3, 4, 0], [5, 12, 0], [1, 1, 1], [0, 0, 0]], dtype=np.float16)
+    assert oracle.row_norms(WT).tolist() == [5.0, 13.0, float(np.float32(math.sqrt(3))), 0.0]
+
+
+def test_gated_mlp_down_product_uses_h_and_mask():
+    vals, t, want_rana, _ = _rana_fixture()
+    d_ff = vals["g"].size
+    x = np.array([1.0], dtype=np.float16)
+    WgT = vals["g"].astype(np.float16).reshape(1, d_ff)
+    WuT = vals["u"].astype(np.float16).reshape(1, d_ff)
+    WdT = np.eye(d_ff, dtype=np.float16)         # y = m . h exactly
+    out = oracle.gated_mlp(x, WgT, WuT, WdT, vals["norm"].astype(np.float32), t)
+    want = np.where(np.array(want_rana, bool), out["h16"], np.float16(0))
+    assert np.array_equal(out["y16"], want)
+
+
+# ---------------------------------------------------------------------------
+# batched N:M product
+# ---------------------------------------------------------------------------
+
+def test_nm_gemm_rows_equal_masked_matvec_and_triple_loop():
+    WT, X = workloads.nm_tokens(seed=1, rows=6, d=32, d_out=5)
+    M = oracle.nm_mask(X, 2, 4)
+    Y, B = oracle.nm_gemm(X, WT, M)
+    for r in range(6):
+        exact = _triple_loop(WT.T, X[r], M[r])
+        assert all(abs(Fraction(float(a)) - b) <= Fraction(1, 10 ** 12) for a, b in zip(Y[r], exact))
+    Yn, _ = oracle.nm_gemm(X, WT, np.ones_like(M))
+    exact = _triple_loop(WT.T, X[0], np.ones(32, bool))
+    assert all(abs(Fraction(float(a)) - b) <= Fraction(1, 10 ** 12) for a, b in zip(Yn[0], exact))
+    Ysub, _ = oracle.nm_gemm(X, WT, M, rows=[4, 1])
+    assert np.array_equal(Ysub, Y[[4, 1]])
+
+
+# ---------------------------------------------------------------------------
+# input recipe
+# ---------------------------------------------------------------------------
+
+def test_quantile_threshold_hits_target_on_distinct_values():
+    x = np.arange(1, 1001, dtype=np.float16)         # distinct magnitudes
+    for s in (0.0, 0.25, 0.5, 0.65):
+        t = workloads.quantile_threshold(x, s)
+        assert int(oracle.threshold_mask(x, t).sum()) == 1000 - math.floor(s * 1000)
+
+
+def test_workloads_are_seeded_and_chunking_invariant():
+    a = workloads.tiny_gemv(0)
+    b = workloads.tiny_gemv(0)
+    assert np.array_equal(a.WT, b.WT) and np.array_equal(a.x, b.x)
+    rng = np.random.default_rng(0)
+    direct = rng.normal(0.0, 0.02, 1024 * 1024).astype(np.float16).reshape(1024, 1024)
+    assert np.array_equal(direct, a.WT)
+    assert a.thresholds[0.5] == workloads.quantile_threshold(a.x, 0.5)
