@@ -1,0 +1,227 @@
+/*
+ * sig.h — C ABI of libsig.so: the activation-sparse linear layer for LLM
+ * decoding on one NVIDIA B200 (sm_100a).
+ *
+ * The layer computes y = W (m . x): a mask m picks the entries of the
+ * activation x that survive, and the product reads only the weight columns of
+ * the surviving entries.  Sources, by page title and section:
+ *   - "Training-Free Activation Sparsity in Large Language Models" (TEAL
+ *     README), Abstract: magnitude threshold on the hidden states.
+ *   - "Q-Sparse: All Large Language Models can be Fully Sparsely-Activated"
+ *     (OpenReview rebuttal), A1 on MoE: top-k by magnitude per token; A2 on
+ *     batched inference: Block Q-Sparse with N:M activation sparsity; A3:
+ *     FLOPs of the product.
+ *   - "Adaptive Rank Allocation: Speeding Up Modern Transformers with RaNA
+ *     Adapters" (OpenReview rebuttal), Q3 Eqn. 12: the gated-MLP neuron
+ *     masker; Q5.1: the masked product skips the columns of zero mask entries.
+ *   - "Motivating Next-Gen Accelerators with Flexible (N:M) Activation
+ *     Sparsity ..." (summary), Methodology: N kept in every block of M.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer named WT, x, X, y, Y, h_out, mask_bits, idx, nnz, ws,
+ *     down_norms, norms, packed, X_masked is a DEVICE pointer.  The caller owns
+ *     every buffer; the library allocates nothing, keeps no pointer after the
+ *     call returns, and never synchronises the device.
+ *   - fp16 buffers hold IEEE binary16 bit patterns (uint16_t).
+ *   - Weights are stored transposed: WT is d_in x d_out, row-major, so row i
+ *     (2*d_out contiguous bytes) holds every weight that multiplies input i.
+ *   - Masks are bit-packed: bit (i % 32) of word (i / 32) is m_i.  2-D masks
+ *     pack each row on its own, rows padded to whole words.
+ *   - Index lists are int32, strictly ascending; the count lives on the device
+ *     (int32 *nnz), so no host round trip separates mask and product.
+ *   - Magnitude ranking (top-k, N:M): larger |x| first; equal |x| by lower
+ *     index first; +v/-v and +0/-0 tie; a NaN ranks below every number.
+ *   - All work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream).  Calls that share a workspace must not overlap on the device.
+ *   - Errors: arguments are checked on the host before anything is enqueued,
+ *     and a non-zero sig_status comes back with nothing launched.  A launch
+ *     failure returns SIG_ERR_CUDA.  Nothing throws across the ABI.
+ */
+#ifndef SIG_H
+#define SIG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported with default visibility; everything else in libsig.so is hidden. */
+#if defined(__GNUC__)
+#define SIG_API __attribute__((visibility("default")))
+#else
+#define SIG_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* sig_stream_t;
+
+typedef enum {
+  SIG_OK = 0,
+  SIG_ERR_NULL = 1,       /* a required pointer is NULL                        */
+  SIG_ERR_SHAPE = 2,      /* a size is out of range or inconsistent            */
+  SIG_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned where required   */
+  SIG_ERR_WORKSPACE = 4,  /* workspace NULL or smaller than sig_workspace_bytes */
+  SIG_ERR_CUDA = 5,       /* the CUDA runtime reported an error                */
+  SIG_ERR_TIMEOUT = 6,    /* a bounded device-side wait gave up                */
+  SIG_ERR_ARG = 7         /* another argument is out of range (k, n, m, op)    */
+} sig_status;
+
+/* Operation codes for sig_workspace_bytes. */
+typedef enum {
+  SIG_OP_SPARSE_GEMV = 1,  /* sparse_gemv(d_in, d_out)                 */
+  SIG_OP_TOPK = 2,         /* sparsify_topk(d = d_in)                  */
+  SIG_OP_GATED_MLP = 3,    /* gated_mlp_sparse(d_model = d_in, d_ff = d_out) */
+  SIG_OP_NM_GEMM = 4       /* nm_act_gemm(K = d_in, N = d_out, rows)   */
+} sig_op;
+
+/* Largest activation length the fused mask prologue accepts. */
+#define SIG_MAX_D_IN 131072
+
+/* Human-readable name of a status code (static storage, never NULL). */
+SIG_API const char* sig_status_string(int status);
+
+/* ABI version of this header; bumps when a signature changes. */
+SIG_API int sig_abi_version(void);
+
+/*
+ * Bytes of device workspace an operation needs for the given sizes (0 when
+ * the operation needs none).  Returns 0 and sets nothing for an unknown op.
+ * The workspace holds split-K partial sums and per-tile arrival counters.
+ */
+SIG_API size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows);
+
+/*
+ * Zero a workspace once before its first use (asynchronously on `stream`).
+ * Every operation leaves its counters at zero again when it completes, so a
+ * workspace needs this only once after allocation.  ws must be 256-byte
+ * aligned.
+ */
+SIG_API int sig_workspace_init(void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * Threshold mask (TEAL README, Abstract; comparison ">= t" as in RaNA
+ * Eqn. 12):  m_i = |x_i| >= t, compared in float32 (exact for fp16 x).
+ *   x          [d] fp16, 16-byte aligned.
+ *   t          threshold (float).  A NaN in x is never kept.
+ *   mask_bits  [ceil(d/32)] uint32 out.
+ *   idx        [d] int32 out, nullable: ascending kept indices (first *nnz valid).
+ *   nnz        [1] int32 out, nullable: number of kept entries.
+ * Errors: SIG_ERR_NULL (x or mask_bits), SIG_ERR_SHAPE (d < 1 or d > SIG_MAX_D_IN),
+ *         SIG_ERR_ALIGN (x).
+ */
+SIG_API int sparsify_threshold(const uint16_t* x, int64_t d, float t,
+                       uint32_t* mask_bits, int32_t* idx, int32_t* nnz,
+                       sig_stream_t stream);
+
+/*
+ * Top-k mask (Q-Sparse rebuttal, A1 on MoE): keep the k entries of largest
+ * |x|, ties by lower index; exactly k bits are set.  Selection runs on the
+ * 15-bit magnitude code of fp16, so no float comparison decides it.
+ *   x          [d] fp16, 16-byte aligned.
+ *   k          0 <= k <= d.
+ *   mask_bits  [ceil(d/32)] uint32 out.   idx [d] int32 out (first k valid).
+ *   nnz        [1] int32 out (= k).
+ *   ws         sig_workspace_bytes(SIG_OP_TOPK, d, 0, 0) bytes (may be 0 → ws may be NULL).
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d < 1 or d > SIG_MAX_D_IN), SIG_ERR_ARG (k),
+ *         SIG_ERR_ALIGN, SIG_ERR_WORKSPACE.
+ */
+SIG_API int sparsify_topk(const uint16_t* x, int64_t d, int64_t k,
+                  uint32_t* mask_bits, int32_t* idx, int32_t* nnz,
+                  void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * N:M activation mask (N:M summary, Methodology; Block Q-Sparse in the
+ * Q-Sparse rebuttal, A2): for every row of X and every block of m consecutive
+ * entries, keep the n of largest |x| (ties by lower index).
+ *   X          [rows x d] fp16 row-major, 16-byte aligned.
+ *   n, m       1 <= n <= m <= 32, d % m == 0.
+ *   X_masked   [rows x d] fp16 out, nullable: X with dropped entries set to +0.
+ *   mask_bits  [rows x ceil(d/32)] uint32 out, nullable.
+ * At least one of X_masked and mask_bits must be non-NULL.  rows == 0 is an
+ * empty batch: the call returns SIG_OK and touches no pointer.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (rows < 0, d < 1, d % m), SIG_ERR_ARG (n, m),
+ *         SIG_ERR_ALIGN.
+ */
+SIG_API int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m,
+                uint16_t* X_masked, uint32_t* mask_bits, sig_stream_t stream);
+
+/*
+ * Sparse-input GEMV y = W (m . x) (RaNA rebuttal, Q5.1; Q-Sparse A3):
+ *   y_j = sum over kept i of WT[i, j] * x_i, accumulated in float32 and
+ *   rounded once to fp16.  Only the kept rows of WT are read.
+ * Mask source:
+ *   idx == NULL: fused threshold |x_i| >= t, computed inside the same launch.
+ *   idx != NULL: the rows idx[0 .. *nnz) from a sparsify_* call; t is ignored.
+ *                Entries outside [0, d_in) are skipped; *nnz is clamped to [0, d_in].
+ *   WT   [d_in x d_out] fp16 row-major, 16-byte aligned, d_out % 8 == 0.
+ *   x    [d_in] fp16, 16-byte aligned.       y [d_out] fp16 out, 16-byte aligned.
+ *   ws   sig_workspace_bytes(SIG_OP_SPARSE_GEMV, d_in, d_out, 0) bytes, 256-byte
+ *        aligned, zeroed once by sig_workspace_init (or allocated zeroed).
+ * The result is bit-identical from run to run (fixed-order split-K reduction;
+ * no floating-point atomics).  An empty mask writes y = 0.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d_in < 1, d_in > SIG_MAX_D_IN, d_out < 8,
+ *         d_out % 8), SIG_ERR_ALIGN, SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
+ */
+SIG_API int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out,
+                const uint16_t* x, float t, const int32_t* idx, const int32_t* nnz,
+                uint16_t* y, void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * Gated MLP with the RaNA neuron masker (RaNA rebuttal, Q3, Eqn. 12):
+ *   g = GateProj(x), u = UpProj(x)       (dense GEMVs, float32 accumulation)
+ *   h = fp16(SiLU(g) * u)                (SiLU(z) = z / (1 + exp(-z)), float32)
+ *   m_i = float32(|h_i|) * down_norms[i] >= t      (one float32 multiply)
+ *   y = W_down (m . h)                   (sparse GEMV as in sparse_gemv)
+ *   x        [d_model] fp16.   WgT, WuT [d_model x d_ff] fp16.   WdT [d_ff x d_model] fp16.
+ *   down_norms [d_ff] float32: ||row i of WdT||_2 (see sig_row_norms).
+ *   y        [d_model] fp16 out.  h_out [d_ff] fp16 out, nullable.
+ *   mask_out [ceil(d_ff/32)] uint32 out, nullable.
+ *   ws       sig_workspace_bytes(SIG_OP_GATED_MLP, d_model, d_ff, 0) bytes.
+ * d_model % 8 == 0, d_ff % 8 == 0, d_model and d_ff <= SIG_MAX_D_IN.
+ * Errors: as sparse_gemv.
+ */
+SIG_API int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                     const uint16_t* WdT, const float* down_norms,
+                     int64_t d_model, int64_t d_ff, float t,
+                     uint16_t* y, uint16_t* h_out, uint32_t* mask_out,
+                     void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * l2 norm of every row of a row-major fp16 matrix, accumulated in float64 and
+ * rounded once to float32.  For WdT it yields the ||W^down_i|| of RaNA Eqn. 12.
+ *   WT [rows x cols] fp16 (16-byte aligned, cols % 8 == 0).  norms [rows] float32 out.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ALIGN.
+ */
+SIG_API int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float* norms,
+                  sig_stream_t stream);
+
+/*
+ * Batched N:M activation GEMM (Block Q-Sparse, Q-Sparse rebuttal A2):
+ *   Y = (M . X) WT, M the per-row n:m mask of X (as sparsify_nm), float32
+ *   accumulation on the tensor cores, Y rounded once to fp16.
+ *   X  [rows x K] fp16 row-major.   WT [K x N] fp16 row-major.   Y [rows x N] fp16 out.
+ *   rows % 128 == 0, K % 64 == 0, N % 128 == 0, K % m == 0; 1 <= n <= m <= 32.
+ *   ws sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows) bytes (holds the masked X).
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ARG, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE,
+ *         SIG_ERR_CUDA.
+ */
+SIG_API int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT,
+                int64_t N, int n, int m, uint16_t* Y, void* ws, size_t ws_bytes,
+                sig_stream_t stream);
+
+/*
+ * Read and clear the library's device error word (no counterpart on the
+ * pages; it reports the bounded waits of the tensor-core GEMM).  Synchronises
+ * `stream`.  *code receives 0 when no kernel gave up on a wait, else a
+ * non-zero bit set; the call then returns SIG_ERR_TIMEOUT.
+ * Errors: SIG_ERR_NULL (code), SIG_ERR_CUDA.
+ */
+SIG_API int sig_take_device_error(unsigned* code, sig_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIG_H */

@@ -1,0 +1,235 @@
+"""Python binding of libsig.so, the activation-sparse linear layer for B200.
+
+Argument marshalling only: every function checks dtypes and devices, takes
+``data_ptr()`` of the torch tensors and the current CUDA stream, and calls the
+C ABI declared in ``include/sig.h``.  Every step of the computation runs in the
+library's CUDA kernels; there is no other implementation behind these calls.
+Importing this module fails loudly when ``libsig.so`` has not been built.
+
+fp16 tensors are ``torch.float16``; masks are ``torch.int32`` tensors holding
+the uint32 bit words (bit i % 32 of word i // 32); index lists are int32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "SigError", "OP_SPARSE_GEMV", "OP_TOPK", "OP_GATED_MLP", "OP_NM_GEMM",
+    "MAX_D_IN", "abi_version", "workspace_bytes", "workspace", "sparsify_threshold",
+    "sparsify_topk", "sparsify_nm", "sparse_gemv", "gated_mlp_sparse", "row_norms",
+    "nm_act_gemm", "take_device_error", "status_string",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
+
+OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM = 1, 2, 3, 4
+MAX_D_IN = 131072
+
+_p, _i64, _i32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                             ctypes.c_float, ctypes.c_size_t)
+
+_SIGNATURES = {
+    "sig_status_string": (ctypes.c_char_p, [_i32]),
+    "sig_abi_version": (_i32, []),
+    "sig_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64]),
+    "sig_workspace_init": (_i32, [_p, _sz, _p]),
+    "sparsify_threshold": (_i32, [_p, _i64, _f32, _p, _p, _p, _p]),
+    "sparsify_topk": (_i32, [_p, _i64, _i64, _p, _p, _p, _p, _sz, _p]),
+    "sparsify_nm": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _p]),
+    "sparse_gemv": (_i32, [_p, _i64, _i64, _p, _f32, _p, _p, _p, _p, _sz, _p]),
+    "gated_mlp_sparse": (_i32, [_p, _p, _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
+    "sig_row_norms": (_i32, [_p, _i64, _i64, _p, _p]),
+    "nm_act_gemm": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _sz, _p]),
+    "sig_take_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _p]),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python sparse_input_gemv_threshold_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+_lib = _load()
+
+
+class SigError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def status_string(status: int) -> str:
+    return _lib.sig_status_string(status).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise SigError(fn, status)
+
+
+def abi_version() -> int:
+    return _lib.sig_abi_version()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, dtype, name, dev=None):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dev is not None and t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_bytes(op: int, d_in: int, d_out: int = 0, rows: int = 0) -> int:
+    return int(_lib.sig_workspace_bytes(op, d_in, d_out, rows))
+
+
+_ws_cache = {}
+_ws_lock = threading.Lock()
+
+
+def workspace(op: int, d_in: int, d_out: int = 0, rows: int = 0, device=None,
+              stream=None) -> torch.Tensor:
+    """A zeroed workspace for ``op`` at these sizes, cached per (device, stream).
+
+    The kernels return their counters to zero, so a cached workspace can be
+    reused by later calls on the same stream.  Calls on different streams get
+    different workspaces.
+    """
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    nbytes = workspace_bytes(op, d_in, d_out, rows)
+    key = (dev, _stream(stream), op, d_in, d_out, rows)
+    with _ws_lock:
+        ws = _ws_cache.get(key)
+        if ws is None:
+            ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+            _ws_cache[key] = ws
+    return ws
+
+
+def sparsify_threshold(x, t: float, mask_bits=None, idx=None, nnz=None, stream=None):
+    """Threshold mask |x_i| >= t.  Returns (mask_bits, idx, nnz) device tensors."""
+    _need(x, torch.float16, "x")
+    d = x.numel()
+    words = (d + 31) // 32
+    mask_bits = torch.empty(words, dtype=torch.int32, device=x.device) if mask_bits is None else mask_bits
+    idx = torch.empty(d, dtype=torch.int32, device=x.device) if idx is None else idx
+    nnz = torch.empty(1, dtype=torch.int32, device=x.device) if nnz is None else nnz
+    _check("sparsify_threshold", _lib.sparsify_threshold(
+        _ptr(x), d, float(t), _ptr(mask_bits), _ptr(idx), _ptr(nnz), _stream(stream)))
+    return mask_bits, idx, nnz
+
+
+def sparsify_topk(x, k: int, mask_bits=None, idx=None, nnz=None, stream=None):
+    """Top-k mask by |x| (ties by lower index).  Returns (mask_bits, idx, nnz)."""
+    _need(x, torch.float16, "x")
+    d = x.numel()
+    mask_bits = torch.empty((d + 31) // 32, dtype=torch.int32, device=x.device) if mask_bits is None else mask_bits
+    idx = torch.empty(d, dtype=torch.int32, device=x.device) if idx is None else idx
+    nnz = torch.empty(1, dtype=torch.int32, device=x.device) if nnz is None else nnz
+    _check("sparsify_topk", _lib.sparsify_topk(
+        _ptr(x), d, int(k), _ptr(mask_bits), _ptr(idx), _ptr(nnz), None, 0, _stream(stream)))
+    return mask_bits, idx, nnz
+
+
+def sparsify_nm(X, n: int, m: int, X_masked=None, mask_bits=None, want_masked=True,
+                want_bits=True, stream=None):
+    """Per-row N:M mask of a 2-D fp16 ``X``.  Returns (X_masked, mask_bits)."""
+    _need(X, torch.float16, "X")
+    rows, d = X.shape
+    if want_masked and X_masked is None:
+        X_masked = torch.empty_like(X)
+    if want_bits and mask_bits is None:
+        mask_bits = torch.empty((rows, (d + 31) // 32), dtype=torch.int32, device=X.device)
+    _check("sparsify_nm", _lib.sparsify_nm(
+        _ptr(X), rows, d, int(n), int(m), _ptr(X_masked), _ptr(mask_bits), _stream(stream)))
+    return X_masked, mask_bits
+
+
+def sparse_gemv(WT, x, t: float = 0.0, idx=None, nnz=None, y=None, ws=None, stream=None):
+    """y = W (m . x) with WT (d_in, d_out) fp16.  idx/nnz select rows; else |x| >= t."""
+    _need(WT, torch.float16, "WT")
+    _need(x, torch.float16, "x", WT.device)
+    d_in, d_out = WT.shape
+    if x.numel() != d_in:
+        raise ValueError("x length must equal WT.shape[0]")
+    if y is None:
+        y = torch.empty(d_out, dtype=torch.float16, device=WT.device)
+    if ws is None:
+        ws = workspace(OP_SPARSE_GEMV, d_in, d_out, device=WT.device, stream=stream)
+    _check("sparse_gemv", _lib.sparse_gemv(
+        _ptr(WT), d_in, d_out, _ptr(x), float(t), _ptr(idx), _ptr(nnz), _ptr(y),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
+                     mask_out=None, ws=None, stream=None):
+    """RaNA gated MLP (Eqn. 12 masker then sparse down projection).  Returns y."""
+    for name, w in (("WgT", WgT), ("WuT", WuT), ("WdT", WdT), ("x", x)):
+        _need(w, torch.float16, name, x.device)
+    _need(down_norms, torch.float32, "down_norms", x.device)
+    d_model, d_ff = WgT.shape
+    if y is None:
+        y = torch.empty(d_model, dtype=torch.float16, device=x.device)
+    if ws is None:
+        ws = workspace(OP_GATED_MLP, d_model, d_ff, device=x.device, stream=stream)
+    _check("gated_mlp_sparse", _lib.gated_mlp_sparse(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
+        _ptr(y), _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def row_norms(WT, out=None, stream=None):
+    """float32 l2 norm of every row of a 2-D fp16 matrix (float64 accumulation)."""
+    _need(WT, torch.float16, "WT")
+    rows, cols = WT.shape
+    out = torch.empty(rows, dtype=torch.float32, device=WT.device) if out is None else out
+    _check("sig_row_norms", _lib.sig_row_norms(_ptr(WT), rows, cols, _ptr(out), _stream(stream)))
+    return out
+
+
+def nm_act_gemm(X, WT, n: int, m: int, Y=None, ws=None, stream=None):
+    """Y = (M . X) WT with M the per-row n:m mask of X, on the tensor cores."""
+    _need(X, torch.float16, "X")
+    _need(WT, torch.float16, "WT", X.device)
+    rows, K = X.shape
+    N = WT.shape[1]
+    if Y is None:
+        Y = torch.empty((rows, N), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(OP_NM_GEMM, K, N, rows, device=X.device, stream=stream)
+    _check("nm_act_gemm", _lib.nm_act_gemm(
+        _ptr(X), rows, K, _ptr(WT), N, int(n), int(m), _ptr(Y), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return Y
+
+
+def take_device_error(stream=None) -> int:
+    """Read and clear the device error word (0 = no kernel gave up on a wait)."""
+    code = ctypes.c_uint(0)
+    st = _lib.sig_take_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (0, 6):
+        raise SigError("sig_take_device_error", st)
+    return int(code.value)

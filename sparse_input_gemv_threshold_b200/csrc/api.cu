@@ -1,0 +1,207 @@
+// C ABI of libsig.so (declared in include/sig.h).  Every entry point checks its
+// arguments on the host and returns a status without launching anything when
+// a check fails; otherwise it enqueues its kernels on the caller's stream and
+// returns at once.
+#include "../../include/sig.h"
+#include "internal.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+using namespace sig;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SIG_OK : SIG_ERR_CUDA; }
+
+int check_gemv_shape(int64_t d_in, int64_t d_out) {
+  if (d_in < 1 || d_in > kMaxDIn) return SIG_ERR_SHAPE;
+  if (d_out < 8 || d_out % 8 != 0 || d_out > (int64_t)1 << 30) return SIG_ERR_SHAPE;
+  if (d_in * d_out > ((int64_t)1 << 40)) return SIG_ERR_SHAPE;
+  return SIG_OK;
+}
+
+struct GatedPlan {
+  GemvPlan up, down;
+  size_t off_down, off_h, total;
+};
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+GatedPlan plan_gated(int64_t d_model, int64_t d_ff) {
+  GatedPlan g;
+  g.up = plan_gemv(d_model, d_ff, true);
+  g.down = plan_gemv(d_ff, d_model, false);
+  g.off_down = round_up(g.up.ws_bytes(), 256);
+  g.off_h = g.off_down + round_up(g.down.ws_bytes(), 256);
+  g.total = g.off_h + round_up((size_t)d_ff * 2, 256);
+  return g;
+}
+
+bool nm_pattern_ok(int n, int m) {
+  const bool pow2 = m == 1 || m == 2 || m == 4 || m == 8 || m == 16 || m == 32;
+  return pow2 && n >= 1 && n <= m;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sig_status_string(int status) {
+  switch (status) {
+    case SIG_OK: return "ok";
+    case SIG_ERR_NULL: return "a required pointer is NULL";
+    case SIG_ERR_SHAPE: return "a size is out of range or inconsistent";
+    case SIG_ERR_ALIGN: return "a pointer is not aligned as required";
+    case SIG_ERR_WORKSPACE: return "workspace missing or too small";
+    case SIG_ERR_CUDA: return "CUDA runtime error";
+    case SIG_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case SIG_ERR_ARG: return "an argument is out of range";
+  }
+  return "unknown status";
+}
+
+int sig_abi_version(void) { return 1; }
+
+size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
+  switch (op) {
+    case SIG_OP_SPARSE_GEMV:
+      if (check_gemv_shape(d_in, d_out) != SIG_OK) return 0;
+      return plan_gemv(d_in, d_out, false).ws_bytes();
+    case SIG_OP_TOPK:
+      return 0;
+    case SIG_OP_GATED_MLP:
+      if (check_gemv_shape(d_in, d_out) != SIG_OK || check_gemv_shape(d_out, d_in) != SIG_OK)
+        return 0;
+      return plan_gated(d_in, d_out).total;
+    case SIG_OP_NM_GEMM:
+      if (rows < 1 || d_in < 1) return 0;
+      return round_up((size_t)rows * (size_t)d_in * 2, 256);
+  }
+  return 0;
+}
+
+int sig_workspace_init(void* ws, size_t ws_bytes, sig_stream_t stream) {
+  if (ws_bytes == 0) return SIG_OK;
+  if (ws == nullptr) return SIG_ERR_NULL;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+int sparsify_threshold(const uint16_t* x, int64_t d, float t, uint32_t* mask_bits, int32_t* idx,
+                       int32_t* nnz, sig_stream_t stream) {
+  if (x == nullptr || mask_bits == nullptr) return SIG_ERR_NULL;
+  if (d < 1 || d > kMaxDIn) return SIG_ERR_SHAPE;
+  if (!aligned16(x)) return SIG_ERR_ALIGN;
+  return cuda_status(launch_threshold_compact(x, (int)d, t, mask_bits, idx, nnz,
+                                              (cudaStream_t)stream));
+}
+
+int sparsify_topk(const uint16_t* x, int64_t d, int64_t k, uint32_t* mask_bits, int32_t* idx,
+                  int32_t* nnz, void* ws, size_t ws_bytes, sig_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (x == nullptr || mask_bits == nullptr || idx == nullptr || nnz == nullptr)
+    return SIG_ERR_NULL;
+  if (d < 1 || d > kMaxDIn) return SIG_ERR_SHAPE;
+  if (k < 0 || k > d) return SIG_ERR_ARG;
+  if (!aligned16(x)) return SIG_ERR_ALIGN;
+  return cuda_status(launch_topk(x, (int)d, (int)k, mask_bits, idx, nnz, (cudaStream_t)stream));
+}
+
+int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m, uint16_t* X_masked,
+                uint32_t* mask_bits, sig_stream_t stream) {
+  if (!nm_pattern_ok(n, m)) return SIG_ERR_ARG;
+  if (rows < 0 || d < 1 || d % m != 0 || d > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
+  if (rows == 0) return SIG_OK;  // an empty batch: nothing to read or write
+  if (X == nullptr || (X_masked == nullptr && mask_bits == nullptr)) return SIG_ERR_NULL;
+  if (d % 8 != 0 || !aligned16(X) || (X_masked != nullptr && !aligned16(X_masked)))
+    return SIG_ERR_ALIGN;
+  return cuda_status(launch_nm_mask(X, rows, (int)d, n, m, X_masked, mask_bits,
+                                    (cudaStream_t)stream));
+}
+
+int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t* x, float t,
+                const int32_t* idx, const int32_t* nnz, uint16_t* y, void* ws, size_t ws_bytes,
+                sig_stream_t stream) {
+  if (WT == nullptr || x == nullptr || y == nullptr) return SIG_ERR_NULL;
+  if (idx != nullptr && nnz == nullptr) return SIG_ERR_NULL;
+  const int sh = check_gemv_shape(d_in, d_out);
+  if (sh != SIG_OK) return sh;
+  if (!aligned16(WT) || !aligned16(x) || !aligned16(y)) return SIG_ERR_ALIGN;
+  const GemvPlan p = plan_gemv(d_in, d_out, false);
+  if (ws == nullptr || ws_bytes < p.ws_bytes()) return SIG_ERR_WORKSPACE;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  GemvLaunch a{};
+  a.WT = WT; a.x = x; a.t = t; a.idx = idx; a.nnz = nnz;
+  a.d_in = (int)d_in; a.d_out = (int)d_out; a.y = y; a.ws = ws;
+  return cuda_status(launch_gemv(idx == nullptr ? MASK_THRESH : MASK_IDX, EPI_STORE, p, a,
+                                 (cudaStream_t)stream));
+}
+
+int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                     const uint16_t* WdT, const float* down_norms, int64_t d_model, int64_t d_ff,
+                     float t, uint16_t* y, uint16_t* h_out, uint32_t* mask_out, void* ws,
+                     size_t ws_bytes, sig_stream_t stream) {
+  if (x == nullptr || WgT == nullptr || WuT == nullptr || WdT == nullptr ||
+      down_norms == nullptr || y == nullptr)
+    return SIG_ERR_NULL;
+  int sh = check_gemv_shape(d_model, d_ff);
+  if (sh == SIG_OK) sh = check_gemv_shape(d_ff, d_model);
+  if (sh != SIG_OK) return sh;
+  if (!aligned16(x) || !aligned16(WgT) || !aligned16(WuT) || !aligned16(WdT) || !aligned16(y) ||
+      (h_out != nullptr && !aligned16(h_out)))
+    return SIG_ERR_ALIGN;
+  const GatedPlan g = plan_gated(d_model, d_ff);
+  if (ws == nullptr || ws_bytes < g.total) return SIG_ERR_WORKSPACE;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  char* base = reinterpret_cast<char*>(ws);
+  uint16_t* h = h_out != nullptr ? h_out : reinterpret_cast<uint16_t*>(base + g.off_h);
+
+  GemvLaunch up{};
+  up.WT = WgT; up.WT2 = WuT; up.x = x; up.d_in = (int)d_model; up.d_out = (int)d_ff;
+  up.y = h; up.ws = base;
+  cudaError_t e = launch_gemv(MASK_DENSE, EPI_SILU_MUL, g.up, up, (cudaStream_t)stream);
+  if (e != cudaSuccess) return SIG_ERR_CUDA;
+
+  GemvLaunch dn{};
+  dn.WT = WdT; dn.x = h; dn.scale = down_norms; dn.t = t; dn.d_in = (int)d_ff;
+  dn.d_out = (int)d_model; dn.y = y; dn.mask_out = mask_out; dn.ws = base + g.off_down;
+  return cuda_status(launch_gemv(MASK_THRESH_SCALED, EPI_STORE, g.down, dn, (cudaStream_t)stream));
+}
+
+int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float* norms,
+                  sig_stream_t stream) {
+  if (WT == nullptr || norms == nullptr) return SIG_ERR_NULL;
+  if (rows < 0 || cols < 8 || cols % 8 != 0 || cols > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
+  if (!aligned16(WT)) return SIG_ERR_ALIGN;
+  return cuda_status(launch_row_norms(WT, rows, (int)cols, norms, (cudaStream_t)stream));
+}
+
+int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT, int64_t N, int n,
+                int m, uint16_t* Y, void* ws, size_t ws_bytes, sig_stream_t stream) {
+  if (X == nullptr || WT == nullptr || Y == nullptr) return SIG_ERR_NULL;
+  if (!nm_pattern_ok(n, m)) return SIG_ERR_ARG;
+  if (rows < 128 || rows % 128 != 0 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0 ||
+      K % m != 0 || rows > (1 << 24) || K > (1 << 20) || N > (1 << 20))
+    return SIG_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(WT) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  const size_t need = sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows);
+  if (ws == nullptr || ws_bytes < need) return SIG_ERR_WORKSPACE;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  uint16_t* Xm = reinterpret_cast<uint16_t*>(ws);
+  cudaError_t e = launch_nm_mask(X, rows, (int)K, n, m, Xm, nullptr, (cudaStream_t)stream);
+  if (e != cudaSuccess) return SIG_ERR_CUDA;
+  return cuda_status(launch_gemm_f16(Xm, WT, Y, (int)rows, (int)N, (int)K, (cudaStream_t)stream));
+}
+
+int sig_take_device_error(unsigned* code, sig_stream_t stream) {
+  if (code == nullptr) return SIG_ERR_NULL;
+  if (read_device_error(code, (cudaStream_t)stream) != cudaSuccess) return SIG_ERR_CUDA;
+  return *code == 0u ? SIG_OK : SIG_ERR_TIMEOUT;
+}
+
+}  // extern "C"

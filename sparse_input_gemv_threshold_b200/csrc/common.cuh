@@ -1,0 +1,111 @@
+// Device helpers shared by the libsig kernels (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace sig {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// 16-byte streaming load of weights: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float h2f(uint16_t bits) {
+  return __half2float(__ushort_as_half(bits));
+}
+
+__device__ __forceinline__ uint16_t f2h_rn(float v) {
+  return __half_as_ushort(__float2half_rn(v));
+}
+
+// acc[k] += w[k] * xv for the eight fp16 weights packed in `v`, float32 FMA.
+__device__ __forceinline__ void fma8(float (&acc)[8], const uint4& v, float xv) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+    acc[2 * k] = fmaf(f.x, xv, acc[2 * k]);
+    acc[2 * k + 1] = fmaf(f.y, xv, acc[2 * k + 1]);
+  }
+}
+
+// fp16 element k (0..7) of a 16-byte vector.
+__device__ __forceinline__ uint16_t lane_half(const uint4& v, int k) {
+  const uint32_t w = (k < 2) ? v.x : (k < 4) ? v.y : (k < 6) ? v.z : v.w;
+  return static_cast<uint16_t>((k & 1) ? (w >> 16) : (w & 0xffffu));
+}
+
+// Magnitude rank key of an fp16 value: 0 for NaN, 1 + (|x| bits) otherwise,
+// so that a larger key means a larger magnitude and NaN ranks lowest.
+__device__ __forceinline__ uint32_t mag_key(uint16_t bits) {
+  const uint32_t a = bits & 0x7fffu;
+  return a > 0x7c00u ? 0u : a + 1u;
+}
+
+// Exclusive prefix sum over a block of BLOCK threads.  `scratch` holds
+// BLOCK/32 ints.  Returns the exclusive prefix; *total receives the sum.
+template <int BLOCK>
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
+  constexpr int kWarps = BLOCK / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kWarps ? scratch[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, wi, o);
+      if (lane >= o) wi += n;
+    }
+    if (lane < kWarps) scratch[lane] = wi - w;  // exclusive warp offsets
+    if (lane == kWarps - 1) scratch[kWarps] = wi;
+  }
+  __syncthreads();
+  const int out = scratch[warp] + incl - v;
+  *total = scratch[kWarps];
+  __syncthreads();
+  return out;
+}
+
+// Build the bit-packed mask of `d` entries into shared `words`
+// (bit i%32 of word i/32) from a per-element predicate, reading the fp16
+// vector x 16 bytes per thread.  Every thread of the block must call it.
+template <int BLOCK, typename Pred>
+__device__ __forceinline__ void build_mask_words(const uint16_t* __restrict__ x, int d,
+                                                 uint32_t* words, Pred pred) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int nwords = (d + 31) >> 5;
+  for (int base = 0; base < d; base += BLOCK * 8) {
+    const int e0 = base + tid * 8;
+    uint32_t b = 0;
+    if (e0 + 8 <= d) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + e0));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) b |= (pred(lane_half(v, k), e0 + k) ? 1u : 0u) << k;
+    } else {
+      for (int k = 0; k < 8; ++k)
+        if (e0 + k < d) b |= (pred(x[e0 + k], e0 + k) ? 1u : 0u) << k;
+    }
+    uint32_t w = b << (8 * (lane & 3));
+    w |= __shfl_xor_sync(kFull, w, 1);
+    w |= __shfl_xor_sync(kFull, w, 2);
+    const int wi = (base >> 5) + (tid >> 2);
+    if ((lane & 3) == 0 && wi < nwords) words[wi] = w;
+  }
+}
+
+}  // namespace sig

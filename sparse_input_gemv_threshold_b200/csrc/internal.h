@@ -1,0 +1,77 @@
+// Internal host-side interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sig {
+
+constexpr int kNumSMs = 148;         // B200: 2 dies x 74 SMs
+constexpr int kGemvThreads = 256;    // 8 warps
+constexpr int kGemvTile = 256;       // output columns per CTA (one warp spans them)
+constexpr int kGemvCtasPerSM = 4;    // target residency; grid = C x S <= 148 * 4
+constexpr int kIdxCap = 4096;        // largest slice of the index list per CTA
+constexpr int kMaxDIn = 131072;
+
+// How the rows of a sparse GEMV are chosen.
+enum MaskMode : int {
+  MASK_THRESH = 0,         // |x_i| >= t, computed in the prologue
+  MASK_THRESH_SCALED = 1,  // |x_i| * scale_i >= t (RaNA Eqn. 12 with scale = norms)
+  MASK_IDX = 2,            // rows idx[0 .. *nnz) given by the caller
+  MASK_DENSE = 3           // every row
+};
+
+// What happens to a finished output column.
+enum Epilogue : int {
+  EPI_STORE = 0,     // y_j = fp16(sum)
+  EPI_SILU_MUL = 1   // dual product (g, u): h_j = fp16(SiLU(g_j) * u_j)
+};
+
+struct GemvPlan {
+  int C;              // column tiles
+  int S;              // K-splits (slices of the kept-row list)
+  int cap;            // most rows one slice can hold
+  size_t smem;        // dynamic shared memory per CTA
+  size_t counters;    // workspace bytes for arrival counters
+  size_t partials;    // workspace bytes for float32 partial sums
+  size_t ws_bytes() const { return counters + partials; }
+};
+
+GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual);
+
+struct GemvLaunch {
+  const uint16_t* WT;
+  const uint16_t* WT2;     // second weight for the dual (gate, up) product
+  const uint16_t* x;
+  const float* scale;      // MASK_THRESH_SCALED
+  const int32_t* idx;      // MASK_IDX
+  const int32_t* nnz;      // MASK_IDX
+  float t;
+  int d_in, d_out;
+  uint16_t* y;             // output (y, or h for EPI_SILU_MUL)
+  uint32_t* mask_out;      // nullable: written by one CTA
+  void* ws;                // plan.ws_bytes() bytes, counters zero on entry
+};
+
+cudaError_t launch_gemv(int mode, int epi, const GemvPlan& plan, const GemvLaunch& a,
+                        cudaStream_t stream);
+
+// Mask kernels (mask.cu).
+cudaError_t launch_threshold_compact(const uint16_t* x, int d, float t, uint32_t* mask_bits,
+                                     int32_t* idx, int32_t* nnz, cudaStream_t stream);
+cudaError_t launch_topk(const uint16_t* x, int d, int k, uint32_t* mask_bits, int32_t* idx,
+                        int32_t* nnz, cudaStream_t stream);
+cudaError_t launch_nm_mask(const uint16_t* X, int64_t rows, int d, int n, int m,
+                           uint16_t* X_masked, uint32_t* mask_bits, cudaStream_t stream);
+cudaError_t launch_row_norms(const uint16_t* WT, int64_t rows, int cols, float* norms,
+                             cudaStream_t stream);
+
+// Tensor-core GEMM (nm_gemm.cu): Y = A * B, A [M x K] fp16 row-major,
+// B given as WT [K x N] fp16 row-major, Y [M x N] fp16.
+cudaError_t read_device_error(unsigned* out, cudaStream_t stream);
+
+cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
+                            int K, cudaStream_t stream);
+
+}  // namespace sig

@@ -1,0 +1,329 @@
+// Tensor-core GEMM Y = A * B for the batched N:M activation product
+// (Block Q-Sparse, "Q-Sparse ..." rebuttal, A2).  A is the masked activation
+// block (tokens x K, K contiguous), B is the transposed weight WT (K x N,
+// N contiguous), Y is tokens x N in fp16 with float32 accumulation.
+//
+// sm_100a design: one CTA per 128 x BN output tile, 128 threads.
+//   - thread 0 streams 64-wide K slices of A and B into a 4-stage shared
+//     ring with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast),
+//     signalling an mbarrier with the transaction byte count;
+//   - thread 32 issues tcgen05.mma (kind::f16, M = 128, N = BN, K = 16) from
+//     shared-memory descriptors into a float32 accumulator in tensor memory
+//     and frees each stage with tcgen05.commit;
+//   - all four warps then read their 32 accumulator lanes with tcgen05.ld,
+//     round to fp16 and store.
+// Every mbarrier wait gives up after ~2 s of clock cycles: the kernel then
+// records SIG_ERR_TIMEOUT in a device error word, lets the copies it issued
+// land (again with a limit), frees its tensor memory and returns.
+#include "common.cuh"
+#include "internal.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace sig {
+
+__device__ unsigned g_device_error = 0u;
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;          // one 128-byte swizzle row of fp16
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr long long kTimeoutCycles = 4000000000ll;  // ~2 s at 1.9 GHz
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false after the time limit or once another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kTimeoutCycles) {
+      *abort_flag = 1;
+      atomicOr(&g_device_error, 1u);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start, leading and stride byte
+// offsets in 16-byte units, version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fffu);
+  d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3fffu) << 32;
+  d |= (uint64_t)1 << 46;        // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;        // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B, float32 D, A K-major,
+// B MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t instr_desc_f16(int M, int N) {
+  return (1u << 4)                       // D format: f32
+         | (0u << 7) | (0u << 10)        // A, B format: f16
+         | (0u << 15)                    // A K-major
+         | (1u << 16)                    // B MN-major
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int BN>
+struct __align__(1024) GemmSmem {
+  uint16_t A[kStages][kBM * kBK];   // 16 KB per stage, K-major, swizzled rows of 128 B
+  uint16_t B[kStages][kBK * BN];    // BN/64 blocks of 64 k-rows x 128 B
+  unsigned long long full[kStages];
+  unsigned long long empty[kStages];
+  unsigned long long accum;
+  uint32_t tmem_base;
+  int abort_flag;
+  int consumed;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                uint16_t* __restrict__ Y, int M, int N, int K) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the dynamic window starts 1024-aligned only by request; align by hand
+  GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+  const int kblocks = K / kBK;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 1);
+      mbar_init(smem_u32(&sm.empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm.accum), 1);
+    sm.abort_flag = 0;
+    sm.consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = sm.tmem_base;
+
+  constexpr uint32_t kStageBytes = (kBM * kBK + kBK * BN) * 2;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer ----
+      int issued = 0;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+        if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag)) break;
+        const uint32_t fb = smem_u32(&sm.full[s]);
+        mbar_expect_tx(fb, kStageBytes);
+        tma_load_2d(smem_u32(sm.A[s]), &mapA, kb * kBK, m0, fb);
+#pragma unroll
+        for (int j = 0; j < BN / 64; ++j)
+          tma_load_2d(smem_u32(sm.B[s]) + j * (kBK * 128), &mapB, n0 + j * 64, kb * kBK, fb);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let the copies already issued land before the CTA can exit
+        for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb) {
+          const long long t0 = clock64();
+          while (!mbar_try(smem_u32(&sm.full[kb % kStages]), (uint32_t)(kb / kStages) & 1u) &&
+                 clock64() - t0 < kTimeoutCycles) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer ----
+      constexpr uint32_t idesc = instr_desc_f16(kBM, BN);
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+        if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag)) break;
+        *(volatile int*)&sm.consumed = kb + 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          // A: K-major, advance 32 B inside the swizzled 128-B row.
+          const uint64_t da = smem_desc(a0 + k * 32, 16, 1024);
+          // B: MN-major, 16 k-rows = two 8-row groups (1024 B each) per step;
+          // 64-wide N blocks sit kBK*128 bytes apart.
+          const uint64_t db = smem_desc(b0 + k * 2048, kBK * 128, 1024);
+          const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "setp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+              "l"(da), "l"(db), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+        asm volatile(
+            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                smem_u32(&sm.empty[s]))
+            : "memory");
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(&sm.accum))
+          : "memory");
+    }
+    __syncwarp();
+  }
+
+  // ---- epilogue: TMEM -> registers -> fp16 -> global ----
+  const bool have_acc = mbar_wait(smem_u32(&sm.accum), 0u, abort_flag) && !*abort_flag;
+  __syncwarp();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (have_acc) {
+    const int row = m0 + warp * 32 + lane;
+    uint16_t* yrow = Y + (size_t)row * N + n0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c;
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+          "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+            "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+            "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+            "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+            "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+            "=r"(r[31])
+          : "r"(taddr));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      uint32_t p[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const __half2 h = __floats2half2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+        p[q] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D fp16 tensor map: inner extent `inner` (contiguous), outer extent
+// `outer`, row pitch `pitch_elems`, box 64 x box_outer, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t pitch_elems, uint32_t box_outer) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, uint16_t* Y, int M, int N,
+                      int K, cudaStream_t stream) {
+  const size_t smem = sizeof(GemmSmem<BN>) + 1024;
+  auto fn = gemm_f16_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(N / BN, M / kBM);
+  fn<<<grid, kThreads, smem, stream>>>(ma, mb, Y, M, N, K);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
+                            int K, cudaStream_t stream) {
+  if (M % kBM != 0 || K % kBK != 0 || N % 128 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kBK)) return cudaErrorInvalidValue;
+  if (N % 256 == 0) return launch_bn<256>(ma, mb, Y, M, N, K, stream);
+  return launch_bn<128>(ma, mb, Y, M, N, K, stream);
+}
+
+cudaError_t read_device_error(unsigned* out, cudaStream_t stream) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_device_error, sizeof(unsigned), 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  const unsigned zero = 0;
+  return cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(unsigned), 0,
+                                 cudaMemcpyHostToDevice, stream);
+}
+
+}  // namespace sig

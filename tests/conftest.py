@@ -15,5 +15,63 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: large shapes; several seconds of CPU work")
 
 
+def load_builder():
+    """The build script as a module, loaded by path (the package import would
+    load the library it builds)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "sig_build", os.path.join(ROOT, "sparse_input_gemv_threshold_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 def golden_path(name: str) -> str:
     return os.path.join(GOLDEN, name)
+
+
+# ---------------------------------------------------------------------------
+# GPU helpers (used only by tests marked gpu)
+# ---------------------------------------------------------------------------
+
+@pytest.fixture(scope="session")
+def sig():
+    """The product binding, built in-tree if needed.  Fails (never skips) when
+    the library or the GPU is missing: a gpu test must run the CUDA path."""
+    import torch
+    load_builder().build()
+    import sparse_input_gemv_threshold_b200 as mod
+    assert torch.cuda.is_available(), "gpu tests need a CUDA device"
+    return mod
+
+
+def to_dev(a):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def to_host(t):
+    return t.detach().cpu().numpy()
+
+
+def mask_words(t):
+    """Device int32 mask words -> numpy uint32."""
+    return to_host(t).view("uint32")
+
+
+def assert_within(y16, y64, bound, what=""):
+    """The benchmark spec tolerance per output: |y - y64| <= 2e-3 * sum|W x| (plus one
+    fp16 subnormal step, the finest spacing an fp16 result can have)."""
+    import numpy as np
+    y = np.asarray(y16, dtype=np.float16).astype(np.float64).ravel()
+    y64 = np.asarray(y64, dtype=np.float64).ravel()
+    bound = np.asarray(bound, dtype=np.float64).ravel()
+    err = np.abs(y - y64)
+    tol = 2e-3 * bound + 2.0 ** -24
+    bad = np.flatnonzero(err > tol)
+    if bad.size:
+        j = bad[np.argmax((err - tol)[bad])]
+        raise AssertionError(f"{what}: {bad.size}/{y.size} outputs out of tolerance; "
+                             f"worst j={j} y={y[j]} ref={y64[j]} bound={bound[j]}")
+    assert np.isfinite(y).all()

@@ -1,0 +1,141 @@
+"""Host-side tests of the C ABI: no GPU needed, no kernel is launched.
+
+Every call here fails argument validation, which runs on the host before any
+CUDA call, so the returned status is the whole behaviour under test.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT, load_builder
+
+HEADER = os.path.join(ROOT, "include", "sig.h")
+
+OK, NULL, SHAPE, ALIGN, WORKSPACE, CUDA, TIMEOUT, ARG = range(8)
+FAKE = 1 << 40            # an aligned, never dereferenced "device" address
+FAKE_ODD = FAKE + 2       # 2-byte aligned only
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = load_builder().build()
+    lib = ctypes.CDLL(path)
+    import sparse_input_gemv_threshold_b200 as sig  # noqa: F401  (sets argtypes on its own handle)
+    for name, (res, args) in sig._SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decl = re.findall(r"^SIG_API\s+(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", src, flags=re.M)
+    return sorted(set(decl))
+
+
+def test_header_declares_the_six_entry_points():
+    names = declared_functions()
+    for fn in ("sparsify_threshold", "sparsify_topk", "sparsify_nm", "sparse_gemv",
+               "gated_mlp_sparse", "nm_act_gemm"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+    # nothing else leaks out with default visibility except the ABI
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(ROOT, "sparse_input_gemv_threshold_b200", "libsig.so")],
+                         capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(names) <= exported
+
+
+def test_binding_covers_every_declared_symbol():
+    import sparse_input_gemv_threshold_b200 as sig
+    assert set(declared_functions()) <= set(sig._SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.sig_abi_version() == 1
+    for s in range(8):
+        assert lib.sig_status_string(s)
+    assert lib.sig_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    ws = lib.sig_workspace_bytes
+    assert ws(1, 4096, 4096, 0) > 0
+    assert ws(1, 4096, 4096, 0) % 256 == 0
+    assert ws(1, 0, 4096, 0) == 0            # invalid shape
+    assert ws(1, 4096, 12, 0) == 0           # d_out % 8
+    assert ws(2, 8192, 0, 0) == 0            # top-k needs none
+    assert ws(3, 4096, 11008, 0) > ws(1, 11008, 4096, 0)
+    assert ws(4, 1024, 1024, 4096) == 4096 * 1024 * 2
+    assert ws(77, 1, 1, 1) == 0
+
+
+def test_sparse_gemv_validation(lib):
+    f = lib.sparse_gemv
+    big = 1 << 30
+    assert f(None, 64, 64, FAKE, 0.0, None, None, FAKE, FAKE, big, None) == NULL
+    assert f(FAKE, 64, 64, FAKE, 0.0, FAKE, None, FAKE, FAKE, big, None) == NULL   # idx w/o nnz
+    assert f(FAKE, 0, 64, FAKE, 0.0, None, None, FAKE, FAKE, big, None) == SHAPE
+    assert f(FAKE, 131073, 64, FAKE, 0.0, None, None, FAKE, FAKE, big, None) == SHAPE
+    assert f(FAKE, 64, 60, FAKE, 0.0, None, None, FAKE, FAKE, big, None) == SHAPE
+    assert f(FAKE, 64, 0, FAKE, 0.0, None, None, FAKE, FAKE, big, None) == SHAPE
+    assert f(FAKE_ODD, 64, 64, FAKE, 0.0, None, None, FAKE, FAKE, big, None) == ALIGN
+    assert f(FAKE, 64, 64, FAKE_ODD, 0.0, None, None, FAKE, FAKE, big, None) == ALIGN
+    assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE_ODD, FAKE, big, None) == ALIGN
+    assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE, None, big, None) == WORKSPACE
+    need = lib.sig_workspace_bytes(1, 64, 64, 0)
+    assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE, FAKE, need - 1, None) == WORKSPACE
+    assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE, FAKE + 16, need, None) == ALIGN
+
+
+def test_mask_validation(lib):
+    assert lib.sparsify_threshold(None, 8, 0.0, FAKE, None, None, None) == NULL
+    assert lib.sparsify_threshold(FAKE, 8, 0.0, None, None, None, None) == NULL
+    assert lib.sparsify_threshold(FAKE, 0, 0.0, FAKE, None, None, None) == SHAPE
+    assert lib.sparsify_threshold(FAKE_ODD, 8, 0.0, FAKE, None, None, None) == ALIGN
+    t = lib.sparsify_topk
+    assert t(FAKE, 8, 9, FAKE, FAKE, FAKE, None, 0, None) == ARG
+    assert t(FAKE, 8, -1, FAKE, FAKE, FAKE, None, 0, None) == ARG
+    assert t(FAKE, 8, 2, FAKE, None, FAKE, None, 0, None) == NULL
+    assert t(FAKE, 0, 0, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
+    n = lib.sparsify_nm
+    assert n(FAKE, 4, 64, 3, 2, FAKE, FAKE, None) == ARG      # n > m
+    assert n(FAKE, 4, 64, 0, 4, FAKE, FAKE, None) == ARG      # n < 1
+    assert n(FAKE, 4, 60, 2, 3, FAKE, FAKE, None) == ARG      # m not a power of two
+    assert n(FAKE, 4, 36, 2, 8, FAKE, FAKE, None) == SHAPE    # m does not divide d
+    assert n(FAKE, 4, 64, 2, 4, None, None, None) == NULL     # no output requested
+    assert n(FAKE, -1, 64, 2, 4, FAKE, FAKE, None) == SHAPE
+    assert n(None, 0, 64, 2, 4, None, None, None) == OK          # empty batch
+
+
+def test_gated_and_gemm_validation(lib):
+    g = lib.gated_mlp_sparse
+    big = 1 << 30
+    assert g(FAKE, FAKE, FAKE, FAKE, None, 64, 128, 0.1, FAKE, None, None, FAKE, big, None) == NULL
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 124, 0.1, FAKE, None, None, FAKE, big, None) == SHAPE
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 0.1, FAKE, None, None, FAKE, 16, None) == WORKSPACE
+    assert g(FAKE, FAKE, FAKE_ODD, FAKE, FAKE, 64, 128, 0.1, FAKE, None, None, FAKE, big, None) == ALIGN
+    m = lib.nm_act_gemm
+    assert m(FAKE, 100, 1024, FAKE, 1024, 2, 4, FAKE, FAKE, big, None) == SHAPE    # rows % 128
+    assert m(FAKE, 256, 1000, FAKE, 1024, 2, 4, FAKE, FAKE, big, None) == SHAPE    # K % 64
+    assert m(FAKE, 256, 1024, FAKE, 1000, 2, 4, FAKE, FAKE, big, None) == SHAPE    # N % 128
+    assert m(FAKE, 256, 1024, FAKE, 1024, 5, 4, FAKE, FAKE, big, None) == ARG
+    assert m(FAKE, 256, 1024, FAKE, 1024, 2, 4, FAKE, FAKE, 10, None) == WORKSPACE
+    assert m(None, 256, 1024, FAKE, 1024, 2, 4, FAKE, FAKE, big, None) == NULL
+    r = lib.sig_row_norms
+    assert r(FAKE, 4, 12, FAKE, None) == SHAPE
+    assert r(FAKE, 4, 16, None, None) == NULL
+    assert lib.sig_take_device_error(None, None) == NULL
+    assert lib.sig_workspace_init(None, 16, None) == NULL
+    assert lib.sig_workspace_init(FAKE + 16, 16, None) == ALIGN
+    assert lib.sig_workspace_init(None, 0, None) == OK
