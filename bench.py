@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary rows")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--profile-case", default=None,
+                    help="for ncu: run only this kernel case eagerly and exit "
+                         "(a Llama-2-7B projection name at 50%%, 'topk70b', 'rana' or 'nm2:4')")
+    ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     return ap.parse_args()
 
 
@@ -169,19 +173,48 @@ def capture(fn, stream):
     return g
 
 
-def time_graphs(graphs, steps, warmup, stream, world=1):
-    """Replay graphs[i % len] for warmup then exactly `steps` timed steps."""
+class StepGraphs:
+    """CUDA graphs over a rotation of step callables.
+
+    `big` holds `per_graph` consecutive steps (step i uses fns[i % R]), so the
+    host pays one graph launch per `per_graph` steps; `singles` cover a
+    remainder, so that exactly the requested number of steps runs.
+    """
+
+    def __init__(self, fns, stream, per_graph):
+        import torch
+        self.fns, self.R = fns, len(fns)
+        self.per = max(self.R, (per_graph // self.R) * self.R)
+        with torch.cuda.stream(stream):
+            for f in fns:                      # one eager pass (kernel attributes)
+                f()
+        torch.cuda.synchronize()
+
+        def many():
+            for i in range(self.per):
+                fns[i % self.R]()
+        self.big = capture(many, stream)
+        self.singles = [capture(f, stream) for f in fns]
+
+    def run(self, n):
+        q, r = divmod(n, self.per)
+        for _ in range(q):
+            self.big.replay()
+        for i in range(r):
+            self.singles[i % self.R].replay()
+
+
+def time_steps(sg, steps, warmup, stream, world=1):
+    """Warm up, then time exactly `steps` steps with CUDA events on `stream`."""
     import torch
     with torch.cuda.stream(stream):
-        for i in range(warmup):
-            graphs[i % len(graphs)].replay()
+        sg.run(warmup)
     barrier(world)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         start.record(stream)
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        sg.run(steps)
         end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -274,18 +307,14 @@ def run_ours(args, rank, world, local):
         return f
 
     def graphs_for(s):
-        with torch.cuda.stream(stream):
-            for c in range(N_COPIES):        # one eager pass (sets kernel attributes)
-                step_fn(c, s)()
-        torch.cuda.synchronize()
-        return [capture(step_fn(c, s), stream) for c in range(N_COPIES)]
+        return StepGraphs([step_fn(c, s) for c in range(N_COPIES)], stream, per_graph=12)
 
     # ---- headline ----
     g50 = graphs_for(HEADLINE_SPARSITY)
     nnz50 = kept_counts(projs, HEADLINE_SPARSITY)
     bytes_step = algorithmic_bytes(projs, nnz50)
     with ClockSampler(local) as clk:
-        secs = time_graphs(g50, args.steps, args.warmup, stream, world)
+        secs = time_steps(g50, args.steps, args.warmup, stream, world)
     clocks = clk.summary()
     slow = max_over_ranks(secs, world)
     value = bytes_step * args.steps * world / slow / 1e9
@@ -330,7 +359,7 @@ def run_ours(args, rank, world, local):
             gs = g50 if s == HEADLINE_SPARSITY else graphs_for(s)
             nz = kept_counts(projs, s)
             b = algorithmic_bytes(projs, nz)
-            sec = time_graphs(gs, steps_x, 20, stream)
+            sec = time_steps(gs, steps_x, 24, stream)
             us = sec / steps_x * 1e6
             sweep.append({"sparsity": s, "us_per_step": round(us, 2),
                           "GBps": round(b / (us * 1e-6) / 1e9, 1),
@@ -355,16 +384,15 @@ def run_ours(args, rank, world, local):
 
 
 def per_projection(projs, copies, dev_x, ys, wss, stream, sig, steps):
-    import torch
     out = {}
     for j, p in enumerate(projs):
         def f(c, j=j, p=p):
             def g():
-                sig.sparse_gemv(copies[c][j] if copies[c] else copies[0][j], dev_x[j],
-                                t=p.thresholds[HEADLINE_SPARSITY], y=ys[j], ws=wss[j], stream=stream)
+                sig.sparse_gemv(copies[c][j], dev_x[j], t=p.thresholds[HEADLINE_SPARSITY], y=ys[j],
+                                ws=wss[j], stream=stream)
             return g
-        gs = [capture(f(c), stream) for c in range(N_COPIES)]
-        sec = time_graphs(gs, steps, 20, stream)
+        sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=48)
+        sec = time_steps(sg, steps, 24, stream)
         us = sec / steps * 1e6
         nnz = kept_counts([p], HEADLINE_SPARSITY)[0]
         b = nnz * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out
@@ -382,11 +410,8 @@ def cublas_dense(projs, copies, dev_x, stream, steps):
             for j in range(len(projs)):
                 torch.matmul(dev_x[j].view(1, -1), copies[c][j], out=outs[j])
         return g
-    with torch.cuda.stream(stream):
-        f(0)()
-    torch.cuda.synchronize()
-    gs = [capture(f(c), stream) for c in range(N_COPIES)]
-    sec = time_graphs(gs, steps, 20, stream)
+    sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=12)
+    sec = time_steps(sg, steps, 24, stream)
     us = sec / steps * 1e6
     dense_bytes = sum(p.d_in * p.d_out * 2 + 2 * p.d_in + 2 * p.d_out for p in projs)
     return {"us_per_step": round(us, 2), "GBps": round(dense_bytes / (us * 1e-6) / 1e9, 1)}
@@ -414,12 +439,9 @@ def bench_topk(args, stream, sig, hbm_peak):
                 sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
                 sig.sparse_gemv(ws_w[j], X[j], idx=idx, nnz=nnz, y=ys[j], ws=ws[j], stream=stream)
         return g
-    with torch.cuda.stream(stream):
-        f(W)()
-    torch.cuda.synchronize()
-    gs = [capture(f(W), stream), capture(f(Wc), stream)]
+    sg = StepGraphs([f(W), f(Wc)], stream, per_graph=8)
     steps = 200
-    sec = time_graphs(gs, steps, 10, stream)
+    sec = time_steps(sg, steps, 8, stream)
     us = sec / steps * 1e6
     b = sum(k * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out for k, p in zip(ks, projs))
     # top-k alone
@@ -427,14 +449,14 @@ def bench_topk(args, stream, sig, hbm_peak):
         for j, p in enumerate(projs):
             mb, idx, nnz = bufs[j]
             sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
-    gt = [capture(h, stream)]
-    sec_t = time_graphs(gt, steps, 10, stream)
+    st = StepGraphs([h], stream, per_graph=8)
+    sec_t = time_steps(st, steps, 8, stream)
     res = {"shapes": "8192->28672 and 28672->8192", "keep": k_frac,
            "us_per_pair": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
            "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
            "topk_select_us_per_pair": round(sec_t / steps * 1e6, 2),
            "l2": "2 rotating weight copies of 940 MB"}
-    del W, Wc, gs, gt
+    del W, Wc, sg, st
     torch.cuda.empty_cache()
     return res
 
@@ -460,13 +482,10 @@ def bench_rana(args, stream, sig, hbm_peak):
         def g():
             sig.gated_mlp_sparse(x, *W, norms, t, y=y, h_out=h, mask_out=mask, ws=ws, stream=stream)
         return g
-    with torch.cuda.stream(stream):
-        f(Ws[0])()
-    torch.cuda.synchronize()
     nnz = int((s >= t).sum())
-    gs = [capture(f(W), stream) for W in Ws]
+    sg = StepGraphs([f(W) for W in Ws], stream, per_graph=8)
     steps = 300
-    sec = time_graphs(gs, steps, 10, stream)
+    sec = time_steps(sg, steps, 8, stream)
     us = sec / steps * 1e6
     d_model, d_ff = mlp.WgT.shape
     b = 2 * d_model * d_ff * 2 + nnz * 2 * d_model + 2 * d_model + 2 * d_ff * 2 + 4 * d_ff
@@ -474,7 +493,7 @@ def bench_rana(args, stream, sig, hbm_peak):
            "us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
            "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
            "l2": "2 rotating weight copies of 258 MB"}
-    del Ws, gs
+    del Ws, sg
     torch.cuda.empty_cache()
     return res
 
@@ -499,26 +518,30 @@ def bench_nm(args, stream, sig, bf16_peak):
             def g():
                 sig.nm_act_gemm(Xs[c], Ws[c], n, m, Y=Y, ws=ws, stream=stream)
             return g
-        with torch.cuda.stream(stream):
-            f(0)()
-        torch.cuda.synchronize()
-        gs = [capture(f(c), stream) for c in range(copies)]
-        sec = time_graphs(gs, steps, 10, stream)
+        sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies)
+        sec = time_steps(sg, steps, copies, stream)
         us = sec / steps * 1e6
+        Xm = torch.empty_like(Xs[0])
+
+        def mk(c, n=n, m=m):
+            def g():
+                sig.sparsify_nm(Xs[c], n, m, X_masked=Xm, want_bits=False, stream=stream)
+            return g
+        sm = StepGraphs([mk(c) for c in range(copies)], stream, per_graph=copies)
+        us_mask = time_steps(sm, steps, copies, stream) / steps * 1e6
         out[f"{n}:{m}"] = {"us": round(us, 2),
                            "TFLOPs_executed": round(flops_dense / (us * 1e-6) / 1e12, 1),
-                           "TFLOPs_algorithmic": round(flops_dense * n / m / (us * 1e-6) / 1e12, 1)}
+                           "TFLOPs_algorithmic": round(flops_dense * n / m / (us * 1e-6) / 1e12, 1),
+                           "mask_only_us": round(us_mask, 2),
+                           "mask_GBps": round(2 * X.nbytes / (us_mask * 1e-6) / 1e9, 1)}
     Yd = torch.empty_like(Y)
 
     def d(c):
         def g():
             torch.matmul(Xs[c], Ws[c], out=Yd)
         return g
-    with torch.cuda.stream(stream):
-        d(0)()
-    torch.cuda.synchronize()
-    gs = [capture(d(c), stream) for c in range(copies)]
-    sec = time_graphs(gs, steps, 10, stream)
+    sg = StepGraphs([d(c) for c in range(copies)], stream, per_graph=copies)
+    sec = time_steps(sg, steps, copies, stream)
     us = sec / steps * 1e6
     out["cublas_dense"] = {"us": round(us, 2), "TFLOPs": round(flops_dense / (us * 1e-6) / 1e12, 1)}
     out["tensor_peak_tflops"] = bf16_peak
@@ -635,8 +658,49 @@ def run_reference(args, rank, world):
             "gpu_launches": 0}
 
 
+def profile_case(args):
+    """A few eager launches of one kernel case, inputs larger than L2, for ncu."""
+    import torch
+    import sparse_input_gemv_threshold_b200 as sig
+    torch.cuda.set_device(0)
+    case = args.profile_case
+    if case in dict((n, 0) for n, _, _ in workloads.LLAMA2_7B_PROJECTIONS):
+        (p,) = workloads.llama2_7b(args.seed, names=(case,))
+        copies = max(2, math.ceil(4 * 126e6 / (p.d_in * p.d_out * 2)))
+        W = [torch.from_numpy(p.WT).cuda()]
+        W += [W[0].clone() for _ in range(copies - 1)]
+        x = torch.from_numpy(p.x).cuda()
+        y = torch.empty(p.d_out, dtype=torch.float16, device="cuda")
+        ws = torch.zeros(sig.workspace_bytes(sig.OP_SPARSE_GEMV, p.d_in, p.d_out), dtype=torch.uint8,
+                         device="cuda")
+        for i in range(args.launches):
+            sig.sparse_gemv(W[i % copies], x, t=p.thresholds[HEADLINE_SPARSITY], y=y, ws=ws)
+        nnz = kept_counts([p], HEADLINE_SPARSITY)[0]
+        info = {"case": case, "launches": args.launches, "copies": copies,
+                "algorithmic_bytes_per_launch": nnz * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out}
+    elif case == "nm2:4":
+        WT, X = workloads.nm_tokens(args.seed)
+        Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()
+        for _ in range(args.launches):
+            Y = sig.nm_act_gemm(Xd, Wd, 2, 4)
+        info = {"case": case, "launches": args.launches}
+    elif case == "topk70b":
+        (p,) = workloads.qsparse_70b(args.seed, names=("down",))
+        x = torch.from_numpy(p.x).cuda()
+        for _ in range(args.launches):
+            sig.sparsify_topk(x, workloads.topk_count(0.5, p.d_in))
+        info = {"case": case, "launches": args.launches}
+    else:
+        raise SystemExit(f"unknown profile case {case!r}")
+    torch.cuda.synchronize()
+    print(json.dumps(info))
+    return 0
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        return profile_case(args)
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         res = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))

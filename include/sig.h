@@ -78,6 +78,8 @@ typedef enum {
 
 /* Largest activation length the fused mask prologue accepts. */
 #define SIG_MAX_D_IN 131072
+/* Largest length sparsify_topk accepts (its keys live in shared memory). */
+#define SIG_MAX_TOPK_D 131072
 
 /* Human-readable name of a status code (static storage, never NULL). */
 SIG_API const char* sig_status_string(int status);
@@ -124,8 +126,8 @@ SIG_API int sparsify_threshold(const uint16_t* x, int64_t d, float t,
  *   mask_bits  [ceil(d/32)] uint32 out.   idx [d] int32 out (first k valid).
  *   nnz        [1] int32 out (= k).
  *   ws         sig_workspace_bytes(SIG_OP_TOPK, d, 0, 0) bytes (may be 0 → ws may be NULL).
- * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d < 1 or d > SIG_MAX_D_IN), SIG_ERR_ARG (k),
- *         SIG_ERR_ALIGN, SIG_ERR_WORKSPACE.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d < 1 or d > SIG_MAX_TOPK_D), SIG_ERR_ARG (k),
+ *         SIG_ERR_ALIGN.
  */
 SIG_API int sparsify_topk(const uint16_t* x, int64_t d, int64_t k,
                   uint32_t* mask_bits, int32_t* idx, int32_t* nnz,

@@ -106,7 +106,7 @@ int sparsify_topk(const uint16_t* x, int64_t d, int64_t k, uint32_t* mask_bits, 
   (void)ws_bytes;
   if (x == nullptr || mask_bits == nullptr || idx == nullptr || nnz == nullptr)
     return SIG_ERR_NULL;
-  if (d < 1 || d > kMaxDIn) return SIG_ERR_SHAPE;
+  if (d < 1 || d > kMaxTopkD) return SIG_ERR_SHAPE;
   if (k < 0 || k > d) return SIG_ERR_ARG;
   if (!aligned16(x)) return SIG_ERR_ALIGN;
   return cuda_status(launch_topk(x, (int)d, (int)k, mask_bits, idx, nnz, (cudaStream_t)stream));

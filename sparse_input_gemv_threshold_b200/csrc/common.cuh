@@ -8,12 +8,30 @@ namespace sig {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-// 16-byte streaming load of weights: read once, do not keep in L1.
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel on the stream drains; it
+// must wait for that grid (and its memory) before touching global memory.
+// Triggering at once lets the next kernel's CTAs take SM slots as ours exit.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// L2 policy for data read exactly once (weight rows): evict first, so that
+// the stream does not push the small reused buffers (x, index lists, split-K
+// partials, counters) out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte streaming load of weights: not kept in L1, evict-first in L2.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p, uint64_t pol) {
   uint4 r;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
       : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-      : "l"(p));
+      : "l"(p), "l"(pol));
   return r;
 }
 
@@ -89,22 +107,34 @@ __device__ __forceinline__ void build_mask_words(const uint16_t* __restrict__ x,
                                                  uint32_t* words, Pred pred) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int nwords = (d + 31) >> 5;
-  for (int base = 0; base < d; base += BLOCK * 8) {
-    const int e0 = base + tid * 8;
-    uint32_t b = 0;
-    if (e0 + 8 <= d) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + e0));
+  constexpr int kChunk = BLOCK * 8;   // elements per pass of the block
+  constexpr int kUnroll = 8;          // passes whose loads are in flight together
+  for (int base0 = 0; base0 < d; base0 += kChunk * kUnroll) {
+    uint4 v[kUnroll];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) b |= (pred(lane_half(v, k), e0 + k) ? 1u : 0u) << k;
-    } else {
-      for (int k = 0; k < 8; ++k)
-        if (e0 + k < d) b |= (pred(x[e0 + k], e0 + k) ? 1u : 0u) << k;
+    for (int u = 0; u < kUnroll; ++u) {
+      const int e0 = base0 + u * kChunk + tid * 8;
+      v[u] = e0 + 8 <= d ? __ldg(reinterpret_cast<const uint4*>(x + e0)) : make_uint4(0, 0, 0, 0);
     }
-    uint32_t w = b << (8 * (lane & 3));
-    w |= __shfl_xor_sync(kFull, w, 1);
-    w |= __shfl_xor_sync(kFull, w, 2);
-    const int wi = (base >> 5) + (tid >> 2);
-    if ((lane & 3) == 0 && wi < nwords) words[wi] = w;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int base = base0 + u * kChunk;
+      if (base >= d) break;               // uniform across the block
+      const int e0 = base + tid * 8;
+      uint32_t b = 0;
+      if (e0 + 8 <= d) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) b |= (pred(lane_half(v[u], k), e0 + k) ? 1u : 0u) << k;
+      } else {
+        for (int k = 0; k < 8; ++k)
+          if (e0 + k < d) b |= (pred(x[e0 + k], e0 + k) ? 1u : 0u) << k;
+      }
+      uint32_t w = b << (8 * (lane & 3));
+      w |= __shfl_xor_sync(kFull, w, 1);
+      w |= __shfl_xor_sync(kFull, w, 2);
+      const int wi = (base >> 5) + (tid >> 2);
+      if ((lane & 3) == 0 && wi < nwords) words[wi] = w;
+    }
   }
 }
 

@@ -8,9 +8,11 @@
 // One launch does everything:
 //   1. every CTA ballots the whole activation (it sits in L2), packs the mask
 //      into shared words and prefix-scans their popcounts, which gives nnz and
-//      the CTA's equal share [lo, hi) of the ascending kept-row list;
+//      the CTA's equal share [lo, hi) of the ascending kept-row list; each
+//      thread then places its ranks by a binary search over the word prefixes;
 //   2. the CTA streams its share of kept rows for its 256-column tile with
-//      16-byte non-allocating loads, 8 rows in flight per warp, fp32 FMA;
+//      16-byte non-allocating loads, 8 rows in flight per warp (each with its
+//      activation value, a broadcast load), fp32 FMA;
 //   3. the 8 warps' sums meet in shared memory, the CTA writes one fp32 partial
 //      per column, and the CTA that arrives last for the tile (a counter in
 //      the workspace) adds the partials in split order and stores fp16.
@@ -34,7 +36,8 @@ struct KArgs {
   const int32_t* nnz;
   float t;
   int d_in, d_out, S, cap;
-  uint32_t union_bytes;   // shared bytes of the words / reduction union
+  uint32_t words_bytes;   // shared bytes of the mask words (and of their prefixes)
+  uint32_t union_bytes;   // shared bytes of the words + prefixes / reduction union
   uint16_t* y;
   uint32_t* mask_out;
   unsigned* counters;
@@ -54,8 +57,11 @@ sgemv_kernel(const KArgs a) {
   const int d_in = a.d_in, d_out = a.d_out, S = a.S;
 
   uint32_t* words = reinterpret_cast<uint32_t*>(smem);
+  int* wpre = reinterpret_cast<int*>(smem + a.words_bytes);
   int* sidx = reinterpret_cast<int*>(smem + a.union_bytes);
-  float* sx = reinterpret_cast<float*>(smem + a.union_bytes + (size_t)a.cap * 4);
+
+  pdl_trigger();
+  pdl_wait();
 
   // ---- 1. which rows does this CTA own? --------------------------------
   int n_rows = 0;
@@ -75,25 +81,24 @@ sgemv_kernel(const KArgs a) {
     for (int w = w0; w < w1; ++w) cnt += __popc(words[w]);
     int total;
     int r = block_exclusive_scan<kGemvThreads>(cnt, scan_scratch, &total);
+    for (int w = w0; w < w1; ++w) {   // exclusive kept-count before each word
+      wpre[w] = r;
+      r += __popc(words[w]);
+    }
+    __syncthreads();
     const int lo = (int)(((long long)s * total) / S);
     const int hi = (int)(((long long)(s + 1) * total) / S);
     n_rows = hi - lo;
-    if (r < hi && r + cnt > lo) {
-      for (int w = w0; w < w1 && r < hi; ++w) {
-        uint32_t bits = words[w];
-        const int pc = __popc(bits);
-        if (r + pc <= lo) { r += pc; continue; }
-        while (bits) {
-          const int b = __ffs(bits) - 1;
-          bits &= bits - 1;
-          if (r >= lo && r < hi) {
-            const int i = w * 32 + b;
-            sidx[r - lo] = i;
-            sx[r - lo] = h2f(a.x[i]);
-          }
-          ++r;
-        }
+    // Every thread places its own ranks: the word holding rank lo + j is the
+    // last one whose prefix is <= that rank; __fns finds the bit inside it.
+    for (int j = tid; j < n_rows; j += kGemvThreads) {
+      const int rank = lo + j;
+      int a0 = 0, a1 = nwords - 1;
+      while (a0 < a1) {
+        const int mid = (a0 + a1 + 1) >> 1;
+        if (wpre[mid] <= rank) a0 = mid; else a1 = mid - 1;
       }
+      sidx[j] = a0 * 32 + (int)__fns(words[a0], 0, rank - wpre[a0] + 1);
     }
     if (a.mask_out != nullptr && c == 0 && s == 0)
       for (int w = tid; w < nwords; w += kGemvThreads) a.mask_out[w] = words[w];
@@ -104,18 +109,13 @@ sgemv_kernel(const KArgs a) {
     n_rows = hi - lo;
     for (int j = tid; j < n_rows; j += kGemvThreads) {
       const int i = __ldg(a.idx + lo + j);
-      const bool ok = (unsigned)i < (unsigned)d_in;
-      sidx[j] = ok ? i : -1;
-      sx[j] = ok ? h2f(a.x[i]) : 0.f;
+      sidx[j] = (unsigned)i < (unsigned)d_in ? i : -1;
     }
   } else {  // MASK_DENSE
     const int lo = (int)(((long long)s * d_in) / S);
     const int hi = (int)(((long long)(s + 1) * d_in) / S);
     n_rows = hi - lo;
-    for (int j = tid; j < n_rows; j += kGemvThreads) {
-      sidx[j] = lo + j;
-      sx[j] = h2f(a.x[lo + j]);
-    }
+    for (int j = tid; j < n_rows; j += kGemvThreads) sidx[j] = lo + j;
   }
   __syncthreads();
 
@@ -129,34 +129,34 @@ sgemv_kernel(const KArgs a) {
   if (col_ok) {
     const uint16_t* wp = a.WT + col;
     const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
+    const uint64_t pol = l2_evict_first_policy();
+    // U rows per warp in flight; the last batch is predicated, so a warp with
+    // only a few rows still issues all of its loads at once.
     constexpr int U = DUAL ? 4 : 8;
-    int j = warp;
-    for (; j + kWarps * (U - 1) < n_rows; j += kWarps * U) {
+    for (int j0 = warp; j0 < n_rows; j0 += kWarps * U) {
       uint4 v[U], v2[U];
-      float xv[U];
+      uint16_t xh[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int r = sidx[j + kWarps * u];
-        xv[u] = sx[j + kWarps * u];
-        if (MODE == MASK_IDX && r < 0) {
-          v[u] = make_uint4(0, 0, 0, 0);
+        const int j = j0 + kWarps * u;
+        const int r = j < n_rows ? sidx[j] : -1;
+        if (r >= 0) {
+          // the activation rides along with its weight row: both in flight
+          xh[u] = __ldg(a.x + r);
+          v[u] = ld_stream_v4(wp + (size_t)r * d_out, pol);
+          if (DUAL) v2[u] = ld_stream_v4(wp2 + (size_t)r * d_out, pol);
         } else {
-          v[u] = ld_stream_v4(wp + (size_t)r * d_out);
-          if (DUAL) v2[u] = ld_stream_v4(wp2 + (size_t)r * d_out);
+          xh[u] = 0;
+          v[u] = make_uint4(0, 0, 0, 0);
+          if (DUAL) v2[u] = make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        fma8(acc, v[u], xv[u]);
-        if (DUAL) fma8(acc2, v2[u], xv[u]);
+        const float xv = h2f(xh[u]);
+        fma8(acc, v[u], xv);
+        if (DUAL) fma8(acc2, v2[u], xv);
       }
-    }
-    for (; j < n_rows; j += kWarps) {
-      const int r = sidx[j];
-      if (MODE == MASK_IDX && r < 0) continue;
-      const float xv = sx[j];
-      fma8(acc, ld_stream_v4(wp + (size_t)r * d_out), xv);
-      if (DUAL) fma8(acc2, ld_stream_v4(wp2 + (size_t)r * d_out), xv);
     }
   }
 
@@ -206,10 +206,22 @@ sgemv_kernel(const KArgs a) {
   if (!s_last) return;
   __threadfence();
   if (colr_ok) {
+    // all loads of a batch in flight together, then added in split order
+    constexpr int B = DUAL ? 16 : 32;
     float g = 0.f, u = 0.f;
-    for (int q = 0; q < S; ++q) {
-      g += __ldcg(a.partials + (size_t)q * d_out + colr);
-      if (DUAL) u += __ldcg(a.partials + (size_t)S * d_out + (size_t)q * d_out + colr);
+    for (int q0 = 0; q0 < S; q0 += B) {
+      float pg[B], pu[B];
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        const bool ok = q0 + k < S;
+        pg[k] = ok ? __ldcg(a.partials + (size_t)(q0 + k) * d_out + colr) : 0.f;
+        if (DUAL) pu[k] = ok ? __ldcg(a.partials + (size_t)S * d_out + (size_t)(q0 + k) * d_out + colr) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        g += pg[k];
+        if (DUAL) u += pu[k];
+      }
     }
     finish(g, u);
   }
@@ -226,9 +238,7 @@ cudaError_t launch_t(const GemvPlan& p, const KArgs& k, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  dim3 grid(p.C, p.S);
-  fn<<<grid, kGemvThreads, p.smem, stream>>>(k);
-  return cudaPeekAtLastError();
+  return launch_pdl(fn, dim3(p.C, p.S), dim3(kGemvThreads), p.smem, stream, k);
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -245,8 +255,8 @@ GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual) {
   p.cap = (int)((d_in + S - 1) / S);
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)(kGemvThreads / 32) * kGemvTile * 4 * (dual ? 2 : 1);
-  const size_t uni = std::max(words, red);
-  p.smem = uni + round_up((size_t)p.cap * 8, 16);
+  const size_t uni = std::max(2 * words, red);
+  p.smem = uni + round_up((size_t)p.cap * 4, 16);
   p.counters = round_up((size_t)p.C * 4, 256);
   p.partials = S > 1 ? round_up((size_t)S * d_out * 4 * (dual ? 2 : 1), 256) : 0;
   return p;
@@ -259,7 +269,8 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   k.t = a.t; k.d_in = a.d_in; k.d_out = a.d_out; k.S = p.S; k.cap = p.cap;
   const size_t words = round_up((size_t)((a.d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)(kGemvThreads / 32) * kGemvTile * 4 * (epi == EPI_SILU_MUL ? 2 : 1);
-  k.union_bytes = (uint32_t)std::max(words, red);
+  k.words_bytes = (uint32_t)words;
+  k.union_bytes = (uint32_t)std::max(2 * words, red);
   k.y = a.y; k.mask_out = a.mask_out;
   k.counters = reinterpret_cast<unsigned*>(a.ws);
   k.partials = reinterpret_cast<float*>(reinterpret_cast<char*>(a.ws) + p.counters);

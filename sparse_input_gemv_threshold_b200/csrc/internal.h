@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace sig {
 
 constexpr int kNumSMs = 148;         // B200: 2 dies x 74 SMs
@@ -13,6 +15,7 @@ constexpr int kGemvTile = 256;       // output columns per CTA (one warp spans t
 constexpr int kGemvCtasPerSM = 4;    // target residency; grid = C x S <= 148 * 4
 constexpr int kIdxCap = 4096;        // largest slice of the index list per CTA
 constexpr int kMaxDIn = 131072;
+constexpr int kMaxTopkD = 131072;    // top-k stages its keys in the cluster's shared memory
 
 // How the rows of a sparse GEMV are chosen.
 enum MaskMode : int {
@@ -27,6 +30,23 @@ enum Epilogue : int {
   EPI_STORE = 0,     // y_j = fp16(sum)
   EPI_SILU_MUL = 1   // dual product (g, u): h_j = fp16(SiLU(g_j) * u_j)
 };
+
+// Launch `kernel` with programmatic stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct GemvPlan {
   int C;              // column tiles

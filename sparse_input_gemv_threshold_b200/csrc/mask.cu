@@ -2,13 +2,16 @@
 //
 //  - threshold (TEAL README, Abstract; ">= t" as in RaNA Eqn. 12);
 //  - top-k by magnitude ("Q-Sparse ..." rebuttal, A1 on MoE): a radix select on
-//    the 16-bit magnitude key finds the k-th largest key K* and the number q of
-//    entries equal to K* that still fit, then the q lowest-index ties are kept;
+//    the 16-bit magnitude key, spread over a thread-block cluster, finds the
+//    k-th largest key K* and the number q of entries equal to K* that still
+//    fit, then the q lowest-index ties are kept;
 //  - N:M ("Flexible (N:M) Activation Sparsity", Methodology; Block Q-Sparse in
 //    the Q-Sparse rebuttal, A2): per block of m, the n entries of largest key;
 //  - row norms (||W^down_i|| of RaNA Eqn. 12), float64 accumulation.
 #include "common.cuh"
 #include "internal.h"
+
+#include <cooperative_groups.h>
 
 namespace sig {
 
@@ -46,6 +49,9 @@ threshold_compact_kernel(const uint16_t* __restrict__ x, int d, float t, uint32_
                          int32_t* idx, int32_t* nnz) {
   extern __shared__ __align__(16) uint32_t words[];
   __shared__ int scratch[kMaskThreads / 32 + 1];
+
+  pdl_trigger();
+  pdl_wait();
   build_mask_words<kMaskThreads>(x, d, words,
                                  [&](uint16_t h, int) { return fabsf(h2f(h)) >= t; });
   __syncthreads();
@@ -72,154 +78,292 @@ __device__ void find_bin(const int* hist, int nbins, int need, int* scratch, int
   __syncthreads();
 }
 
+// Count key `bin` into a per-warp histogram; lanes with equal bins add once.
+__device__ __forceinline__ void warp_hist_add(int* hist, uint32_t bin, bool active) {
+  const unsigned grp = __match_any_sync(kFull, active ? bin : 0xffffffffu);
+  const int lane = threadIdx.x & 31;
+  if (active && lane == __ffs(grp) - 1) atomicAdd(&hist[bin], __popc(grp));
+}
+
+// Radix select on the 16-bit magnitude key, spread over a cluster of
+// kTopkCluster CTAs.  CTA q owns the keys [q*chunk, (q+1)*chunk) (whole mask
+// words) and stages them in its shared memory.
+//   pass 1  local histogram of key >> 8; after a cluster barrier every CTA sums
+//           all CTAs' histograms through distributed shared memory and finds
+//           the high byte of K* (the k-th largest key) the same way;
+//   pass 2  the same for the low byte among keys with that high byte, giving
+//           K* and q = the number of entries equal to K* that still fit;
+//   then    local bitmaps key > K* and key == K*; a CTA's first tie rank and
+//           its first output slot are the counts published by lower-ranked
+//           CTAs, so the q lowest-index ties are kept and the index list comes
+//           out ascending.
+constexpr int kTopkCluster = 8;
+
 __global__ void __launch_bounds__(kMaskThreads)
-topk_kernel(const uint16_t* __restrict__ x, int d, int k, uint32_t* mask_bits, int32_t* idx,
-            int32_t* nnz) {
-  extern __shared__ __align__(16) uint32_t dyn[];
+topk_cluster_kernel(const uint16_t* __restrict__ x, int d, int k, int chunk, uint32_t* mask_bits,
+                    int32_t* idx, int32_t* nnz) {
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(16) unsigned char dyn_raw[];
   constexpr int kWarps = kMaskThreads / 32;
-  __shared__ int hist[kMaskThreads];           // merged histogram
   __shared__ int whist[kWarps][256];           // per-warp histograms
+  __shared__ int hist1[256], hist2[256];       // this CTA's pass-1 / pass-2 histograms
+  __shared__ int ghist[256];                   // cluster-wide histogram
   __shared__ int scratch[kWarps + 1];
   __shared__ int sel[2];
-  __shared__ int tie_cut;                      // index after the q-th tie (exclusive)
+  __shared__ int pub[2];                       // [0] ties here, [1] kept here
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwords = (d + 31) >> 5;
-  uint32_t* gt = dyn;                          // key > K*
-  uint32_t* eq = dyn + nwords;                 // key == K*
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cq = (int)cluster.block_rank();
+  pdl_trigger();
+  pdl_wait();
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int e_begin = cq * chunk;
+  const int nloc = max(0, min(d, e_begin + chunk) - e_begin);
+  const int nwl = (nloc + 31) >> 5;             // local words holding keys
+  const int w_begin = e_begin >> 5;             // first global mask word of this CTA
+  uint16_t* keys = reinterpret_cast<uint16_t*>(dyn_raw);
+  uint32_t* gt = reinterpret_cast<uint32_t*>(dyn_raw + (size_t)chunk * 2);
+  uint32_t* eq = gt + (chunk >> 5);
 
   if (k <= 0) {
-    for (int w = tid; w < nwords; w += kMaskThreads) { mask_bits[w] = 0u; gt[w] = 0u; }
-    __syncthreads();
-    compact_words<kMaskThreads>(gt, nwords, idx, nnz, scratch);
+    for (int w = tid; w < nwl; w += kMaskThreads) mask_bits[w_begin + w] = 0u;
+    if (cq == 0 && tid == 0) *nnz = 0;
     return;
   }
 
-  // Pass 1: histogram of key >> 8 (keys are <= 0x7c01, so 125 bins used).
+  // Stage the keys of this CTA's range (zero padding is never counted).
+  for (int e0 = tid * 8; e0 < nwl * 32; e0 += kMaskThreads * 8) {
+    const int g0 = e_begin + e0;
+    uint32_t p[4];
+    if (g0 + 8 <= d) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + g0));
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        p[q] = mag_key(lane_half(v, 2 * q)) | (mag_key(lane_half(v, 2 * q + 1)) << 16);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = g0 + 2 * q < d ? mag_key(x[g0 + 2 * q]) : 0u;
+        const uint32_t hi = g0 + 2 * q + 1 < d ? mag_key(x[g0 + 2 * q + 1]) : 0u;
+        p[q] = lo | (hi << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(keys + e0) = make_uint4(p[0], p[1], p[2], p[3]);
+  }
   for (int i = tid; i < kWarps * 256; i += kMaskThreads) (&whist[0][0])[i] = 0;
   __syncthreads();
-  for (int i = tid; i < d; i += kMaskThreads) atomicAdd(&whist[warp][mag_key(x[i]) >> 8], 1);
-  __syncthreads();
-  if (tid < 256) {
-    int s = 0;
-    for (int w = 0; w < kWarps; ++w) s += whist[w][tid];
-    hist[tid] = s;
+
+  // ---- pass 1: high byte ----
+  for (int i0 = 0; i0 < nloc; i0 += kMaskThreads) {
+    const int i = i0 + tid;
+    const bool ok = i < nloc;
+    warp_hist_add(whist[warp], ok ? (uint32_t)keys[i] >> 8 : 0u, ok);
   }
   __syncthreads();
-  find_bin<kMaskThreads>(hist, 256, k, scratch, sel);
+  if (tid < 256) {
+    int v = 0;
+    for (int w = 0; w < kWarps; ++w) { v += whist[w][tid]; whist[w][tid] = 0; }
+    hist1[tid] = v;
+  }
+  cluster.sync();
+  if (tid < 256) {
+    int v = 0;
+    for (int r = 0; r < kTopkCluster; ++r) v += cluster.map_shared_rank(hist1, r)[tid];
+    ghist[tid] = v;
+  }
+  __syncthreads();
+  find_bin<kMaskThreads>(ghist, 256, k, scratch, sel);
   const int hi_bin = sel[0], above_hi = sel[1];
 
-  // Pass 2: histogram of the low byte within the chosen high bin.
-  for (int i = tid; i < kWarps * 256; i += kMaskThreads) (&whist[0][0])[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < d; i += kMaskThreads) {
-    const uint32_t key = mag_key(x[i]);
-    if ((int)(key >> 8) == hi_bin) atomicAdd(&whist[warp][key & 0xff], 1);
+  // ---- pass 2: low byte among keys with that high byte ----
+  for (int i0 = 0; i0 < nloc; i0 += kMaskThreads) {
+    const int i = i0 + tid;
+    const uint32_t key = i < nloc ? keys[i] : 0u;
+    const bool ok = i < nloc && (int)(key >> 8) == hi_bin;
+    warp_hist_add(whist[warp], key & 0xffu, ok);
   }
   __syncthreads();
   if (tid < 256) {
-    int s = 0;
-    for (int w = 0; w < kWarps; ++w) s += whist[w][tid];
-    hist[tid] = s;
+    int v = 0;
+    for (int w = 0; w < kWarps; ++w) v += whist[w][tid];
+    hist2[tid] = v;
+  }
+  cluster.sync();
+  if (tid < 256) {
+    int v = 0;
+    for (int r = 0; r < kTopkCluster; ++r) v += cluster.map_shared_rank(hist2, r)[tid];
+    ghist[tid] = v;
   }
   __syncthreads();
-  find_bin<kMaskThreads>(hist, 256, k - above_hi, scratch, sel);
+  find_bin<kMaskThreads>(ghist, 256, k - above_hi, scratch, sel);
   const uint32_t kstar = ((uint32_t)hi_bin << 8) | (uint32_t)sel[0];
-  const int q = k - above_hi - sel[1];          // ties at K* to keep, 1..count(K*)
+  const int q_ties = k - above_hi - sel[1];     // ties at K* to keep, cluster-wide
 
-  // Pass 3: bitmaps of key > K* and key == K*.
-  build_mask_words<kMaskThreads>(x, d, gt, [&](uint16_t h, int) { return mag_key(h) > kstar; });
-  build_mask_words<kMaskThreads>(x, d, eq, [&](uint16_t h, int) { return mag_key(h) == kstar; });
+  // ---- bitmaps of key > K* and key == K* for this CTA's words ----
+  for (int w = tid; w < nwl; w += kMaskThreads) {
+    const uint4* kp = reinterpret_cast<const uint4*>(keys + w * 32);
+    uint32_t g = 0, e = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = kp[c];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t key = lane_half(v, j);
+        const bool in = w * 32 + c * 8 + j < nloc;
+        g |= (in && key > kstar ? 1u : 0u) << (c * 8 + j);
+        e |= (in && key == kstar ? 1u : 0u) << (c * 8 + j);
+      }
+    }
+    gt[w] = g;
+    eq[w] = e;
+  }
   __syncthreads();
 
-  // Keep the q lowest-index ties: find the word holding the q-th tie.
-  {
-    const int per = (nwords + kMaskThreads - 1) / kMaskThreads;
-    const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(eq[w]);
-    int total;
-    int r = block_exclusive_scan<kMaskThreads>(cnt, scratch, &total);
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = eq[w];
-      uint32_t kept = 0;
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (r < q) kept |= 1u << b;
-        ++r;
-      }
-      gt[w] |= kept;
+  // ---- ties: this CTA's first tie rank is the ties of lower-ranked CTAs ----
+  const int per = (nwl + kMaskThreads - 1) / kMaskThreads;
+  const int w0 = min(nwl, tid * per), w1 = min(nwl, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(eq[w]);
+  int ties_here;
+  int r = block_exclusive_scan<kMaskThreads>(cnt, scratch, &ties_here);
+  if (tid == 0) pub[0] = ties_here;
+  cluster.sync();
+  int tie_base = 0;
+  for (int rr = 0; rr < cq; ++rr) tie_base += cluster.map_shared_rank(pub, rr)[0];
+  r += tie_base;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = eq[w], kept = 0;
+    while (bits && r < q_ties) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      kept |= 1u << b;
+      ++r;
+    }
+    gt[w] |= kept;
+  }
+  __syncthreads();
+
+  // ---- output: mask words and the ascending index list ----
+  cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(gt[w]);
+  int kept_here;
+  int o = block_exclusive_scan<kMaskThreads>(cnt, scratch, &kept_here);
+  if (tid == 0) pub[1] = kept_here;
+  cluster.sync();
+  int out_base = 0;
+  for (int rr = 0; rr < cq; ++rr) out_base += cluster.map_shared_rank(pub, rr)[1];
+  o += out_base;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = gt[w];
+    mask_bits[w_begin + w] = bits;
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      idx[o++] = e_begin + w * 32 + b;
     }
   }
-  (void)tie_cut;
-  (void)lane;
-  __syncthreads();
-  for (int w = tid; w < nwords; w += kMaskThreads) mask_bits[w] = gt[w];
-  compact_words<kMaskThreads>(gt, nwords, idx, nnz, scratch);
+  if (cq == 0 && tid == 0) *nnz = k;
+  cluster.sync();   // no CTA leaves while another may still read its shared memory
 }
 
-// One thread per 32-entry mask word of one row (m divides 32, so the blocks of
-// m never straddle a word).  Selection inside a block: the entry's rank is the
-// number of entries with a larger (key, lower index) composite; keep rank < n.
+// One bitonic stage (K = run length, J = partner distance) and the ones after
+// it; template recursion keeps every index a compile-time constant.
+template <int M, int K, int J>
+__device__ __forceinline__ void bitonic_stage(uint32_t (&s)[M]) {
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    const int l = i ^ J;
+    if (l > i) {
+      const uint32_t a = s[i], b = s[l];
+      const bool desc = (i & K) == 0;      // the final merge leaves s descending
+      s[i] = desc ? max(a, b) : min(a, b);
+      s[l] = desc ? min(a, b) : max(a, b);
+    }
+  }
+  if constexpr (J > 1) bitonic_stage<M, K, J / 2>(s);
+  else if constexpr (K < M) bitonic_stage<M, K * 2, K>(s);
+}
+
+// Bits of the n largest composites among M unique composites (bit j for c[j]).
+// M <= 8: count, for each entry, the entries ranked above it.  M >= 16: sort a
+// copy descending with a bitonic network; the n-th largest is the minimum of
+// the first n, and an entry is kept when it is at least that.
+template <int M>
+__device__ __forceinline__ uint32_t select_top_n(const uint32_t (&c)[M], int n) {
+  uint32_t bits = 0;
+  if constexpr (M <= 8) {
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      int rank = 0;
+#pragma unroll
+      for (int l = 0; l < M; ++l) rank += c[l] > c[j] ? 1 : 0;
+      bits |= (rank < n ? 1u : 0u) << j;
+    }
+  } else {
+    uint32_t s[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) s[j] = c[j];
+    bitonic_stage<M, 2, 1>(s);
+    uint32_t thr = 0xffffffffu;
+#pragma unroll
+    for (int j = 0; j < M; ++j) thr = min(thr, j < n ? s[j] : 0xffffffffu);
+#pragma unroll
+    for (int j = 0; j < M; ++j) bits |= (c[j] >= thr ? 1u : 0u) << j;
+  }
+  return bits;
+}
+
+// One thread per 32-entry mask word of one row (m divides 32, so blocks of m
+// never straddle a word).  Inside a block the entries are ranked by the
+// composite (magnitude key << 5 | (31 - position)): unique, larger magnitude
+// first, lower index first among equal magnitudes.
 template <int M>
 __global__ void __launch_bounds__(256)
 nm_mask_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, uint16_t* X_masked,
                uint32_t* mask_bits) {
   const int wpr = (d + 31) >> 5;
+  pdl_trigger();
+  pdl_wait();
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= rows * wpr) return;
   const int64_t row = g / wpr;
   const int w = (int)(g % wpr);
   const int e0 = w * 32;
-  const int cnt = min(32, d - e0);   // a multiple of M
+  const int cnt = min(32, d - e0);   // a multiple of 8 and of M
   const uint16_t* src = X + row * (int64_t)d + e0;
-  uint16_t v[32];
-  if (cnt == 32) {
+  uint4 q[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src) + q);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[q * 8 + k] = lane_half(u, k);
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) v[k] = k < cnt ? src[k] : (uint16_t)0;
-  }
+  for (int i = 0; i < 4; ++i)
+    q[i] = i * 8 < cnt ? __ldg(reinterpret_cast<const uint4*>(src) + i) : make_uint4(0, 0, 0, 0);
   uint32_t bits = 0;
 #pragma unroll
   for (int b0 = 0; b0 < 32; b0 += M) {
     if (b0 < cnt) {
       uint32_t comp[M];
 #pragma unroll
-      for (int j = 0; j < M; ++j) comp[j] = (mag_key(v[b0 + j]) << 5) | (uint32_t)(31 - j);
-#pragma unroll
-      for (int j = 0; j < M; ++j) {
-        int rank = 0;
-#pragma unroll
-        for (int l = 0; l < M; ++l) rank += comp[l] > comp[j] ? 1 : 0;
-        if (rank < n) bits |= 1u << (b0 + j);
-      }
+      for (int j = 0; j < M; ++j)
+        comp[j] = (mag_key(lane_half(q[(b0 + j) >> 3], (b0 + j) & 7)) << 5) | (uint32_t)(31 - j);
+      bits |= select_top_n<M>(comp, n) << b0;
     }
   }
   if (mask_bits != nullptr) mask_bits[row * wpr + w] = bits;
   if (X_masked != nullptr) {
     uint16_t* dst = X_masked + row * (int64_t)d + e0;
-    if (cnt == 32) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+    for (int i = 0; i < 4; ++i) {
+      if (i * 8 < cnt) {
+        const uint32_t wv[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
         uint32_t p[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int a = q * 8 + 2 * k;
-          const uint32_t lo = ((bits >> a) & 1u) ? v[a] : 0u;
-          const uint32_t hi = ((bits >> (a + 1)) & 1u) ? v[a + 1] : 0u;
-          p[k] = lo | (hi << 16);
+          const int a = i * 8 + 2 * k;
+          const uint32_t lo = ((bits >> a) & 1u) ? (wv[k] & 0xffffu) : 0u;
+          const uint32_t hi = ((bits >> (a + 1)) & 1u) ? (wv[k] & 0xffff0000u) : 0u;
+          p[k] = lo | hi;
         }
-        reinterpret_cast<uint4*>(dst)[q] = make_uint4(p[0], p[1], p[2], p[3]);
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(p[0], p[1], p[2], p[3]);
       }
-    } else {
-      for (int k = 0; k < cnt; ++k) dst[k] = ((bits >> k) & 1u) ? v[k] : (uint16_t)0;
     }
   }
 }
@@ -227,6 +371,8 @@ nm_mask_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, uint1
 // One warp per row: sum of squares in float64, sqrt, one rounding to float32.
 __global__ void __launch_bounds__(256)
 row_norms_kernel(const uint16_t* __restrict__ WT, int64_t rows, int cols, float* norms) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -255,18 +401,33 @@ cudaError_t launch_threshold_compact(const uint16_t* x, int d, float t, uint32_t
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  threshold_compact_kernel<<<1, kMaskThreads, smem, stream>>>(x, d, t, mask_bits, idx, nnz);
-  return cudaPeekAtLastError();
+  return launch_pdl(threshold_compact_kernel, dim3(1), dim3(kMaskThreads), smem, stream, x, d, t,
+                    mask_bits, idx, nnz);
 }
 
 cudaError_t launch_topk(const uint16_t* x, int d, int k, uint32_t* mask_bits, int32_t* idx,
                         int32_t* nnz, cudaStream_t stream) {
-  const size_t smem = (size_t)((d + 31) / 32) * 4 * 2 + 16;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  // whole words per CTA, and a multiple of 8 keys for the 16-byte staging loads
+  const int chunk = ((d + kTopkCluster - 1) / kTopkCluster + 31) / 32 * 32;
+  const size_t smem = (size_t)chunk * 2 + (size_t)(chunk / 32) * 8;
+  cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_kernel<<<1, kMaskThreads, smem, stream>>>(x, d, k, mask_bits, idx, nnz);
-  return cudaPeekAtLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kTopkCluster);
+  cfg.blockDim = dim3(kMaskThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kTopkCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, x, d, k, chunk, mask_bits, idx, nnz);
 }
 
 cudaError_t launch_nm_mask(const uint16_t* X, int64_t rows, int d, int n, int m,
@@ -274,24 +435,24 @@ cudaError_t launch_nm_mask(const uint16_t* X, int64_t rows, int d, int n, int m,
   const int64_t threads = rows * ((d + 31) / 32);
   if (threads == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((threads + 255) / 256);
+  cudaError_t e = cudaSuccess;
   switch (m) {
-    case 1: nm_mask_kernel<1><<<blocks, 256, 0, stream>>>(X, rows, d, n, X_masked, mask_bits); break;
-    case 2: nm_mask_kernel<2><<<blocks, 256, 0, stream>>>(X, rows, d, n, X_masked, mask_bits); break;
-    case 4: nm_mask_kernel<4><<<blocks, 256, 0, stream>>>(X, rows, d, n, X_masked, mask_bits); break;
-    case 8: nm_mask_kernel<8><<<blocks, 256, 0, stream>>>(X, rows, d, n, X_masked, mask_bits); break;
-    case 16: nm_mask_kernel<16><<<blocks, 256, 0, stream>>>(X, rows, d, n, X_masked, mask_bits); break;
-    case 32: nm_mask_kernel<32><<<blocks, 256, 0, stream>>>(X, rows, d, n, X_masked, mask_bits); break;
+    case 1: e = launch_pdl(nm_mask_kernel<1>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, X_masked, mask_bits); break;
+    case 2: e = launch_pdl(nm_mask_kernel<2>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, X_masked, mask_bits); break;
+    case 4: e = launch_pdl(nm_mask_kernel<4>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, X_masked, mask_bits); break;
+    case 8: e = launch_pdl(nm_mask_kernel<8>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, X_masked, mask_bits); break;
+    case 16: e = launch_pdl(nm_mask_kernel<16>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, X_masked, mask_bits); break;
+    case 32: e = launch_pdl(nm_mask_kernel<32>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, X_masked, mask_bits); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaPeekAtLastError();
+  return e;
 }
 
 cudaError_t launch_row_norms(const uint16_t* WT, int64_t rows, int cols, float* norms,
                              cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((rows + 7) / 8);
-  row_norms_kernel<<<blocks, 256, 0, stream>>>(WT, rows, cols, norms);
-  return cudaPeekAtLastError();
+  return launch_pdl(row_norms_kernel, dim3(blocks), dim3(256), 0, stream, WT, rows, cols, norms);
 }
 
 }  // namespace sig

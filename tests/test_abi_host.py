@@ -108,6 +108,7 @@ def test_mask_validation(lib):
     assert t(FAKE, 8, -1, FAKE, FAKE, FAKE, None, 0, None) == ARG
     assert t(FAKE, 8, 2, FAKE, None, FAKE, None, 0, None) == NULL
     assert t(FAKE, 0, 0, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
+    assert t(FAKE, 131073, 5, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
     n = lib.sparsify_nm
     assert n(FAKE, 4, 64, 3, 2, FAKE, FAKE, None) == ARG      # n > m
     assert n(FAKE, 4, 64, 0, 4, FAKE, FAKE, None) == ARG      # n < 1
