@@ -214,6 +214,35 @@ SIG_API int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16
                 sig_stream_t stream);
 
 /*
+ * gated_mlp_sparse without a workspace argument, for callers that cannot
+ * allocate device memory where they run this layer: a plugin inside a host
+ * program whose own pool owns all device memory, a serving loop whose memory
+ * budget is fixed at start-up, or plain C code with no allocator.  The pages
+ * have no counterpart to this entry point; it computes exactly what
+ * gated_mlp_sparse computes, with the same arguments minus ws / ws_bytes.
+ * Its scratch lives in one device array of SIG_NOALLOC_SCRATCH_BYTES inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.  It allocates nothing and calls no allocating routine.
+ *   - A call whose scratch (sig_workspace_bytes(SIG_OP_GATED_MLP, d_model,
+ *     d_ff, 0)) exceeds SIG_NOALLOC_SCRATCH_BYTES returns SIG_ERR_SHAPE with
+ *     nothing enqueued.  Llama-2-7B (4096, 11008) and Llama-70B (8192, 28672)
+ *     MLP shapes fit.
+ *   - Every call shares the array and finds the previous call's contents in
+ *     it; the call clears what must start at zero.  Calls that overlap on the
+ *     GPU (other streams, other host threads) race; serialise them.
+ *   - The first call on each device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ * Errors: as gated_mlp_sparse, except SIG_ERR_WORKSPACE (none is taken).
+ */
+#define SIG_NOALLOC_SCRATCH_BYTES (2u << 20)
+SIG_API int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                     const uint16_t* WdT, const float* down_norms,
+                                     int64_t d_model, int64_t d_ff, float t,
+                                     uint16_t* y, uint16_t* h_out, uint32_t* mask_out,
+                                     sig_stream_t stream);
+
+/*
  * Read and clear the library's device error word (no counterpart on the
  * pages; it reports the bounded waits of the tensor-core GEMM).  Synchronises
  * `stream`.  *code receives 0 when no kernel gave up on a wait, else a

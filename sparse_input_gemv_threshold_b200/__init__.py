@@ -21,7 +21,7 @@ __all__ = [
     "LIB_PATH", "SigError", "OP_SPARSE_GEMV", "OP_TOPK", "OP_GATED_MLP", "OP_NM_GEMM",
     "MAX_D_IN", "abi_version", "workspace_bytes", "workspace", "sparsify_threshold",
     "sparsify_topk", "sparsify_nm", "sparse_gemv", "gated_mlp_sparse", "row_norms",
-    "nm_act_gemm", "take_device_error", "status_string",
+    "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -45,6 +45,7 @@ _SIGNATURES = {
     "sig_row_norms": (_i32, [_p, _i64, _i64, _p, _p]),
     "nm_act_gemm": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _sz, _p]),
     "sig_take_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _p]),
+    "gated_mlp_sparse_noalloc": (_i32, [_p, _p, _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p]),
 }
 
 
@@ -198,6 +199,24 @@ def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
     _check("gated_mlp_sparse", _lib.gated_mlp_sparse(
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
         _ptr(y), _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def gated_mlp_sparse_noalloc(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
+                             mask_out=None, stream=None):
+    """gated_mlp_sparse with no workspace: for callers that cannot allocate
+    device memory at the call site.  Its scratch is a fixed array inside the
+    library (SIG_NOALLOC_SCRATCH_BYTES per GPU); calls that overlap on the GPU
+    race on it.  Make the first call on a device before any stream capture."""
+    for name, w in (("WgT", WgT), ("WuT", WuT), ("WdT", WdT), ("x", x)):
+        _need(w, torch.float16, name, x.device)
+    _need(down_norms, torch.float32, "down_norms", x.device)
+    d_model, d_ff = WgT.shape
+    if y is None:
+        y = torch.empty(d_model, dtype=torch.float16, device=x.device)
+    _check("gated_mlp_sparse_noalloc", _lib.gated_mlp_sparse_noalloc(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
+        _ptr(y), _ptr(h_out), _ptr(mask_out), _stream(stream)))
     return y
 
 

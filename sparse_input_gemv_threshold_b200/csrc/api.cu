@@ -24,22 +24,7 @@ int check_gemv_shape(int64_t d_in, int64_t d_out) {
   return SIG_OK;
 }
 
-struct GatedPlan {
-  GemvPlan up, down;
-  size_t off_down, off_h, total;
-};
-
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-GatedPlan plan_gated(int64_t d_model, int64_t d_ff) {
-  GatedPlan g;
-  g.up = plan_gemv(d_model, d_ff, true);
-  g.down = plan_gemv(d_ff, d_model, false);
-  g.off_down = round_up(g.up.ws_bytes(), 256);
-  g.off_h = g.off_down + round_up(g.down.ws_bytes(), 256);
-  g.total = g.off_h + round_up((size_t)d_ff * 2, 256);
-  return g;
-}
 
 bool nm_pattern_ok(int n, int m) {
   const bool pow2 = m == 1 || m == 2 || m == 4 || m == 8 || m == 16 || m == 32;

@@ -60,6 +60,24 @@ struct GemvPlan {
 
 GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual);
 
+// Workspace layout of the gated MLP: the dual (gate, up) product's counters and
+// partials, then the down product's, then the fp16 hidden vector h.
+struct GatedPlan {
+  GemvPlan up, down;
+  size_t off_down, off_h, total;
+};
+
+inline GatedPlan plan_gated(int64_t d_model, int64_t d_ff) {
+  auto up256 = [](size_t v) { return (v + 255) / 256 * 256; };
+  GatedPlan g;
+  g.up = plan_gemv(d_model, d_ff, true);
+  g.down = plan_gemv(d_ff, d_model, false);
+  g.off_down = up256(g.up.ws_bytes());
+  g.off_h = g.off_down + up256(g.down.ws_bytes());
+  g.total = g.off_h + up256((size_t)d_ff * 2);
+  return g;
+}
+
 struct GemvLaunch {
   const uint16_t* WT;
   const uint16_t* WT2;     // second weight for the dual (gate, up) product
