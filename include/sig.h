@@ -90,7 +90,9 @@ SIG_API int sig_abi_version(void);
 /*
  * Bytes of device workspace an operation needs for the given sizes (0 when
  * the operation needs none).  Returns 0 and sets nothing for an unknown op.
- * The workspace holds split-K partial sums and per-tile arrival counters.
+ * It holds split-K partial sums and arrival counters; the gated MLP also
+ * keeps its fp16 hidden vector there when h_out is NULL, and the N:M GEMM its
+ * masked activation block.
  */
 SIG_API size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows);
 
@@ -160,7 +162,10 @@ SIG_API int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m
  *   WT   [d_in x d_out] fp16 row-major, 16-byte aligned, d_out % 8 == 0.
  *   x    [d_in] fp16, 16-byte aligned.       y [d_out] fp16 out, 16-byte aligned.
  *   ws   sig_workspace_bytes(SIG_OP_SPARSE_GEMV, d_in, d_out, 0) bytes, 256-byte
- *        aligned, zeroed once by sig_workspace_init (or allocated zeroed).
+ *        aligned, zeroed once by sig_workspace_init (or allocated zeroed); it
+ *        holds the partial sums of the cluster groups of a column tile and
+ *        their arrival counters.  When the size is 0 (one group per tile, as
+ *        for d_out >= 37888) ws may be NULL.
  * The result is bit-identical from run to run (fixed-order split-K reduction;
  * no floating-point atomics).  An empty mask writes y = 0.
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d_in < 1, d_in > SIG_MAX_D_IN, d_out < 8,
@@ -202,10 +207,12 @@ SIG_API int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float*
 /*
  * Batched N:M activation GEMM (Block Q-Sparse, Q-Sparse rebuttal A2):
  *   Y = (M . X) WT, M the per-row n:m mask of X (as sparsify_nm), float32
- *   accumulation on the tensor cores, Y rounded once to fp16.
+ *   accumulation on the tensor cores, Y rounded once to fp16.  When n == m
+ *   the GEMM runs on X directly.
  *   X  [rows x K] fp16 row-major.   WT [K x N] fp16 row-major.   Y [rows x N] fp16 out.
- *   rows % 128 == 0, K % 64 == 0, N % 128 == 0, K % m == 0; 1 <= n <= m <= 32.
- *   ws sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows) bytes (holds the masked X).
+ *   rows % 128 == 0, K % 64 == 0, N % 128 == 0; m in {1,2,4,8,16,32}, 1 <= n <= m.
+ *   ws sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows) bytes (the masked X;
+ *      not touched when n == m, so it may be NULL then).
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ARG, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE,
  *         SIG_ERR_CUDA.
  */
@@ -220,13 +227,16 @@ SIG_API int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16
  * budget is fixed at start-up, or plain C code with no allocator.  The pages
  * have no counterpart to this entry point; it computes exactly what
  * gated_mlp_sparse computes, with the same arguments minus ws / ws_bytes.
- * Its scratch lives in one device array of SIG_NOALLOC_SCRATCH_BYTES inside
- * the library, which every GPU that loads the library holds until the
- * process exits.  It allocates nothing and calls no allocating routine.
+ * Its scratch (split-K partial sums and arrival counters of the two
+ * products, and the fp16 hidden vector h when h_out is NULL) lives in one
+ * device array of SIG_NOALLOC_SCRATCH_BYTES (2 MiB) inside the library,
+ * which every GPU that loads the library holds until the process exits.  It
+ * allocates nothing and calls no allocating routine.
  *   - A call whose scratch (sig_workspace_bytes(SIG_OP_GATED_MLP, d_model,
- *     d_ff, 0)) exceeds SIG_NOALLOC_SCRATCH_BYTES returns SIG_ERR_SHAPE with
- *     nothing enqueued.  Llama-2-7B (4096, 11008) and Llama-70B (8192, 28672)
- *     MLP shapes fit.
+ *     d_ff, 0)) would exceed SIG_NOALLOC_SCRATCH_BYTES returns SIG_ERR_SHAPE
+ *     with nothing enqueued.  Every shape gated_mlp_sparse accepts
+ *     (d_model, d_ff <= SIG_MAX_D_IN) needs at most 1927 KiB, so it fits;
+ *     larger sizes are rejected with SIG_ERR_SHAPE like everywhere else.
  *   - Every call shares the array and finds the previous call's contents in
  *     it; the call clears what must start at zero.  Calls that overlap on the
  *     GPU (other streams, other host threads) race; serialise them.

@@ -64,7 +64,7 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
       return plan_gated(d_in, d_out).total;
     case SIG_OP_NM_GEMM:
       if (rows < 1 || d_in < 1) return 0;
-      return round_up((size_t)rows * (size_t)d_in * 2, 256);
+      return round_up((size_t)rows * (size_t)d_in * 2, 256);   // the masked activation block
   }
   return 0;
 }
@@ -118,8 +118,8 @@ int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t*
   if (sh != SIG_OK) return sh;
   if (!aligned16(WT) || !aligned16(x) || !aligned16(y)) return SIG_ERR_ALIGN;
   const GemvPlan p = plan_gemv(d_in, d_out, false);
-  if (ws == nullptr || ws_bytes < p.ws_bytes()) return SIG_ERR_WORKSPACE;
-  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
   GemvLaunch a{};
   a.WT = WT; a.x = x; a.t = t; a.idx = idx; a.nnz = nnz;
   a.d_in = (int)d_in; a.d_out = (int)d_out; a.y = y; a.ws = ws;
@@ -174,6 +174,8 @@ int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT, 
       K % m != 0 || rows > (1 << 24) || K > (1 << 20) || N > (1 << 20))
     return SIG_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(WT) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  if (n == m)   // every entry kept: the plain tensor-core GEMM on X
+    return cuda_status(launch_gemm_f16(X, WT, Y, (int)rows, (int)N, (int)K, (cudaStream_t)stream));
   const size_t need = sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows);
   if (ws == nullptr || ws_bytes < need) return SIG_ERR_WORKSPACE;
   if (!aligned256(ws)) return SIG_ERR_ALIGN;

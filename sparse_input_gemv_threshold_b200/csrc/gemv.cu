@@ -5,19 +5,25 @@
 // entry are skipped).  WT is stored transposed (d_in x d_out, row-major), so a
 // kept input i costs one contiguous row of 2*d_out bytes.
 //
-// One launch does everything:
-//   1. every CTA ballots the whole activation (it sits in L2), packs the mask
-//      into shared words and prefix-scans their popcounts, which gives nnz and
-//      the CTA's equal share [lo, hi) of the ascending kept-row list; each
-//      thread then places its ranks by a binary search over the word prefixes;
-//   2. the CTA streams its share of kept rows for its 256-column tile with
-//      16-byte non-allocating loads, 8 rows in flight per warp (each with its
-//      activation value, a broadcast load), fp32 FMA;
-//   3. the 8 warps' sums meet in shared memory, the CTA writes one fp32 partial
-//      per column, and the CTA that arrives last for the tile (a counter in
-//      the workspace) adds the partials in split order and stores fp16.
-// The reduction order is fixed, so y is bit-identical from run to run; no
-// floating-point atomics are used and no CTA ever waits for another.
+// Launch shape: C x S CTAs of 256 threads, about four per SM on every SM.  A
+// CTA owns a 256-output column tile (one warp spans it with 16-byte lanes) and
+// one of S <= 32 equal slices of the ascending kept-row list.  One launch does
+// everything:
+//   1. every CTA ballots the whole activation (it sits in L2) into shared
+//      mask words with fp16 SIMD compares against the threshold rounded up to
+//      fp16 (exact for fp16 inputs), prefix-sums the words' popcounts (one
+//      barrier) to get nnz, its slice [lo, hi) and each word's first rank;
+//      the warps then place the slice's rows in parallel, one word per warp
+//      and one bit per lane (rank = word prefix + popcount of the lower bits);
+//   2. 8 warps stream the slice's rows of the tile, 8 rows in flight per warp:
+//      16-byte non-allocating loads with an L2 evict-first policy, the
+//      activation value riding along as a broadcast load, fp32 FMA;
+//   3. the warps' sums meet in shared memory (fixed order), the CTA writes one
+//      partial per column, and the CTA that arrives last for the tile (an
+//      atomic counter) loads the S partials in one batch, adds them in slice
+//      order and stores fp16.
+// No floating-point atomics and no spin-waits; y is bit-identical from run to
+// run.
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,6 +33,11 @@ namespace sig {
 
 namespace {
 
+constexpr int kThreads = kGemvThreads;        // 256
+constexpr int kWarps = kThreads / 32;         // 8
+constexpr int kTile = kGemvTile;              // 256 outputs per CTA
+constexpr int kMaxS = kGemvMaxSplits;         // 32
+
 struct KArgs {
   const uint16_t* WT;
   const uint16_t* WT2;
@@ -35,23 +46,78 @@ struct KArgs {
   const int32_t* idx;
   const int32_t* nnz;
   float t;
-  int d_in, d_out, S, cap;
-  uint32_t words_bytes;   // shared bytes of the mask words (and of their prefixes)
-  uint32_t union_bytes;   // shared bytes of the words + prefixes / reduction union
+  int d_in, d_out, S, chunk;
+  uint32_t words_bytes;   // shared bytes of the mask words (and again of their prefixes)
+  uint32_t union_bytes;   // shared bytes of words + prefixes / the warp-sum buffer
   uint16_t* y;
   uint32_t* mask_out;
-  unsigned* counters;
-  float* partials;        // [S][d_out] (then [S][d_out] for the second product)
+  unsigned* counters;     // [C]
+  float* partials;        // [S][d_out] (then the same again for the second product)
 };
 
+// 8 mask bits for the 8 fp16 values in v: |x| >= th (th = t rounded up to
+// fp16; NaN never passes an ordered compare).
+__device__ __forceinline__ uint32_t thresh_bits8(const uint4& v, __half2 th2) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t b = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t m = __hge2_mask(__habs2(*reinterpret_cast<const __half2*>(&w[q])), th2);
+    b |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
+  }
+  return b;
+}
+
+// All mask words of x into words[] (bit i%32 of word i/32 is m_i).
+template <int MODE>
+__device__ __forceinline__ void build_words(const KArgs& a, int nwords, uint32_t* words) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int d_in = a.d_in;
+  constexpr int kPass = kThreads * 8;
+  const float t = a.t;
+  const __half2 th2 = __half2half2(t <= 0.f ? __float2half(0.f) : __float2half_ru(t));
+  for (int base0 = 0; base0 < d_in; base0 += kPass * 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {   // eight passes' loads in flight together
+      const int e0 = base0 + u * kPass + tid * 8;
+      v[u] = e0 + 8 <= d_in ? __ldg(reinterpret_cast<const uint4*>(a.x + e0))
+                            : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int base = base0 + u * kPass;
+      if (base >= d_in) break;                         // uniform across the block
+      const int e0 = base + tid * 8;
+      uint32_t b = 0;
+      if (MODE == MASK_THRESH && e0 + 8 <= d_in) {
+        b = thresh_bits8(v[u], th2);
+      } else {
+        for (int k = 0; k < 8; ++k) {
+          const int i = e0 + k;
+          if (i >= d_in) break;
+          const float m = fabsf(h2f(e0 + 8 <= d_in ? lane_half(v[u], k) : a.x[i]));
+          const bool keep = MODE == MASK_THRESH_SCALED ? __fmul_rn(m, __ldg(a.scale + i)) >= t
+                                                       : m >= t;
+          b |= (keep ? 1u : 0u) << k;
+        }
+      }
+      uint32_t w = b << (8 * (lane & 3));
+      w |= __shfl_xor_sync(kFull, w, 1);
+      w |= __shfl_xor_sync(kFull, w, 2);
+      const int wi = (base >> 5) + (tid >> 2);
+      if ((lane & 3) == 0 && wi < nwords) words[wi] = w;
+    }
+  }
+}
+
 template <int MODE, bool DUAL, int EPI>
-__global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSM)
+__global__ void __launch_bounds__(kThreads, 4)
 sgemv_kernel(const KArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ int scan_scratch[kGemvThreads / 32 + 1];
+  __shared__ int warp_tot[kWarps];
   __shared__ int s_last;
 
-  constexpr int kWarps = kGemvThreads / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, s = blockIdx.y;
   const int d_in = a.d_in, d_out = a.d_out, S = a.S;
@@ -63,122 +129,144 @@ sgemv_kernel(const KArgs a) {
   pdl_trigger();
   pdl_wait();
 
-  // ---- 1. which rows does this CTA own? --------------------------------
-  int n_rows = 0;
+  // ---- 1. this CTA's slice [lo, hi) of the kept-row list ---------------
+  int lo = 0, hi = 0, nwords = 0;
   if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED) {
-    const float t = a.t;
-    const float* scale = a.scale;
-    build_mask_words<kGemvThreads>(a.x, d_in, words, [&](uint16_t h, int i) {
-      const float m = fabsf(h2f(h));
-      if (MODE == MASK_THRESH_SCALED) return __fmul_rn(m, __ldg(scale + i)) >= t;
-      return m >= t;
-    });
+    nwords = (d_in + 31) >> 5;
+    build_words<MODE>(a, nwords, words);
     __syncthreads();
-    const int nwords = (d_in + 31) >> 5;
-    const int per = (nwords + kGemvThreads - 1) / kGemvThreads;
+    // exclusive prefix of the words' popcounts, thread-contiguous word ranges
+    const int per = (nwords + kThreads - 1) / kThreads;
     const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
     int cnt = 0;
     for (int w = w0; w < w1; ++w) cnt += __popc(words[w]);
-    int total;
-    int r = block_exclusive_scan<kGemvThreads>(cnt, scan_scratch, &total);
-    for (int w = w0; w < w1; ++w) {   // exclusive kept-count before each word
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int v = warp_tot[w];
+      before += w < warp ? v : 0;
+      total += v;
+    }
+    int r = before + incl - cnt;
+    for (int w = w0; w < w1; ++w) {            // first rank held by each word
       wpre[w] = r;
       r += __popc(words[w]);
     }
-    __syncthreads();
-    const int lo = (int)(((long long)s * total) / S);
-    const int hi = (int)(((long long)(s + 1) * total) / S);
-    n_rows = hi - lo;
-    // Every thread places its own ranks: the word holding rank lo + j is the
-    // last one whose prefix is <= that rank; __fns finds the bit inside it.
-    for (int j = tid; j < n_rows; j += kGemvThreads) {
-      const int rank = lo + j;
-      int a0 = 0, a1 = nwords - 1;
-      while (a0 < a1) {
-        const int mid = (a0 + a1 + 1) >> 1;
-        if (wpre[mid] <= rank) a0 = mid; else a1 = mid - 1;
-      }
-      sidx[j] = a0 * 32 + (int)__fns(words[a0], 0, rank - wpre[a0] + 1);
-    }
+    lo = (int)(((long long)s * total) / S);
+    hi = (int)(((long long)(s + 1) * total) / S);
     if (a.mask_out != nullptr && c == 0 && s == 0)
-      for (int w = tid; w < nwords; w += kGemvThreads) a.mask_out[w] = words[w];
+      for (int w = tid; w < nwords; w += kThreads) a.mask_out[w] = words[w];
+    __syncthreads();
   } else if (MODE == MASK_IDX) {
     const int total = min(max(__ldg(a.nnz), 0), d_in);
-    const int lo = (int)(((long long)s * total) / S);
-    const int hi = (int)(((long long)(s + 1) * total) / S);
-    n_rows = hi - lo;
-    for (int j = tid; j < n_rows; j += kGemvThreads) {
-      const int i = __ldg(a.idx + lo + j);
-      sidx[j] = (unsigned)i < (unsigned)d_in ? i : -1;
-    }
+    lo = (int)(((long long)s * total) / S);
+    hi = (int)(((long long)(s + 1) * total) / S);
   } else {  // MASK_DENSE
-    const int lo = (int)(((long long)s * d_in) / S);
-    const int hi = (int)(((long long)(s + 1) * d_in) / S);
-    n_rows = hi - lo;
-    for (int j = tid; j < n_rows; j += kGemvThreads) sidx[j] = lo + j;
+    lo = (int)(((long long)s * d_in) / S);
+    hi = (int)(((long long)(s + 1) * d_in) / S);
   }
-  __syncthreads();
+  const int n_rows = hi - lo;
 
-  // ---- 2. stream the kept rows of this column tile ----------------------
-  const int col = c * kGemvTile + lane * 8;
+  // first word that can hold rank lo: the last one whose prefix is <= lo
+  int w_first = 0;
+  if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED) {
+    int a1 = nwords - 1;
+    while (w_first < a1) {
+      const int mid = (w_first + a1 + 1) >> 1;
+      if (wpre[mid] <= lo) w_first = mid; else a1 = mid - 1;
+    }
+  }
+
+  // ---- 2. stream the slice's rows of this column tile ------------------
+  const int col = c * kTile + lane * 8;
   const bool col_ok = col < d_out;
+  const uint16_t* wp = a.WT + col;
+  const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
+  const uint64_t pol = l2_evict_first_policy();
   float acc[8], acc2[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) { acc[k] = 0.f; acc2[k] = 0.f; }
+  constexpr int U = DUAL ? 4 : 8;
 
-  if (col_ok) {
-    const uint16_t* wp = a.WT + col;
-    const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
-    const uint64_t pol = l2_evict_first_policy();
-    // U rows per warp in flight; the last batch is predicated, so a warp with
-    // only a few rows still issues all of its loads at once.
-    constexpr int U = DUAL ? 4 : 8;
-    for (int j0 = warp; j0 < n_rows; j0 += kWarps * U) {
-      uint4 v[U], v2[U];
-      uint16_t xh[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + kWarps * u;
-        const int r = j < n_rows ? sidx[j] : -1;
-        if (r >= 0) {
-          // the activation rides along with its weight row: both in flight
-          xh[u] = __ldg(a.x + r);
-          v[u] = ld_stream_v4(wp + (size_t)r * d_out, pol);
-          if (DUAL) v2[u] = ld_stream_v4(wp2 + (size_t)r * d_out, pol);
-        } else {
-          xh[u] = 0;
-          v[u] = make_uint4(0, 0, 0, 0);
-          if (DUAL) v2[u] = make_uint4(0, 0, 0, 0);
+  for (int cb = 0; cb < n_rows; cb += a.chunk) {
+    const int c_lo = lo + cb, c_hi = min(hi, c_lo + a.chunk), cn = c_hi - c_lo;
+    if (MODE != MASK_DENSE) {
+      if (cb > 0) __syncthreads();   // the previous chunk's rows are no longer read
+      if (MODE == MASK_IDX) {
+        for (int j = tid; j < cn; j += kThreads) {
+          const int i = __ldg(a.idx + c_lo + j);
+          sidx[j] = (unsigned)i < (unsigned)d_in ? i : -1;
+        }
+      } else {
+        // one word per warp, one bit per lane: rank = word's first rank +
+        // popcount of the word's lower bits
+        for (int w = w_first + warp; w < nwords; w += kWarps) {
+          const int base = wpre[w];
+          if (base >= c_hi) break;                     // uniform across the warp
+          const uint32_t bits = words[w];
+          const int rk = base + __popc(bits & ((1u << lane) - 1u));
+          if (((bits >> lane) & 1u) && rk >= c_lo && rk < c_hi) sidx[rk - c_lo] = w * 32 + lane;
         }
       }
+      __syncthreads();
+    }
+    if (col_ok) {
+      for (int j0 = warp; j0 < cn; j0 += kWarps * U) {
+        uint4 v[U], v2[U];
+        uint16_t xh[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const float xv = h2f(xh[u]);
-        fma8(acc, v[u], xv);
-        if (DUAL) fma8(acc2, v2[u], xv);
+        for (int u = 0; u < U; ++u) {
+          const int j = j0 + kWarps * u;
+          const int r = j < cn ? (MODE == MASK_DENSE ? c_lo + j : sidx[j]) : -1;
+          if (r >= 0) {
+            xh[u] = __ldg(a.x + r);
+            v[u] = ld_stream_v4(wp + (size_t)r * d_out, pol);
+            if (DUAL) v2[u] = ld_stream_v4(wp2 + (size_t)r * d_out, pol);
+          } else {
+            xh[u] = 0;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (DUAL) v2[u] = make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const float xv = h2f(xh[u]);
+          fma8(acc, v[u], xv);
+          if (DUAL) fma8(acc2, v2[u], xv);
+        }
       }
     }
   }
 
   // ---- 3. CTA partial, then the last arriver finishes the tile ---------
-  // The words region is free again (only the prologue read it).
+  __syncthreads();   // the words / prefixes region becomes the warp-sum buffer
   float* red = reinterpret_cast<float*>(smem);
-  float4* red4 = reinterpret_cast<float4*>(red + warp * kGemvTile + lane * 8);
-  red4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  red4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  if (DUAL) {
-    float4* r2 = reinterpret_cast<float4*>(red + kWarps * kGemvTile + warp * kGemvTile + lane * 8);
-    r2[0] = make_float4(acc2[0], acc2[1], acc2[2], acc2[3]);
-    r2[1] = make_float4(acc2[4], acc2[5], acc2[6], acc2[7]);
+  {
+    float4* r4 = reinterpret_cast<float4*>(red + warp * kTile + lane * 8);
+    r4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    r4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    if (DUAL) {
+      float4* q4 = reinterpret_cast<float4*>(red + kWarps * kTile + warp * kTile + lane * 8);
+      q4[0] = make_float4(acc2[0], acc2[1], acc2[2], acc2[3]);
+      q4[1] = make_float4(acc2[4], acc2[5], acc2[6], acc2[7]);
+    }
   }
   __syncthreads();
   float p = 0.f, p2 = 0.f;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    p += red[w * kGemvTile + tid];
-    if (DUAL) p2 += red[kWarps * kGemvTile + w * kGemvTile + tid];
+    p += red[w * kTile + tid];
+    if (DUAL) p2 += red[kWarps * kTile + w * kTile + tid];
   }
-  const int colr = c * kGemvTile + tid;
+  const int colr = c * kTile + tid;
   const bool colr_ok = colr < d_out;
 
   auto finish = [&](float g, float u) {
@@ -194,7 +282,6 @@ sgemv_kernel(const KArgs a) {
     if (colr_ok) finish(p, p2);
     return;
   }
-
   if (colr_ok) {
     a.partials[(size_t)s * d_out + colr] = p;
     if (DUAL) a.partials[(size_t)S * d_out + (size_t)s * d_out + colr] = p2;
@@ -206,59 +293,48 @@ sgemv_kernel(const KArgs a) {
   if (!s_last) return;
   __threadfence();
   if (colr_ok) {
-    // all loads of a batch in flight together, then added in split order
-    constexpr int B = DUAL ? 16 : 32;
+    // every partial of the column in flight at once, then added in slice order
+    float pg[kMaxS], pu[kMaxS];
+#pragma unroll
+    for (int q = 0; q < kMaxS; ++q) {
+      const bool ok = q < S;
+      pg[q] = ok ? __ldcg(a.partials + (size_t)q * d_out + colr) : 0.f;
+      if (DUAL) pu[q] = ok ? __ldcg(a.partials + (size_t)S * d_out + (size_t)q * d_out + colr) : 0.f;
+    }
     float g = 0.f, u = 0.f;
-    for (int q0 = 0; q0 < S; q0 += B) {
-      float pg[B], pu[B];
 #pragma unroll
-      for (int k = 0; k < B; ++k) {
-        const bool ok = q0 + k < S;
-        pg[k] = ok ? __ldcg(a.partials + (size_t)(q0 + k) * d_out + colr) : 0.f;
-        if (DUAL) pu[k] = ok ? __ldcg(a.partials + (size_t)S * d_out + (size_t)(q0 + k) * d_out + colr) : 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < B; ++k) {
-        g += pg[k];
-        if (DUAL) u += pu[k];
-      }
+    for (int q = 0; q < kMaxS; ++q) {
+      g += pg[q];
+      if (DUAL) u += pu[q];
     }
     finish(g, u);
   }
   if (tid == 0) a.counters[c] = 0u;  // ready for the next call on this workspace
 }
 
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
 template <int MODE, bool DUAL, int EPI>
 cudaError_t launch_t(const GemvPlan& p, const KArgs& k, cudaStream_t stream) {
   auto fn = sgemv_kernel<MODE, DUAL, EPI>;
-  static bool attr_done = false;  // per instantiation; the attribute is per function
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         96 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
-  return launch_pdl(fn, dim3(p.C, p.S), dim3(kGemvThreads), p.smem, stream, k);
+  cudaError_t e =
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(fn, dim3(p.C, p.S), dim3(kThreads), p.smem, stream, k);
 }
-
-size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
 GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual) {
   GemvPlan p{};
-  p.C = (int)((d_out + kGemvTile - 1) / kGemvTile);
-  int S = std::max(1, (kNumSMs * kGemvCtasPerSM) / p.C);
-  S = (int)std::min<int64_t>(S, std::max<int64_t>(1, d_in));
-  S = std::max<int>(S, (int)((d_in + kIdxCap - 1) / kIdxCap));
-  p.S = S;
-  p.cap = (int)((d_in + S - 1) / S);
+  p.C = (int)((d_out + kTile - 1) / kTile);
+  p.S = std::max(1, std::min(kMaxS, (kNumSMs * kGemvCtasPerSM) / p.C));
+  p.chunk = (int)std::max<int64_t>(1, std::min<int64_t>((d_in + p.S - 1) / p.S, kIdxCap));
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
-  const size_t red = (size_t)(kGemvThreads / 32) * kGemvTile * 4 * (dual ? 2 : 1);
-  const size_t uni = std::max(2 * words, red);
-  p.smem = uni + round_up((size_t)p.cap * 4, 16);
-  p.counters = round_up((size_t)p.C * 4, 256);
-  p.partials = S > 1 ? round_up((size_t)S * d_out * 4 * (dual ? 2 : 1), 256) : 0;
+  const size_t red = (size_t)kWarps * kTile * 4 * (dual ? 2 : 1);
+  p.smem = std::max(2 * words, red) + round_up((size_t)p.chunk * 4, 16);
+  p.counters = p.S > 1 ? round_up((size_t)p.C * 4, 256) : 0;
+  p.partials = p.S > 1 ? round_up((size_t)p.S * d_out * 4 * (dual ? 2 : 1), 256) : 0;
   return p;
 }
 
@@ -266,14 +342,15 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
                         cudaStream_t stream) {
   KArgs k{};
   k.WT = a.WT; k.WT2 = a.WT2; k.x = a.x; k.scale = a.scale; k.idx = a.idx; k.nnz = a.nnz;
-  k.t = a.t; k.d_in = a.d_in; k.d_out = a.d_out; k.S = p.S; k.cap = p.cap;
+  k.t = a.t; k.d_in = a.d_in; k.d_out = a.d_out; k.S = p.S; k.chunk = p.chunk;
   const size_t words = round_up((size_t)((a.d_in + 31) / 32) * 4, 16);
-  const size_t red = (size_t)(kGemvThreads / 32) * kGemvTile * 4 * (epi == EPI_SILU_MUL ? 2 : 1);
+  const size_t red = (size_t)kWarps * kTile * 4 * (epi == EPI_SILU_MUL ? 2 : 1);
   k.words_bytes = (uint32_t)words;
   k.union_bytes = (uint32_t)std::max(2 * words, red);
   k.y = a.y; k.mask_out = a.mask_out;
   k.counters = reinterpret_cast<unsigned*>(a.ws);
-  k.partials = reinterpret_cast<float*>(reinterpret_cast<char*>(a.ws) + p.counters);
+  k.partials = a.ws != nullptr ? reinterpret_cast<float*>(reinterpret_cast<char*>(a.ws) + p.counters)
+                               : nullptr;
   if (epi == EPI_SILU_MUL) {
     if (mode != MASK_DENSE) return cudaErrorInvalidValue;
     return launch_t<MASK_DENSE, true, EPI_SILU_MUL>(p, k, stream);

@@ -11,9 +11,10 @@ namespace sig {
 
 constexpr int kNumSMs = 148;         // B200: 2 dies x 74 SMs
 constexpr int kGemvThreads = 256;    // 8 warps
+constexpr int kGemvCtasPerSM = 4;    // residency the grid is sized for
 constexpr int kGemvTile = 256;       // output columns per CTA (one warp spans them)
-constexpr int kGemvCtasPerSM = 4;    // target residency; grid = C x S <= 148 * 4
-constexpr int kIdxCap = 4096;        // largest slice of the index list per CTA
+constexpr int kGemvMaxSplits = 32;   // K-splits per column tile (one batch of partial loads)
+constexpr int kIdxCap = 4096;        // rows of a slice staged in shared memory at once
 constexpr int kMaxDIn = 131072;
 constexpr int kMaxTopkD = 131072;    // top-k stages its keys in the cluster's shared memory
 
@@ -50,11 +51,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 struct GemvPlan {
   int C;              // column tiles
-  int S;              // K-splits (slices of the kept-row list)
-  int cap;            // most rows one slice can hold
+  int S;              // K-splits (slices of the kept-row list), <= kGemvMaxSplits
+  int chunk;          // rows of a slice staged in shared memory at once
   size_t smem;        // dynamic shared memory per CTA
-  size_t counters;    // workspace bytes for arrival counters
-  size_t partials;    // workspace bytes for float32 partial sums
+  size_t counters;    // workspace bytes for per-tile arrival counters
+  size_t partials;    // workspace bytes for the slices' float32 partial sums
   size_t ws_bytes() const { return counters + partials; }
 };
 

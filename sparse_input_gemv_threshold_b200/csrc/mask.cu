@@ -10,6 +10,7 @@
 //  - row norms (||W^down_i|| of RaNA Eqn. 12), float64 accumulation.
 #include "common.cuh"
 #include "internal.h"
+#include "nm_select.cuh"
 
 #include <cooperative_groups.h>
 
@@ -267,53 +268,6 @@ topk_cluster_kernel(const uint16_t* __restrict__ x, int d, int k, int chunk, uin
   cluster.sync();   // no CTA leaves while another may still read its shared memory
 }
 
-// One bitonic stage (K = run length, J = partner distance) and the ones after
-// it; template recursion keeps every index a compile-time constant.
-template <int M, int K, int J>
-__device__ __forceinline__ void bitonic_stage(uint32_t (&s)[M]) {
-#pragma unroll
-  for (int i = 0; i < M; ++i) {
-    const int l = i ^ J;
-    if (l > i) {
-      const uint32_t a = s[i], b = s[l];
-      const bool desc = (i & K) == 0;      // the final merge leaves s descending
-      s[i] = desc ? max(a, b) : min(a, b);
-      s[l] = desc ? min(a, b) : max(a, b);
-    }
-  }
-  if constexpr (J > 1) bitonic_stage<M, K, J / 2>(s);
-  else if constexpr (K < M) bitonic_stage<M, K * 2, K>(s);
-}
-
-// Bits of the n largest composites among M unique composites (bit j for c[j]).
-// M <= 8: count, for each entry, the entries ranked above it.  M >= 16: sort a
-// copy descending with a bitonic network; the n-th largest is the minimum of
-// the first n, and an entry is kept when it is at least that.
-template <int M>
-__device__ __forceinline__ uint32_t select_top_n(const uint32_t (&c)[M], int n) {
-  uint32_t bits = 0;
-  if constexpr (M <= 8) {
-#pragma unroll
-    for (int j = 0; j < M; ++j) {
-      int rank = 0;
-#pragma unroll
-      for (int l = 0; l < M; ++l) rank += c[l] > c[j] ? 1 : 0;
-      bits |= (rank < n ? 1u : 0u) << j;
-    }
-  } else {
-    uint32_t s[M];
-#pragma unroll
-    for (int j = 0; j < M; ++j) s[j] = c[j];
-    bitonic_stage<M, 2, 1>(s);
-    uint32_t thr = 0xffffffffu;
-#pragma unroll
-    for (int j = 0; j < M; ++j) thr = min(thr, j < n ? s[j] : 0xffffffffu);
-#pragma unroll
-    for (int j = 0; j < M; ++j) bits |= (c[j] >= thr ? 1u : 0u) << j;
-  }
-  return bits;
-}
-
 // One thread per 32-entry mask word of one row (m divides 32, so blocks of m
 // never straddle a word).  Inside a block the entries are ranked by the
 // composite (magnitude key << 5 | (31 - position)): unique, larger magnitude
@@ -336,35 +290,13 @@ nm_mask_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, uint1
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     q[i] = i * 8 < cnt ? __ldg(reinterpret_cast<const uint4*>(src) + i) : make_uint4(0, 0, 0, 0);
-  uint32_t bits = 0;
-#pragma unroll
-  for (int b0 = 0; b0 < 32; b0 += M) {
-    if (b0 < cnt) {
-      uint32_t comp[M];
-#pragma unroll
-      for (int j = 0; j < M; ++j)
-        comp[j] = (mag_key(lane_half(q[(b0 + j) >> 3], (b0 + j) & 7)) << 5) | (uint32_t)(31 - j);
-      bits |= select_top_n<M>(comp, n) << b0;
-    }
-  }
+  const uint32_t bits = nm_word_bits<M>(q, n, cnt);
   if (mask_bits != nullptr) mask_bits[row * wpr + w] = bits;
   if (X_masked != nullptr) {
     uint16_t* dst = X_masked + row * (int64_t)d + e0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (i * 8 < cnt) {
-        const uint32_t wv[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
-        uint32_t p[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int a = i * 8 + 2 * k;
-          const uint32_t lo = ((bits >> a) & 1u) ? (wv[k] & 0xffffu) : 0u;
-          const uint32_t hi = ((bits >> (a + 1)) & 1u) ? (wv[k] & 0xffff0000u) : 0u;
-          p[k] = lo | hi;
-        }
-        reinterpret_cast<uint4*>(dst)[i] = make_uint4(p[0], p[1], p[2], p[3]);
-      }
-    }
+    for (int i = 0; i < 4; ++i)
+      if (i * 8 < cnt) reinterpret_cast<uint4*>(dst)[i] = nm_apply(q[i], bits, i);
   }
 }
 

@@ -5,10 +5,11 @@
 // they run this layer: a plugin inside a host program that owns all device
 // memory through its own pool, a serving loop with a fixed memory budget
 // decided at start-up, or C code with no allocator of its own.  This entry
-// point takes only the inputs and outputs.  Its scratch (split-K partial sums,
-// arrival counters and the fp16 hidden vector h) lives in one file-scope
-// device array of SIG_NOALLOC_SCRATCH_BYTES that every GPU which loads the
-// library holds until the process exits.
+// point takes only the inputs and outputs.  Its scratch (split-K partial sums
+// and arrival counters of the two products, and the fp16 hidden vector h when
+// h_out is NULL) lives in one file-scope device array of
+// SIG_NOALLOC_SCRATCH_BYTES (2 MiB) that every GPU which loads the library
+// holds until the process exits.
 //
 // The array is shared by every call on a device and keeps the last call's
 // contents, so each call first clears the counters that must start at zero.
@@ -79,9 +80,11 @@ extern "C" int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT,
   char* base = static_cast<char*>(scratch);
   cudaStream_t st = (cudaStream_t)stream;
 
-  // the arrival counters of both products must start at zero
-  if (cudaMemsetAsync(base, 0, g.up.counters, st) != cudaSuccess) return SIG_ERR_CUDA;
-  if (cudaMemsetAsync(base + g.off_down, 0, g.down.counters, st) != cudaSuccess)
+  // arrival counters (if the products use any) must start at zero
+  if (g.up.counters > 0 && cudaMemsetAsync(base, 0, g.up.counters, st) != cudaSuccess)
+    return SIG_ERR_CUDA;
+  if (g.down.counters > 0 &&
+      cudaMemsetAsync(base + g.off_down, 0, g.down.counters, st) != cudaSuccess)
     return SIG_ERR_CUDA;
 
   uint16_t* h = h_out != nullptr ? h_out : reinterpret_cast<uint16_t*>(base + g.off_h);

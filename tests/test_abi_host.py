@@ -70,13 +70,14 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_sizes(lib):
     ws = lib.sig_workspace_bytes
-    assert ws(1, 4096, 4096, 0) > 0
+    assert ws(1, 4096, 4096, 0) > 0           # split-K partials and per-tile counters
     assert ws(1, 4096, 4096, 0) % 256 == 0
+    assert ws(1, 64, 131072, 0) == 0          # > 296 column tiles: one slice, no partials
     assert ws(1, 0, 4096, 0) == 0            # invalid shape
     assert ws(1, 4096, 12, 0) == 0           # d_out % 8
     assert ws(2, 8192, 0, 0) == 0            # top-k needs none
     assert ws(3, 4096, 11008, 0) > ws(1, 11008, 4096, 0)
-    assert ws(4, 1024, 1024, 4096) == 4096 * 1024 * 2
+    assert ws(4, 1024, 1024, 4096) == 4096 * 1024 * 2   # the masked activation block
     assert ws(77, 1, 1, 1) == 0
 
 
@@ -94,6 +95,7 @@ def test_sparse_gemv_validation(lib):
     assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE_ODD, FAKE, big, None) == ALIGN
     assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE, None, big, None) == WORKSPACE
     need = lib.sig_workspace_bytes(1, 64, 64, 0)
+    assert need > 0
     assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE, FAKE, need - 1, None) == WORKSPACE
     assert f(FAKE, 64, 64, FAKE, 0.0, None, None, FAKE, FAKE + 16, need, None) == ALIGN
 

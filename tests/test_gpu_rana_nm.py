@@ -41,14 +41,27 @@ def _rana_case(sig, mlp, t, what):
     ref = oracle.sparse_linear(mlp.WdT, h, m_strict)
     assert_within(y, ref["y64"], ref["bound"], what + " strict")
 
-    # end to end against the oracle's own h
+    # end to end against the oracle's own h.  g and u are float32 sums on the
+    # GPU: give each the product tolerance 2e-3 * sum|W x| and carry it through
+    # h = SiLU(g) u (dSiLU/dg = sigma(g) (1 + g (1 - sigma(g)))), plus one fp16
+    # ulp for the final rounding.
     full = oracle.gated_mlp(mlp.x, mlp.WgT, mlp.WuT, mlp.WdT, norms, t)
-    h_ref = full["h16"]
-    ulp = np.spacing(np.abs(h_ref)).astype(np.float64)
-    assert (np.abs(h.astype(np.float64) - h_ref.astype(np.float64)) <= ulp).all(), what + " h"
+    h_ref, g, u = full["h16"], full["g"], full["u"]
+    x64 = np.abs(mlp.x.astype(np.float64))
+    Bg = x64 @ np.abs(mlp.WgT.astype(np.float64))
+    Bu = x64 @ np.abs(mlp.WuT.astype(np.float64))
+    with np.errstate(over="ignore"):
+        sg = 1.0 / (1.0 + np.exp(-g))
+    dsilu = sg * (1.0 + g * (1.0 - sg))
+    tol_h = (np.spacing(np.abs(h_ref)).astype(np.float64)
+             + np.abs(dsilu * u) * 2e-3 * Bg + np.abs(g * sg) * 2e-3 * Bu)
+    dh = np.abs(h.astype(np.float64) - h_ref.astype(np.float64))
+    assert (dh <= tol_h).all(), (what + " h", int((dh > tol_h).sum()))
+    assert (dh <= np.spacing(np.abs(h_ref))).mean() > 0.999, what + " h mostly within 1 ulp"
     diff = np.flatnonzero(m_gpu != full["mask"])
     s_ref = full["s32"].astype(np.float64)
-    assert (np.abs(s_ref[diff] - t) <= 2.0 ** -10 * t).all(), what + " mask"
+    slack = tol_h[diff] * norms[diff].astype(np.float64) + 2.0 ** -10 * t
+    assert (np.abs(s_ref[diff] - t) <= slack).all(), what + " mask"
     extra = np.abs(mlp.WdT[diff].astype(np.float64) *
                    np.maximum(np.abs(h[diff]), np.abs(h_ref[diff])).astype(np.float64)[:, None]).sum(0)
     err = np.abs(y.astype(np.float64) - full["y64"])

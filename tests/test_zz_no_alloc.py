@@ -59,12 +59,23 @@ def test_noalloc_matches_gated_mlp_twice_in_a_row(sig):
     torch.cuda.synchronize()
 
 
-def test_noalloc_rejects_sizes_beyond_its_array(sig):
-    import ctypes
-    lib = sig._lib
-    fake = 1 << 40                      # never dereferenced: the size check comes first
-    d_model, d_ff = 65536, 131072       # scratch far above the array
-    assert sig.workspace_bytes(sig.OP_GATED_MLP, d_model, d_ff) > 2 << 20
-    st = lib.gated_mlp_sparse_noalloc(fake, fake, fake, fake, fake, d_model, d_ff,
-                                      ctypes.c_float(0.1), fake, None, None, None)
-    assert st == 2   # SIG_ERR_SHAPE
+def test_noalloc_rejects_sizes_beyond_its_maximum(sig):
+    """The largest accepted d_ff fits the 2 MiB array; one step beyond is
+    rejected with SIG_ERR_SHAPE.  Real (small) device buffers back every
+    pointer, so nothing could fault even if the size checks did not stop it."""
+    import torch
+    d_model, d_ff = 8, 131072 + 8
+    assert sig.workspace_bytes(sig.OP_GATED_MLP, d_model, 131072) <= 2 << 20
+    x = torch.zeros(d_model, dtype=torch.float16, device="cuda")
+    Wg = torch.zeros((d_model, d_ff), dtype=torch.float16, device="cuda")
+    Wu = torch.zeros_like(Wg)
+    Wd = torch.zeros((d_ff, d_model), dtype=torch.float16, device="cuda")
+    norms = torch.ones(d_ff, dtype=torch.float32, device="cuda")
+    with pytest.raises(sig.SigError) as e:
+        sig.gated_mlp_sparse_noalloc(x, Wg, Wu, Wd, norms, 0.1)
+    assert e.value.status == 2   # SIG_ERR_SHAPE
+    # the largest d_ff that is accepted runs (zero weights: y = 0)
+    Wg, Wu = Wg[:, :131072].contiguous(), Wu[:, :131072].contiguous()
+    Wd, norms = Wd[:131072].contiguous(), norms[:131072].contiguous()
+    y = sig.gated_mlp_sparse_noalloc(x, Wg, Wu, Wd, norms, 0.1)
+    assert not y.float().abs().sum().item()
