@@ -5,8 +5,10 @@
 Workload (one step): one Llama-2-7B decoder layer's seven projections at
 batch 1 (q, k, v, o 4096x4096; gate, up 4096->11008; down 11008->4096), fp16
 weights ~ N(0, 0.02^2), Laplace activations, TEAL-style magnitude threshold
-set at the 50 % quantile of |x|.  Each projection is one fused
-threshold -> compact -> split-K GEMV -> deterministic reduce launch.
+set at the 50 % quantile of |x|.  As in the model, q, k and v read one hidden
+state and gate and up another, so the step is four fused
+threshold -> compact -> split-K GEMV -> deterministic reduce launches:
+(q|k|v), o, (gate|up), down; a shared input is read and masked once.
 
 Metric: effective HBM GB/s = (kept weight rows + x + y bytes) / time, with
 inputs resident in HBM; three copies of the layer's weights rotate so that
@@ -55,7 +57,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--profile-case", default=None,
                     help="for ncu: run only this kernel case eagerly and exit "
-                         "(a Llama-2-7B projection name at 50%%, 'topk70b', 'rana' or 'nm2:4')")
+                         "(a Llama-2-7B projection name or launch group such as 'q|k|v' or "
+                         "'gate|up' at 50%%, 'topk70b' or 'nm2:4')")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     return ap.parse_args()
 
@@ -91,7 +94,8 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -271,16 +275,48 @@ def ncu_traffic_per_launch():
 # our implementation
 # ---------------------------------------------------------------------------
 
+# Projections that read the same input, in launch order.
+GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
+
+
+def layer_groups(projs):
+    by = {p.name: p for p in projs}
+    return [[by[n] for n in g] for g in GROUPS]
+
+
+def kept_count(p, sparsity):
+    return int((np.abs(p.x.astype(np.float32)) >= p.thresholds[sparsity]).sum())
+
+
 def kept_counts(projs, sparsity):
-    out = []
-    for p in projs:
-        t = p.thresholds[sparsity]
-        out.append(int((np.abs(p.x.astype(np.float32)) >= t).sum()))
-    return out
+    return [kept_count(p, sparsity) for p in projs]
 
 
-def algorithmic_bytes(projs, nnzs):
-    return sum(n * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out for p, n in zip(projs, nnzs))
+def group_bytes(group, nnz):
+    """Kept rows of every weight in the group + the shared x once + each y."""
+    dsum = sum(p.d_out for p in group)
+    return nnz * 2 * dsum + 2 * group[0].d_in + 2 * dsum
+
+
+def layer_bytes(groups, sparsity):
+    return sum(group_bytes(g, kept_count(g[0], sparsity)) for g in groups)
+
+
+def launch_group(sig, W, x, t, ys, ws, stream):
+    """One launch for every projection that reads x."""
+    if len(W) == 1:
+        sig.sparse_gemv(W[0], x, t=t, y=ys[0], ws=ws, stream=stream)
+    else:
+        sig.sparse_gemv_multi(W, x, t=t, ys=ys, ws=ws, stream=stream)
+
+
+def group_workspace(sig, group):
+    import torch
+    if len(group) == 1:
+        n = sig.workspace_bytes(sig.OP_SPARSE_GEMV, group[0].d_in, group[0].d_out)
+    else:
+        n = sig.workspace_bytes_multi([p.d_out for p in group], group[0].d_in)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device="cuda")
 
 
 def run_ours(args, rank, world, local):
@@ -288,22 +324,19 @@ def run_ours(args, rank, world, local):
     import sparse_input_gemv_threshold_b200 as sig
 
     stream = torch.cuda.Stream()
-    projs = workloads.llama2_7b(args.seed)
-    dev_x = [torch.from_numpy(p.x).cuda() for p in projs]
-    copies = []
-    for c in range(N_COPIES):
-        copies.append([torch.from_numpy(p.WT).cuda() if c == 0 else None for p in projs])
-    for c in range(1, N_COPIES):
-        copies[c] = [w.clone() for w in copies[0]]
-    ys = [torch.empty(p.d_out, dtype=torch.float16, device="cuda") for p in projs]
-    wss = [torch.zeros(sig.workspace_bytes(sig.OP_SPARSE_GEMV, p.d_in, p.d_out),
-                       dtype=torch.uint8, device="cuda") for p in projs]
+    projs = workloads.llama2_7b_layer(args.seed)
+    groups = layer_groups(projs)
+    gx = [torch.from_numpy(g[0].x).cuda() for g in groups]
+    first = [[torch.from_numpy(p.WT).cuda() for p in g] for g in groups]
+    copies = [first] + [[[w.clone() for w in g] for g in first] for _ in range(N_COPIES - 1)]
+    gys = [[torch.empty(p.d_out, dtype=torch.float16, device="cuda") for p in g] for g in groups]
+    gws = [group_workspace(sig, g) for g in groups]
 
     def step_fn(c, s):
         def f():
-            for j, p in enumerate(projs):
-                sig.sparse_gemv(copies[c][j], dev_x[j], t=p.thresholds[s], y=ys[j], ws=wss[j],
-                                stream=stream)
+            for gi, g in enumerate(groups):
+                launch_group(sig, copies[c][gi], gx[gi], g[0].thresholds[s], gys[gi], gws[gi],
+                             stream)
         return f
 
     def graphs_for(s):
@@ -311,8 +344,9 @@ def run_ours(args, rank, world, local):
 
     # ---- headline ----
     g50 = graphs_for(HEADLINE_SPARSITY)
-    nnz50 = kept_counts(projs, HEADLINE_SPARSITY)
-    bytes_step = algorithmic_bytes(projs, nnz50)
+    nnz50 = [kept_count(g[0], HEADLINE_SPARSITY) for g in groups]
+    bytes_step = layer_bytes(groups, HEADLINE_SPARSITY)
+    n_launch = len(groups)
     with ClockSampler(local) as clk:
         secs = time_steps(g50, args.steps, args.warmup, stream, world)
     clocks = clk.summary()
@@ -327,28 +361,29 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
         "config": {"workload": "llama2_7b_decode_layer_b1", "projections": "q,k,v,o 4096x4096; gate,up 4096->11008; down 11008->4096",
+                   "launches": "(q|k|v) o (gate|up) down: q,k,v share one input and one mask, gate,up another",
                    "batch": 1, "sparsity": HEADLINE_SPARSITY, "mask": "threshold |x|>=t, t=50% quantile of |x|",
                    "weights": "fp16 N(0,0.02^2), transposed (d_in x d_out)", "x": "fp16 Laplace(0,1)",
                    "seed": args.seed, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {N_COPIES} rotating weight copies, "
                          f"{N_COPIES * bytes_step / 1e6:.0f} MB of kept rows per rotation",
-                   "bytes_per_step": bytes_step, "nnz_per_projection": nnz50},
-        "gpu_launches": 7 * args.steps,
+                   "bytes_per_step": bytes_step, "nnz_per_launch": nnz50},
+        "gpu_launches": n_launch * args.steps,
         "clocks": clocks,
     }
-    us_launch = slow / args.steps / 7 * 1e6
+    us_launch = slow / args.steps / n_launch * 1e6
     traffic = ncu_traffic_per_launch()
     result["roofline"] = {
         "kernel": "sgemv_kernel (fused threshold + split-K GEMV + reduce)", "bound": "hbm",
-        "achieved": round(bytes_step / 7 / (us_launch * 1e-6) / 1e9, 1), "peak": hbm_peak,
+        "achieved": round(bytes_step / n_launch / (us_launch * 1e-6) / 1e9, 1), "peak": hbm_peak,
         "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
-        "frac": round(bytes_step / 7 / (us_launch * 1e-6) / 1e9 / hbm_peak, 4),
-        "traffic": traffic, "algorithmic_bytes_per_launch": bytes_step // 7,
+        "frac": round(bytes_step / n_launch / (us_launch * 1e-6) / 1e9 / hbm_peak, 4),
+        "traffic": traffic, "algorithmic_bytes_per_launch": bytes_step // n_launch,
         "avg_launch_us": round(us_launch, 3),
     }
 
     # ---- e2e through the public API with host buffers ----
-    result["e2e"] = e2e(args, projs, copies[0], ys, wss, stream, sig, world, bytes_step)
+    result["e2e"] = e2e(args, groups, copies[0], gys, gws, stream, sig, world, bytes_step)
 
     if not args.no_extras and rank == 0:
         extras = {}
@@ -357,8 +392,7 @@ def run_ours(args, rank, world, local):
         sweep = []
         for s in workloads.LLAMA2_SPARSITIES:
             gs = g50 if s == HEADLINE_SPARSITY else graphs_for(s)
-            nz = kept_counts(projs, s)
-            b = algorithmic_bytes(projs, nz)
+            b = layer_bytes(groups, s)
             sec = time_steps(gs, steps_x, 24, stream)
             us = sec / steps_x * 1e6
             sweep.append({"sparsity": s, "us_per_step": round(us, 2),
@@ -367,53 +401,77 @@ def run_ours(args, rank, world, local):
             if gs is not g50:
                 del gs
         extras["sweep_llama2_7b_layer"] = sweep
-        extras["per_projection_us_at_50"] = per_projection(projs, copies, dev_x, ys, wss, stream, sig,
-                                                           steps_x)
-        extras["cublas_dense_layer_us"] = cublas_dense(projs, copies, dev_x, stream, steps_x)
+        extras["per_launch_us_at_50"] = per_launch(groups, copies, gx, gys, gws, stream, sig,
+                                                   steps_x)
+        extras["seven_single_launches"] = seven_launches(groups, copies, gx, stream, sig, steps_x,
+                                                         bytes_step)
+        extras["cublas_dense_layer_us"] = cublas_dense(groups, copies, gx, stream, steps_x)
         del g50
         torch.cuda.synchronize()
-        for c in copies[1:]:
-            c.clear()
+        del copies[1:]
         torch.cuda.empty_cache()
         extras["topk_qsparse_70b"] = bench_topk(args, stream, sig, hbm_peak)
         extras["rana_gated_mlp"] = bench_rana(args, stream, sig, hbm_peak)
         extras["nm_gemm"] = bench_nm(args, stream, sig, bf16_peak)
         result["extras"] = extras
-        result["cpu_baseline"] = cpu_baseline(projs)
+        result["cpu_baseline"] = cpu_baseline(groups)
     return result
 
 
-def per_projection(projs, copies, dev_x, ys, wss, stream, sig, steps):
+def per_launch(groups, copies, gx, gys, gws, stream, sig, steps):
     out = {}
-    for j, p in enumerate(projs):
-        def f(c, j=j, p=p):
+    for gi, grp in enumerate(groups):
+        def f(c, gi=gi, grp=grp):
             def g():
-                sig.sparse_gemv(copies[c][j], dev_x[j], t=p.thresholds[HEADLINE_SPARSITY], y=ys[j],
-                                ws=wss[j], stream=stream)
+                launch_group(sig, copies[c][gi], gx[gi], grp[0].thresholds[HEADLINE_SPARSITY],
+                             gys[gi], gws[gi], stream)
             return g
         sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=48)
         sec = time_steps(sg, steps, 24, stream)
         us = sec / steps * 1e6
-        nnz = kept_counts([p], HEADLINE_SPARSITY)[0]
-        b = nnz * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out
-        out[p.name] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1)}
+        b = group_bytes(grp, kept_count(grp[0], HEADLINE_SPARSITY))
+        out["|".join(p.name for p in grp)] = {"us": round(us, 2),
+                                              "GBps": round(b / (us * 1e-6) / 1e9, 1)}
     return out
 
 
-def cublas_dense(projs, copies, dev_x, stream, steps):
-    """Dense fp16 GEMV through torch (cuBLAS), same shapes, same weight rotation."""
+def seven_launches(groups, copies, gx, stream, sig, steps, bytes_step):
+    """The same layer as seven single-weight launches (each re-reads and
+    re-masks its input), for comparison with the grouped launches."""
     import torch
-    outs = [torch.empty((1, p.d_out), dtype=torch.float16, device="cuda") for p in projs]
+    flat = [(gi, j, p) for gi, g in enumerate(groups) for j, p in enumerate(g)]
+    ys = [torch.empty(p.d_out, dtype=torch.float16, device="cuda") for _, _, p in flat]
+    wss = [torch.zeros(max(256, sig.workspace_bytes(sig.OP_SPARSE_GEMV, p.d_in, p.d_out)),
+                       dtype=torch.uint8, device="cuda") for _, _, p in flat]
 
     def f(c):
         def g():
-            for j in range(len(projs)):
-                torch.matmul(dev_x[j].view(1, -1), copies[c][j], out=outs[j])
+            for k, (gi, j, p) in enumerate(flat):
+                sig.sparse_gemv(copies[c][gi][j], gx[gi], t=p.thresholds[HEADLINE_SPARSITY],
+                                y=ys[k], ws=wss[k], stream=stream)
         return g
     sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=12)
     sec = time_steps(sg, steps, 24, stream)
     us = sec / steps * 1e6
-    dense_bytes = sum(p.d_in * p.d_out * 2 + 2 * p.d_in + 2 * p.d_out for p in projs)
+    return {"us_per_step": round(us, 2), "GBps_same_bytes": round(bytes_step / (us * 1e-6) / 1e9, 1)}
+
+
+def cublas_dense(groups, copies, gx, stream, steps):
+    """Dense fp16 GEMV through torch (cuBLAS), same shapes, same weight rotation."""
+    import torch
+    flat = [(gi, j, p) for gi, g in enumerate(groups) for j, p in enumerate(g)]
+    outs = [torch.empty((1, p.d_out), dtype=torch.float16, device="cuda") for _, _, p in flat]
+
+    def f(c):
+        def g():
+            for k, (gi, j, p) in enumerate(flat):
+                torch.matmul(gx[gi].view(1, -1), copies[c][gi][j], out=outs[k])
+        return g
+    sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=12)
+    sec = time_steps(sg, steps, 24, stream)
+    us = sec / steps * 1e6
+    dense_bytes = sum(sum(p.d_in * p.d_out * 2 + 2 * p.d_out for p in g) + 2 * g[0].d_in
+                      for g in groups)
     return {"us_per_step": round(us, 2), "GBps": round(dense_bytes / (us * 1e-6) / 1e9, 1)}
 
 
@@ -548,20 +606,21 @@ def bench_nm(args, stream, sig, bf16_peak):
     return out
 
 
-def e2e(args, projs, W, ys, wss, stream, sig, world, bytes_step):
+def e2e(args, groups, W, gys, gws, stream, sig, world, bytes_step):
     """Public binding calls with host buffers: pinned x in, y out, every step."""
     import torch
-    xh = [torch.from_numpy(p.x).pin_memory() for p in projs]
-    yh = [torch.empty(p.d_out, dtype=torch.float16).pin_memory() for p in projs]
-    xd = [torch.empty(p.d_in, dtype=torch.float16, device="cuda") for p in projs]
+    xh = [torch.from_numpy(g[0].x).pin_memory() for g in groups]
+    yh = [[torch.empty(p.d_out, dtype=torch.float16).pin_memory() for p in g] for g in groups]
+    xd = [torch.empty(g[0].d_in, dtype=torch.float16, device="cuda") for g in groups]
     steps = max(10, min(args.steps // 20, 1000))
 
     def step():
-        for j, p in enumerate(projs):
-            xd[j].copy_(xh[j], non_blocking=True)
-            sig.sparse_gemv(W[j], xd[j], t=p.thresholds[HEADLINE_SPARSITY], y=ys[j], ws=wss[j],
-                            stream=stream)
-            yh[j].copy_(ys[j], non_blocking=True)
+        for gi, g in enumerate(groups):
+            xd[gi].copy_(xh[gi], non_blocking=True)
+            launch_group(sig, W[gi], xd[gi], g[0].thresholds[HEADLINE_SPARSITY], gys[gi], gws[gi],
+                         stream)
+            for j in range(len(g)):
+                yh[gi][j].copy_(gys[gi][j], non_blocking=True)
     with torch.cuda.stream(stream):
         for _ in range(5):
             step()
@@ -577,10 +636,10 @@ def e2e(args, projs, W, ys, wss, stream, sig, world, bytes_step):
     sec = max_over_ranks(s.elapsed_time(e) / 1e3, world)
     return {"value": round(bytes_step * steps * world / sec / 1e9, 1), "unit": UNIT,
             "steps": steps, "us_per_step": round(sec / steps * 1e6, 2),
-            "h2d_bytes_per_step": sum(2 * p.d_in for p in projs),
-            "d2h_bytes_per_step": sum(2 * p.d_out for p in projs),
-            "note": "weights resident (model parameters); x copied in and y copied out per projection; "
-                    "eager binding calls, no graph"}
+            "h2d_bytes_per_step": sum(2 * g[0].d_in for g in groups),
+            "d2h_bytes_per_step": sum(2 * p.d_out for g in groups for p in g),
+            "note": "weights resident (model parameters); each launch's x copied in and its y's "
+                    "copied out; eager binding calls, no graph"}
 
 
 # ---------------------------------------------------------------------------
@@ -596,54 +655,55 @@ def _blas_threads():
         return os.cpu_count()
 
 
-def oracle_sample(projs, cols_per_proj, rng):
-    """Run the oracle on `cols_per_proj` output columns of every projection;
-    returns (algorithmic bytes of the sample, seconds)."""
+def oracle_sample(groups, cols_per_proj, rng):
+    """Run the oracle on `cols_per_proj` output columns of every projection,
+    one mask per shared input; returns (algorithmic bytes of the sample, seconds)."""
     import oracle
     b = 0
     t0 = time.perf_counter()
-    for p in projs:
-        cols = rng.choice(p.d_out, cols_per_proj, replace=False)
-        m = oracle.threshold_mask(p.x, p.thresholds[HEADLINE_SPARSITY])
-        oracle.sparse_linear(p.WT, p.x, m, cols=cols)
-        b += int(m.sum()) * 2 * cols_per_proj + 2 * p.d_in + 2 * cols_per_proj
+    for g in groups:
+        m = oracle.threshold_mask(g[0].x, g[0].thresholds[HEADLINE_SPARSITY])
+        for p in g:
+            cols = rng.choice(p.d_out, cols_per_proj, replace=False)
+            oracle.sparse_linear(p.WT, p.x, m, cols=cols)
+        b += int(m.sum()) * 2 * cols_per_proj * len(g) + 2 * g[0].d_in + 2 * cols_per_proj * len(g)
     return b, time.perf_counter() - t0
 
 
-def cpu_baseline(projs, budget_s=12.0):
+def cpu_baseline(groups, budget_s=12.0):
     rng = np.random.default_rng(0)
-    _, t1 = oracle_sample(projs, 256, rng)                      # warm-up and calibration
+    _, t1 = oracle_sample(groups, 256, rng)                      # warm-up and calibration
     reps = max(1, int(budget_s / max(t1, 1e-3)))
     tot_b, tot_t = 0, 0.0
     for _ in range(reps):
-        b, t = oracle_sample(projs, 256, rng)
+        b, t = oracle_sample(groups, 256, rng)
         tot_b += b
         tot_t += t
     return {"value": round(tot_b / tot_t / 1e9, 3), "unit": UNIT, "cores": _blas_threads(),
             "kind": "oracle",
             "sample": f"{reps} passes over the 7 projections, 256 random output columns each, "
-                      f"50% threshold mask, numpy float64 ({tot_t:.1f} s)"}
+                      f"one 50% threshold mask per shared input, numpy float64 ({tot_t:.1f} s)"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    projs = workloads.llama2_7b(args.seed)
+    groups = layer_groups(workloads.llama2_7b_layer(args.seed))
     rng = np.random.default_rng(1)
     # size the per-step sample so that warmup + steps stay within ~90 s
-    _, t64 = oracle_sample(projs, 64, rng)
+    _, t64 = oracle_sample(groups, 64, rng)
     per_step = 90.0 / max(1, args.steps + args.warmup)
     cols = int(max(1, min(4096, 64 * per_step / max(t64, 1e-6))))
     for _ in range(args.warmup):
-        oracle_sample(projs, cols, rng)
+        oracle_sample(groups, cols, rng)
     tot_b, tot_t = 0, 0.0
     for _ in range(args.steps):
-        b, t = oracle_sample(projs, cols, rng)
+        b, t = oracle_sample(groups, cols, rng)
         tot_b += b
         tot_t += t
     value = tot_b / tot_t / 1e9
     sample = (f"each step: the 7 projections' oracle product on {cols} random output columns "
-              f"(50% threshold mask, numpy float64)")
+              f"(one 50% threshold mask per shared input, numpy float64)")
     return {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(tot_t / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
@@ -664,20 +724,22 @@ def profile_case(args):
     import sparse_input_gemv_threshold_b200 as sig
     torch.cuda.set_device(0)
     case = args.profile_case
-    if case in dict((n, 0) for n, _, _ in workloads.LLAMA2_7B_PROJECTIONS):
-        (p,) = workloads.llama2_7b(args.seed, names=(case,))
-        copies = max(2, math.ceil(4 * 126e6 / (p.d_in * p.d_out * 2)))
-        W = [torch.from_numpy(p.WT).cuda()]
-        W += [W[0].clone() for _ in range(copies - 1)]
-        x = torch.from_numpy(p.x).cuda()
-        y = torch.empty(p.d_out, dtype=torch.float16, device="cuda")
-        ws = torch.zeros(sig.workspace_bytes(sig.OP_SPARSE_GEMV, p.d_in, p.d_out), dtype=torch.uint8,
-                         device="cuda")
+    group_names = {"|".join(g): g for g in GROUPS}
+    group_names.update({n: (n,) for n, _, _ in workloads.LLAMA2_7B_PROJECTIONS})
+    if case in group_names:
+        by = {p.name: p for p in workloads.llama2_7b_layer(args.seed)}
+        grp = [by[n] for n in group_names[case]]
+        wbytes = sum(p.d_in * p.d_out * 2 for p in grp)
+        copies = max(2, math.ceil(4 * 126e6 / wbytes))
+        W = [[torch.from_numpy(p.WT).cuda() for p in grp]]
+        W += [[w.clone() for w in W[0]] for _ in range(copies - 1)]
+        x = torch.from_numpy(grp[0].x).cuda()
+        ys = [torch.empty(p.d_out, dtype=torch.float16, device="cuda") for p in grp]
+        ws = group_workspace(sig, grp)
         for i in range(args.launches):
-            sig.sparse_gemv(W[i % copies], x, t=p.thresholds[HEADLINE_SPARSITY], y=y, ws=ws)
-        nnz = kept_counts([p], HEADLINE_SPARSITY)[0]
+            launch_group(sig, W[i % copies], x, grp[0].thresholds[HEADLINE_SPARSITY], ys, ws, None)
         info = {"case": case, "launches": args.launches, "copies": copies,
-                "algorithmic_bytes_per_launch": nnz * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out}
+                "algorithmic_bytes_per_launch": group_bytes(grp, kept_count(grp[0], HEADLINE_SPARSITY))}
     elif case == "nm2:4":
         WT, X = workloads.nm_tokens(args.seed)
         Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()

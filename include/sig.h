@@ -176,6 +176,35 @@ SIG_API int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out,
                 uint16_t* y, void* ws, size_t ws_bytes, sig_stream_t stream);
 
 /*
+ * Sparse-input GEMV for several weights that read the same input, in one
+ * launch: y_p = W_p (m . x) for p < n_mat, with ONE mask m.  In a transformer
+ * block the query, key and value projections read the same hidden state, and
+ * so do the gate and up projections of the MLP; TEAL thresholds that shared
+ * hidden state once (TEAL README, Abstract), and the product is that of
+ * sparse_gemv for each weight (RaNA rebuttal, Q5.1).  The mask is computed
+ * once per CTA for all the weights and their column tiles share the grid.
+ *   n_mat    1 .. 4.
+ *   WT, y    HOST arrays of n_mat DEVICE pointers: WT[p] [d_in x d_out[p]]
+ *            fp16 row-major, y[p] [d_out[p]] fp16 out; all 16-byte aligned.
+ *   d_out    HOST array of n_mat sizes, each a multiple of 8.
+ *   x, t, idx, nnz   as sparse_gemv (one mask for all the weights).
+ *   ws       sig_workspace_bytes_multi(n_mat, d_out, d_in) bytes, 256-byte
+ *            aligned, zeroed once (it may be NULL when that size is 0).
+ * Results are bit-identical to n_mat separate sparse_gemv calls only up to
+ * the split-K order (the grid is planned for all the weights together).
+ * Errors: SIG_ERR_NULL, SIG_ERR_ARG (n_mat), SIG_ERR_SHAPE, SIG_ERR_ALIGN,
+ *         SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
+ */
+SIG_API int sparse_gemv_multi(int n_mat, const uint16_t* const* WT, const int64_t* d_out,
+                              int64_t d_in, const uint16_t* x, float t,
+                              const int32_t* idx, const int32_t* nnz,
+                              uint16_t* const* y, void* ws, size_t ws_bytes,
+                              sig_stream_t stream);
+
+/* Workspace bytes of sparse_gemv_multi (0 for invalid arguments or none needed). */
+SIG_API size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in);
+
+/*
  * Gated MLP with the RaNA neuron masker (RaNA rebuttal, Q3, Eqn. 12):
  *   g = GateProj(x), u = UpProj(x)       (dense GEMVs, float32 accumulation)
  *   h = fp16(SiLU(g) * u)                (SiLU(z) = z / (1 + exp(-z)), float32)

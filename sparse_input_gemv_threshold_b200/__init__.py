@@ -22,6 +22,7 @@ __all__ = [
     "MAX_D_IN", "abi_version", "workspace_bytes", "workspace", "sparsify_threshold",
     "sparsify_topk", "sparsify_nm", "sparse_gemv", "gated_mlp_sparse", "row_norms",
     "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
+    "sparse_gemv_multi", "workspace_bytes_multi",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -46,6 +47,8 @@ _SIGNATURES = {
     "nm_act_gemm": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _sz, _p]),
     "sig_take_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _p]),
     "gated_mlp_sparse_noalloc": (_i32, [_p, _p, _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p]),
+    "sparse_gemv_multi": (_i32, [_i32, _p, _p, _i64, _p, _f32, _p, _p, _p, _p, _sz, _p]),
+    "sig_workspace_bytes_multi": (_sz, [_i32, _p, _i64]),
 }
 
 
@@ -183,6 +186,42 @@ def sparse_gemv(WT, x, t: float = 0.0, idx=None, nnz=None, y=None, ws=None, stre
         _ptr(WT), d_in, d_out, _ptr(x), float(t), _ptr(idx), _ptr(nnz), _ptr(y),
         _ptr(ws), ws.numel(), _stream(stream)))
     return y
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def workspace_bytes_multi(d_outs, d_in: int) -> int:
+    arr = (ctypes.c_int64 * len(d_outs))(*d_outs)
+    return int(_lib.sig_workspace_bytes_multi(len(d_outs), arr, d_in))
+
+
+def sparse_gemv_multi(WTs, x, t: float = 0.0, idx=None, nnz=None, ys=None, ws=None, stream=None):
+    """y_p = W_p (m . x) for weights that read the same x, one mask, one launch."""
+    _need(x, torch.float16, "x")
+    d_in = x.numel()
+    for i, w in enumerate(WTs):
+        _need(w, torch.float16, f"WT[{i}]", x.device)
+        if w.shape[0] != d_in:
+            raise ValueError("every WT must have d_in rows")
+    d_outs = [int(w.shape[1]) for w in WTs]
+    if ys is None:
+        ys = [torch.empty(n, dtype=torch.float16, device=x.device) for n in d_outs]
+    if ws is None:
+        nbytes = workspace_bytes_multi(d_outs, d_in)
+        key = (x.device, _stream(stream), "multi", d_in, tuple(d_outs))
+        with _ws_lock:
+            ws = _ws_cache.get(key)
+            if ws is None:
+                ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=x.device)
+                _ws_cache[key] = ws
+    wt_arr, y_arr = _ptr_array(WTs), _ptr_array(ys)
+    d_arr = (ctypes.c_int64 * len(d_outs))(*d_outs)
+    _check("sparse_gemv_multi", _lib.sparse_gemv_multi(
+        len(WTs), wt_arr, d_arr, d_in, _ptr(x), float(t), _ptr(idx), _ptr(nnz), y_arr,
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return ys
 
 
 def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,

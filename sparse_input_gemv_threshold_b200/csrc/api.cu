@@ -121,8 +121,46 @@ int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t*
   if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
   if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
   GemvLaunch a{};
-  a.WT = WT; a.x = x; a.t = t; a.idx = idx; a.nnz = nnz;
-  a.d_in = (int)d_in; a.d_out = (int)d_out; a.y = y; a.ws = ws;
+  a.WT[0] = WT; a.y[0] = y; a.d_out[0] = (int)d_out;
+  a.x = x; a.t = t; a.idx = idx; a.nnz = nnz; a.d_in = (int)d_in; a.ws = ws;
+  return cuda_status(launch_gemv(idx == nullptr ? MASK_THRESH : MASK_IDX, EPI_STORE, p, a,
+                                 (cudaStream_t)stream));
+}
+
+size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in) {
+  if (n_mat < 1 || n_mat > kGemvMaxMat || d_out == nullptr) return 0;
+  for (int i = 0; i < n_mat; ++i)
+    if (check_gemv_shape(d_in, d_out[i]) != SIG_OK) return 0;
+  return plan_gemv_multi(d_in, d_out, n_mat, false).ws_bytes();
+}
+
+int sparse_gemv_multi(int n_mat, const uint16_t* const* WT, const int64_t* d_out, int64_t d_in,
+                      const uint16_t* x, float t, const int32_t* idx, const int32_t* nnz,
+                      uint16_t* const* y, void* ws, size_t ws_bytes, sig_stream_t stream) {
+  if (WT == nullptr || d_out == nullptr || y == nullptr || x == nullptr) return SIG_ERR_NULL;
+  if (idx != nullptr && nnz == nullptr) return SIG_ERR_NULL;
+  if (n_mat < 1 || n_mat > kGemvMaxMat) return SIG_ERR_ARG;
+  int64_t total = 0;
+  for (int i = 0; i < n_mat; ++i) {
+    if (WT[i] == nullptr || y[i] == nullptr) return SIG_ERR_NULL;
+    const int sh = check_gemv_shape(d_in, d_out[i]);
+    if (sh != SIG_OK) return sh;
+    if (!aligned16(WT[i]) || !aligned16(y[i])) return SIG_ERR_ALIGN;
+    total += d_out[i];
+  }
+  if (total > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
+  if (!aligned16(x)) return SIG_ERR_ALIGN;
+  const GemvPlan p = plan_gemv_multi(d_in, d_out, n_mat, false);
+  if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
+  GemvLaunch a{};
+  a.n_mat = n_mat;
+  for (int i = 0; i < n_mat; ++i) {
+    a.WT[i] = WT[i];
+    a.y[i] = y[i];
+    a.d_out[i] = (int)d_out[i];
+  }
+  a.x = x; a.t = t; a.idx = idx; a.nnz = nnz; a.d_in = (int)d_in; a.ws = ws;
   return cuda_status(launch_gemv(idx == nullptr ? MASK_THRESH : MASK_IDX, EPI_STORE, p, a,
                                  (cudaStream_t)stream));
 }
@@ -147,14 +185,15 @@ int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT
   uint16_t* h = h_out != nullptr ? h_out : reinterpret_cast<uint16_t*>(base + g.off_h);
 
   GemvLaunch up{};
-  up.WT = WgT; up.WT2 = WuT; up.x = x; up.d_in = (int)d_model; up.d_out = (int)d_ff;
-  up.y = h; up.ws = base;
+  up.WT[0] = WgT; up.WT2 = WuT; up.y[0] = h; up.d_out[0] = (int)d_ff;
+  up.x = x; up.d_in = (int)d_model; up.ws = base;
   cudaError_t e = launch_gemv(MASK_DENSE, EPI_SILU_MUL, g.up, up, (cudaStream_t)stream);
   if (e != cudaSuccess) return SIG_ERR_CUDA;
 
   GemvLaunch dn{};
-  dn.WT = WdT; dn.x = h; dn.scale = down_norms; dn.t = t; dn.d_in = (int)d_ff;
-  dn.d_out = (int)d_model; dn.y = y; dn.mask_out = mask_out; dn.ws = base + g.off_down;
+  dn.WT[0] = WdT; dn.y[0] = y; dn.d_out[0] = (int)d_model;
+  dn.x = h; dn.scale = down_norms; dn.t = t; dn.d_in = (int)d_ff; dn.mask_out = mask_out;
+  dn.ws = base + g.off_down;
   return cuda_status(launch_gemv(MASK_THRESH_SCALED, EPI_STORE, g.down, dn, (cudaStream_t)stream));
 }
 

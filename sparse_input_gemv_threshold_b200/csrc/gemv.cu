@@ -7,7 +7,9 @@
 //
 // Launch shape: C x S CTAs of 256 threads, about four per SM on every SM.  A
 // CTA owns a 256-output column tile (one warp spans it with 16-byte lanes) and
-// one of S <= 32 equal slices of the ascending kept-row list.  One launch does
+// one of S <= 32 equal slices of the ascending kept-row list.  Up to four
+// weights that read the same input (q, k, v; gate, up) share one launch and
+// one mask: their column tiles are laid end to end.  One launch does
 // everything:
 //   1. every CTA ballots the whole activation (it sits in L2) into shared
 //      mask words with fp16 SIMD compares against the threshold rounded up to
@@ -39,20 +41,27 @@ constexpr int kTile = kGemvTile;              // 256 outputs per CTA
 constexpr int kMaxS = kGemvMaxSplits;         // 32
 
 struct KArgs {
-  const uint16_t* WT;
-  const uint16_t* WT2;
+  // weights that share the input and its mask: column tiles [tile0[p],
+  // tile0[p+1]) belong to weight p, whose columns start at col0[p] in the
+  // concatenated partial-sum space of d_out_total columns
+  const uint16_t* WT[kGemvMaxMat];
+  uint16_t* y[kGemvMaxMat];
+  int d_out[kGemvMaxMat];
+  int tile0[kGemvMaxMat + 1];
+  int col0[kGemvMaxMat];
+  int n_mat, d_out_total;
+  const uint16_t* WT2;    // dual partner of WT[0] (gate/up)
   const uint16_t* x;
   const float* scale;
   const int32_t* idx;
   const int32_t* nnz;
   float t;
-  int d_in, d_out, S, chunk;
+  int d_in, S, chunk;
   uint32_t words_bytes;   // shared bytes of the mask words (and again of their prefixes)
   uint32_t union_bytes;   // shared bytes of words + prefixes / the warp-sum buffer
-  uint16_t* y;
   uint32_t* mask_out;
   unsigned* counters;     // [C]
-  float* partials;        // [S][d_out] (then the same again for the second product)
+  float* partials;        // [S][d_out_total] (then the same again for the second product)
 };
 
 // 8 mask bits for the 8 fp16 values in v: |x| >= th (th = t rounded up to
@@ -111,16 +120,16 @@ __device__ __forceinline__ void build_words(const KArgs& a, int nwords, uint32_t
   }
 }
 
-template <int MODE, bool DUAL, int EPI>
+template <int MODE, bool DUAL, int EPI, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 4)
-sgemv_kernel(const KArgs a) {
+sgemv_kernel(const __grid_constant__ KArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_tot[kWarps];
   __shared__ int s_last;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = blockIdx.x, s = blockIdx.y;
-  const int d_in = a.d_in, d_out = a.d_out, S = a.S;
+  const int cg = blockIdx.x, s = blockIdx.y;   // global column tile, slice
+  const int d_in = a.d_in, S = a.S;
 
   uint32_t* words = reinterpret_cast<uint32_t*>(smem);
   int* wpre = reinterpret_cast<int*>(smem + a.words_bytes);
@@ -162,7 +171,7 @@ sgemv_kernel(const KArgs a) {
     }
     lo = (int)(((long long)s * total) / S);
     hi = (int)(((long long)(s + 1) * total) / S);
-    if (a.mask_out != nullptr && c == 0 && s == 0)
+    if (a.mask_out != nullptr && cg == 0 && s == 0)
       for (int w = tid; w < nwords; w += kThreads) a.mask_out[w] = words[w];
     __syncthreads();
   } else if (MODE == MASK_IDX) {
@@ -186,9 +195,14 @@ sgemv_kernel(const KArgs a) {
   }
 
   // ---- 2. stream the slice's rows of this column tile ------------------
+  int pm = 0;                                  // the weight this tile belongs to
+  if (MULTI)
+    while (pm + 1 < a.n_mat && cg >= a.tile0[pm + 1]) ++pm;
+  const int c = cg - a.tile0[pm];              // tile within that weight
+  const int d_out = a.d_out[pm];
   const int col = c * kTile + lane * 8;
   const bool col_ok = col < d_out;
-  const uint16_t* wp = a.WT + col;
+  const uint16_t* wp = a.WT[pm] + col;
   const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
   const uint64_t pol = l2_evict_first_policy();
   float acc[8], acc2[8];
@@ -266,15 +280,21 @@ sgemv_kernel(const KArgs a) {
     p += red[w * kTile + tid];
     if (DUAL) p2 += red[kWarps * kTile + w * kTile + tid];
   }
-  const int colr = c * kTile + tid;
-  const bool colr_ok = colr < d_out;
+  // the tile's weight again (kept out of registers through the main loop)
+  int pe = 0;
+  if (MULTI)
+    while (pe + 1 < a.n_mat && cg >= a.tile0[pe + 1]) ++pe;
+  const int colr = (cg - a.tile0[pe]) * kTile + tid;
+  const bool colr_ok = colr < a.d_out[pe];
+  uint16_t* __restrict__ Y = a.y[pe];
+  const int dtot = a.d_out_total;
 
   auto finish = [&](float g, float u) {
     if (EPI == EPI_STORE) {
-      a.y[colr] = f2h_rn(g);
+      Y[colr] = f2h_rn(g);
     } else {
       const float sg = g / (1.0f + expf(-g));
-      a.y[colr] = f2h_rn(sg * u);
+      Y[colr] = f2h_rn(sg * u);
     }
   };
 
@@ -282,41 +302,47 @@ sgemv_kernel(const KArgs a) {
     if (colr_ok) finish(p, p2);
     return;
   }
+  const size_t pcol = (size_t)a.col0[pe] + colr;   // column in the partial-sum space
   if (colr_ok) {
-    a.partials[(size_t)s * d_out + colr] = p;
-    if (DUAL) a.partials[(size_t)S * d_out + (size_t)s * d_out + colr] = p2;
+    a.partials[(size_t)s * dtot + pcol] = p;
+    if (DUAL) a.partials[(size_t)S * dtot + (size_t)s * dtot + pcol] = p2;
   }
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(a.counters + c, 1u) == (unsigned)(S - 1));
+  if (tid == 0) s_last = (atomicAdd(a.counters + cg, 1u) == (unsigned)(S - 1));
   __syncthreads();
   if (!s_last) return;
   __threadfence();
   if (colr_ok) {
-    // every partial of the column in flight at once, then added in slice order
-    float pg[kMaxS], pu[kMaxS];
-#pragma unroll
-    for (int q = 0; q < kMaxS; ++q) {
-      const bool ok = q < S;
-      pg[q] = ok ? __ldcg(a.partials + (size_t)q * d_out + colr) : 0.f;
-      if (DUAL) pu[q] = ok ? __ldcg(a.partials + (size_t)S * d_out + (size_t)q * d_out + colr) : 0.f;
-    }
+    // the partials of the column in flight together (all of them for S <= 16
+    // single, 8 per batch for the dual product), then added in slice order
+    constexpr int B = DUAL ? 8 : 16;
+    const float* pp = a.partials + pcol;
     float g = 0.f, u = 0.f;
+    for (int q0 = 0; q0 < S; q0 += B) {
+      float pg[B], pu[B];
 #pragma unroll
-    for (int q = 0; q < kMaxS; ++q) {
-      g += pg[q];
-      if (DUAL) u += pu[q];
+      for (int k = 0; k < B; ++k) {
+        const bool ok = q0 + k < S;
+        pg[k] = ok ? __ldcg(pp + (size_t)(q0 + k) * dtot) : 0.f;
+        if (DUAL) pu[k] = ok ? __ldcg(pp + (size_t)(S + q0 + k) * dtot) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        g += pg[k];
+        if (DUAL) u += pu[k];
+      }
     }
     finish(g, u);
   }
-  if (tid == 0) a.counters[c] = 0u;  // ready for the next call on this workspace
+  if (tid == 0) a.counters[cg] = 0u;  // ready for the next call on this workspace
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-template <int MODE, bool DUAL, int EPI>
+template <int MODE, bool DUAL, int EPI, bool MULTI = false>
 cudaError_t launch_t(const GemvPlan& p, const KArgs& k, cudaStream_t stream) {
-  auto fn = sgemv_kernel<MODE, DUAL, EPI>;
+  auto fn = sgemv_kernel<MODE, DUAL, EPI, MULTI>;
   cudaError_t e =
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return e;
@@ -325,35 +351,65 @@ cudaError_t launch_t(const GemvPlan& p, const KArgs& k, cudaStream_t stream) {
 
 }  // namespace
 
-GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual) {
+GemvPlan plan_gemv_multi(int64_t d_in, const int64_t* d_out, int n_mat, bool dual) {
   GemvPlan p{};
-  p.C = (int)((d_out + kTile - 1) / kTile);
-  p.S = std::max(1, std::min(kMaxS, (kNumSMs * kGemvCtasPerSM) / p.C));
+  int64_t total = 0;
+  p.C = 0;
+  for (int i = 0; i < n_mat; ++i) {
+    p.C += (int)((d_out[i] + kTile - 1) / kTile);
+    total += d_out[i];
+  }
+  p.S = std::max(1, std::min(kMaxS, (kNumSMs * kGemvCtasPerSM) / std::max(1, p.C)));
   p.chunk = (int)std::max<int64_t>(1, std::min<int64_t>((d_in + p.S - 1) / p.S, kIdxCap));
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)kWarps * kTile * 4 * (dual ? 2 : 1);
   p.smem = std::max(2 * words, red) + round_up((size_t)p.chunk * 4, 16);
   p.counters = p.S > 1 ? round_up((size_t)p.C * 4, 256) : 0;
-  p.partials = p.S > 1 ? round_up((size_t)p.S * d_out * 4 * (dual ? 2 : 1), 256) : 0;
+  p.partials = p.S > 1 ? round_up((size_t)p.S * total * 4 * (dual ? 2 : 1), 256) : 0;
   return p;
+}
+
+GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual) {
+  return plan_gemv_multi(d_in, &d_out, 1, dual);
 }
 
 cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& a,
                         cudaStream_t stream) {
+  if (a.n_mat < 1 || a.n_mat > kGemvMaxMat) return cudaErrorInvalidValue;
+  if (epi == EPI_SILU_MUL && a.n_mat != 1) return cudaErrorInvalidValue;
   KArgs k{};
-  k.WT = a.WT; k.WT2 = a.WT2; k.x = a.x; k.scale = a.scale; k.idx = a.idx; k.nnz = a.nnz;
-  k.t = a.t; k.d_in = a.d_in; k.d_out = a.d_out; k.S = p.S; k.chunk = p.chunk;
+  k.n_mat = a.n_mat;
+  int tiles = 0, cols = 0;
+  for (int i = 0; i < a.n_mat; ++i) {
+    k.WT[i] = a.WT[i];
+    k.y[i] = a.y[i];
+    k.d_out[i] = a.d_out[i];
+    k.tile0[i] = tiles;
+    k.col0[i] = cols;
+    tiles += (a.d_out[i] + kTile - 1) / kTile;
+    cols += a.d_out[i];
+  }
+  k.tile0[a.n_mat] = tiles;
+  k.d_out_total = cols;
+  if (tiles != p.C) return cudaErrorInvalidValue;
+  k.WT2 = a.WT2; k.x = a.x; k.scale = a.scale; k.idx = a.idx; k.nnz = a.nnz;
+  k.t = a.t; k.d_in = a.d_in; k.S = p.S; k.chunk = p.chunk;
   const size_t words = round_up((size_t)((a.d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)kWarps * kTile * 4 * (epi == EPI_SILU_MUL ? 2 : 1);
   k.words_bytes = (uint32_t)words;
   k.union_bytes = (uint32_t)std::max(2 * words, red);
-  k.y = a.y; k.mask_out = a.mask_out;
+  k.mask_out = a.mask_out;
   k.counters = reinterpret_cast<unsigned*>(a.ws);
   k.partials = a.ws != nullptr ? reinterpret_cast<float*>(reinterpret_cast<char*>(a.ws) + p.counters)
                                : nullptr;
   if (epi == EPI_SILU_MUL) {
     if (mode != MASK_DENSE) return cudaErrorInvalidValue;
     return launch_t<MASK_DENSE, true, EPI_SILU_MUL>(p, k, stream);
+  }
+  if (a.n_mat > 1) {
+    if (mode == MASK_THRESH) return launch_t<MASK_THRESH, false, EPI_STORE, true>(p, k, stream);
+    if (mode == MASK_IDX) return launch_t<MASK_IDX, false, EPI_STORE, true>(p, k, stream);
+    return cudaErrorInvalidValue;
   }
   switch (mode) {
     case MASK_THRESH: return launch_t<MASK_THRESH, false, EPI_STORE>(p, k, stream);

@@ -15,6 +15,7 @@ constexpr int kGemvCtasPerSM = 4;    // residency the grid is sized for
 constexpr int kGemvTile = 256;       // output columns per CTA (one warp spans them)
 constexpr int kGemvMaxSplits = 32;   // K-splits per column tile (one batch of partial loads)
 constexpr int kIdxCap = 4096;        // rows of a slice staged in shared memory at once
+constexpr int kGemvMaxMat = 4;       // weights that can share one input in one launch
 constexpr int kMaxDIn = 131072;
 constexpr int kMaxTopkD = 131072;    // top-k stages its keys in the cluster's shared memory
 
@@ -60,6 +61,7 @@ struct GemvPlan {
 };
 
 GemvPlan plan_gemv(int64_t d_in, int64_t d_out, bool dual);
+GemvPlan plan_gemv_multi(int64_t d_in, const int64_t* d_out, int n_mat, bool dual);
 
 // Workspace layout of the gated MLP: the dual (gate, up) product's counters and
 // partials, then the down product's, then the fp16 hidden vector h.
@@ -80,17 +82,19 @@ inline GatedPlan plan_gated(int64_t d_model, int64_t d_ff) {
 }
 
 struct GemvLaunch {
-  const uint16_t* WT;
-  const uint16_t* WT2;     // second weight for the dual (gate, up) product
-  const uint16_t* x;
-  const float* scale;      // MASK_THRESH_SCALED
-  const int32_t* idx;      // MASK_IDX
-  const int32_t* nnz;      // MASK_IDX
-  float t;
-  int d_in, d_out;
-  uint16_t* y;             // output (y, or h for EPI_SILU_MUL)
-  uint32_t* mask_out;      // nullable: written by one CTA
-  void* ws;                // plan.ws_bytes() bytes, counters zero on entry
+  int n_mat = 1;                         // weights sharing the input and its mask
+  const uint16_t* WT[kGemvMaxMat] = {};  // each d_in x d_out[i], row-major
+  uint16_t* y[kGemvMaxMat] = {};         // outputs (y, or h for EPI_SILU_MUL)
+  int d_out[kGemvMaxMat] = {};
+  const uint16_t* WT2 = nullptr;         // second weight of the dual (gate, up) product
+  const uint16_t* x = nullptr;
+  const float* scale = nullptr;          // MASK_THRESH_SCALED
+  const int32_t* idx = nullptr;          // MASK_IDX
+  const int32_t* nnz = nullptr;          // MASK_IDX
+  float t = 0.f;
+  int d_in = 0;
+  uint32_t* mask_out = nullptr;          // nullable: written by one CTA
+  void* ws = nullptr;                    // plan.ws_bytes() bytes, counters zero on entry
 };
 
 cudaError_t launch_gemv(int mode, int epi, const GemvPlan& plan, const GemvLaunch& a,

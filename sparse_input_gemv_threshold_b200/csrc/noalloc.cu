@@ -89,12 +89,13 @@ extern "C" int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT,
 
   uint16_t* h = h_out != nullptr ? h_out : reinterpret_cast<uint16_t*>(base + g.off_h);
   GemvLaunch up{};
-  up.WT = WgT; up.WT2 = WuT; up.x = x; up.d_in = (int)d_model; up.d_out = (int)d_ff;
-  up.y = h; up.ws = base;
+  up.WT[0] = WgT; up.WT2 = WuT; up.y[0] = h; up.d_out[0] = (int)d_ff;
+  up.x = x; up.d_in = (int)d_model; up.ws = base;
   if (launch_gemv(MASK_DENSE, EPI_SILU_MUL, g.up, up, st) != cudaSuccess) return SIG_ERR_CUDA;
   GemvLaunch dn{};
-  dn.WT = WdT; dn.x = h; dn.scale = down_norms; dn.t = t; dn.d_in = (int)d_ff;
-  dn.d_out = (int)d_model; dn.y = y; dn.mask_out = mask_out; dn.ws = base + g.off_down;
+  dn.WT[0] = WdT; dn.y[0] = y; dn.d_out[0] = (int)d_model;
+  dn.x = h; dn.scale = down_norms; dn.t = t; dn.d_in = (int)d_ff; dn.mask_out = mask_out;
+  dn.ws = base + g.off_down;
   if (launch_gemv(MASK_THRESH_SCALED, EPI_STORE, g.down, dn, st) != cudaSuccess)
     return SIG_ERR_CUDA;
   return SIG_OK;

@@ -121,6 +121,25 @@ def test_mask_validation(lib):
     assert n(None, 0, 64, 2, 4, None, None, None) == OK          # empty batch
 
 
+def test_multi_validation(lib):
+    f = lib.sparse_gemv_multi
+    P = ctypes.c_void_p * 2
+    I = ctypes.c_int64 * 2
+    W, Y, D = P(FAKE, FAKE), P(FAKE, FAKE), I(64, 64)
+    big = 1 << 30
+    assert f(0, W, D, 64, FAKE, 0.0, None, None, Y, FAKE, big, None) == ARG
+    assert f(5, W, D, 64, FAKE, 0.0, None, None, Y, FAKE, big, None) == ARG
+    assert f(2, None, D, 64, FAKE, 0.0, None, None, Y, FAKE, big, None) == NULL
+    assert f(2, P(FAKE, None), D, 64, FAKE, 0.0, None, None, Y, FAKE, big, None) == NULL
+    assert f(2, W, I(64, 60), 64, FAKE, 0.0, None, None, Y, FAKE, big, None) == SHAPE
+    assert f(2, P(FAKE, FAKE_ODD), D, 64, FAKE, 0.0, None, None, Y, FAKE, big, None) == ALIGN
+    assert f(2, W, D, 64, FAKE, 0.0, None, None, Y, None, big, None) == WORKSPACE
+    need = lib.sig_workspace_bytes_multi(2, D, 64)
+    assert need > 0
+    assert f(2, W, D, 64, FAKE, 0.0, None, None, Y, FAKE, need - 1, None) == WORKSPACE
+    assert lib.sig_workspace_bytes_multi(0, D, 64) == 0
+
+
 def test_gated_and_gemm_validation(lib):
     g = lib.gated_mlp_sparse
     big = 1 << 30

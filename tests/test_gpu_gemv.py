@@ -116,6 +116,44 @@ def test_llama2_7b_projection_all_sparsities(sig, name):
 
 
 # ---------------------------------------------------------------------------
+# several weights sharing one input (q, k, v; gate, up)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d_in,d_outs", [(4096, (4096, 4096, 4096)), (4096, (11008, 11008)),
+                                         (1000, (4096, 1024, 1024)), (257, (264, 8, 1000, 4104))])
+def test_multi_weight_threshold(sig, d_in, d_outs):
+    rng = np.random.default_rng(d_in + sum(d_outs))
+    x = workloads.draw_vector(rng, d_in, "laplace")
+    Ws = [workloads.draw_weight(rng, d_in, d, 0.02) for d in d_outs]
+    t = workloads.quantile_threshold(x, 0.5)
+    m = oracle.threshold_mask(x, t)
+    ys = sig.sparse_gemv_multi([to_dev(W) for W in Ws], to_dev(x), t=t)
+    for p, (W, y) in enumerate(zip(Ws, ys)):
+        ref = oracle.sparse_linear(W, x, m)
+        assert_within(to_host(y), ref["y64"], ref["bound"], f"multi weight {p} of {d_outs}")
+
+
+def test_multi_weight_index_path_and_single_weight_equivalence(sig):
+    layer = workloads.llama2_7b_layer(0)
+    q, k, v = layer[0], layer[1], layer[2]
+    assert q.x is k.x and q.x is v.x
+    dx = to_dev(q.x)
+    kk = workloads.topk_count(0.5, q.d_in)
+    mb, idx, nnz = sig.sparsify_topk(dx, kk)
+    m = oracle.topk_mask(q.x, kk)
+    ys = sig.sparse_gemv_multi([to_dev(p.WT) for p in (q, k, v)], dx, idx=idx, nnz=nnz)
+    for p, y in zip((q, k, v), ys):
+        ref = oracle.sparse_linear(p.WT, p.x, m)
+        assert_within(to_host(y), ref["y64"], ref["bound"], f"multi idx {p.name}")
+    # one weight through the multi entry point is the single-weight call
+    dW = to_dev(q.WT)
+    t = q.thresholds[0.5]
+    (y1,) = sig.sparse_gemv_multi([dW], dx, t=t)
+    y2 = sig.sparse_gemv(dW, dx, t=t)
+    assert np.array_equal(to_host(y1).view(np.uint16), to_host(y2).view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
 # top-k
 # ---------------------------------------------------------------------------
 

@@ -35,7 +35,7 @@ __all__ = [
     "LLAMA2_7B_PROJECTIONS", "QSPARSE_70B_PROJECTIONS", "NM_PATTERNS",
     "LLAMA2_SPARSITIES", "QSPARSE_KEEP_FRACTIONS",
     "draw_weight", "draw_vector", "quantile_threshold", "topk_count",
-    "Projection", "projection", "rana_mlp", "nm_tokens", "tiny_gemv",
+    "Projection", "projection", "rana_mlp", "nm_tokens", "tiny_gemv", "llama2_7b_layer",
 ]
 
 # Llama-2-7B decode projections at batch 1: (name, d_in, d_out).
@@ -136,6 +136,17 @@ def llama2_7b(seed: int = 0, names=None):
         out.append(projection(name, d_in, d_out, sigma=0.02, dist="laplace",
                               seed=1000 * seed + j, sparsities=LLAMA2_SPARSITIES))
     return out
+
+
+def llama2_7b_layer(seed: int = 0):
+    """One decoder layer as the model wires it: k and v read the same hidden
+    state as q, and up the same as gate, so they share its threshold mask.
+    Returns the seven projections in order q, k, v, o, gate, up, down."""
+    projs = {p.name: p for p in llama2_7b(seed)}
+    for shared, src in (("k", "q"), ("v", "q"), ("up", "gate")):
+        p = projs[shared]
+        projs[shared] = Projection(p.name, p.WT, projs[src].x, dict(projs[src].thresholds))
+    return [projs[n] for n, _, _ in LLAMA2_7B_PROJECTIONS]
 
 
 def qsparse_70b(seed: int = 0, names=None):
