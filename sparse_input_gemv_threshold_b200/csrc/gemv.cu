@@ -7,16 +7,18 @@
 //
 // Launch shape: C x S CTAs of 256 threads, about four per SM on every SM.  A
 // CTA owns a 256-output column tile (one warp spans it with 16-byte lanes) and
-// one of S <= 32 equal slices of the ascending kept-row list.  Up to four
-// weights that read the same input (q, k, v; gate, up) share one launch and
-// one mask: their column tiles are laid end to end.  One launch does
-// everything:
-//   1. every CTA ballots the whole activation (it sits in L2) into shared
-//      mask words with fp16 SIMD compares against the threshold rounded up to
-//      fp16 (exact for fp16 inputs), prefix-sums the words' popcounts (one
-//      barrier) to get nnz, its slice [lo, hi) and each word's first rank;
-//      the warps then place the slice's rows in parallel, one word per warp
-//      and one bit per lane (rank = word prefix + popcount of the lower bits);
+// one slice s of the kept rows.  Under a threshold the slices interleave by
+// 8-input groups (slice s owns groups s, s+S, s+2S, ...), so a CTA needs only
+// its own 1/S of the activation to know its rows; an index list is cut into S
+// equal runs.  Up to four weights that read the same input (q, k, v; gate, up)
+// share one launch and one mask: their column tiles are laid end to end.  One
+// launch does everything:
+//   1. the CTA loads its groups of the activation (from L2), ballots them into
+//      shared mask words with fp16 SIMD compares against the threshold rounded
+//      up to fp16 (exact for fp16 inputs), prefix-sums the words' popcounts
+//      (one barrier), and the warps place its kept rows in ascending order,
+//      one word per warp and one bit per lane (rank = word prefix + popcount
+//      of the lower bits);
 //   2. 8 warps stream the slice's rows of the tile, 8 rows in flight per warp:
 //      16-byte non-allocating loads with an L2 evict-first policy, the
 //      activation value riding along as a broadcast load, fp32 FMA;
@@ -77,46 +79,46 @@ __device__ __forceinline__ uint32_t thresh_bits8(const uint4& v, __half2 th2) {
   return b;
 }
 
-// All mask words of x into words[] (bit i%32 of word i/32 is m_i).
+// Mask bits of the 8-input groups this slice owns.  Group g covers inputs
+// 8g .. 8g+7; slice s owns groups s, s + S, s + 2S, ... (K of them), four to
+// a local word: bit 8q + b of local word lw is input 8 (s + (4 lw + q) S) + b.
 template <int MODE>
-__device__ __forceinline__ void build_words(const KArgs& a, int nwords, uint32_t* words) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int d_in = a.d_in;
-  constexpr int kPass = kThreads * 8;
+__device__ __forceinline__ void build_local_words(const KArgs& a, int s, int K, int nlw,
+                                                  uint32_t* words) {
+  const int d_in = a.d_in, S = a.S;
   const float t = a.t;
   const __half2 th2 = __half2half2(t <= 0.f ? __float2half(0.f) : __float2half_ru(t));
-  for (int base0 = 0; base0 < d_in; base0 += kPass * 8) {
-    uint4 v[8];
+  for (int lw = threadIdx.x; lw < nlw; lw += kThreads) {
+    uint4 v[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {   // eight passes' loads in flight together
-      const int e0 = base0 + u * kPass + tid * 8;
-      v[u] = e0 + 8 <= d_in ? __ldg(reinterpret_cast<const uint4*>(a.x + e0))
-                            : make_uint4(0, 0, 0, 0);
+    for (int q = 0; q < 4; ++q) {     // the word's four groups in flight together
+      const int k = lw * 4 + q;
+      const int e0 = (s + k * S) * 8;
+      v[q] = k < K && e0 + 8 <= d_in ? __ldg(reinterpret_cast<const uint4*>(a.x + e0))
+                                     : make_uint4(0, 0, 0, 0);
     }
+    uint32_t w = 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int base = base0 + u * kPass;
-      if (base >= d_in) break;                         // uniform across the block
-      const int e0 = base + tid * 8;
+    for (int q = 0; q < 4; ++q) {
+      const int k = lw * 4 + q;
+      if (k >= K) break;
+      const int e0 = (s + k * S) * 8;
       uint32_t b = 0;
       if (MODE == MASK_THRESH && e0 + 8 <= d_in) {
-        b = thresh_bits8(v[u], th2);
+        b = thresh_bits8(v[q], th2);
       } else {
-        for (int k = 0; k < 8; ++k) {
-          const int i = e0 + k;
+        for (int j = 0; j < 8; ++j) {
+          const int i = e0 + j;
           if (i >= d_in) break;
-          const float m = fabsf(h2f(e0 + 8 <= d_in ? lane_half(v[u], k) : a.x[i]));
+          const float m = fabsf(h2f(e0 + 8 <= d_in ? lane_half(v[q], j) : a.x[i]));
           const bool keep = MODE == MASK_THRESH_SCALED ? __fmul_rn(m, __ldg(a.scale + i)) >= t
                                                        : m >= t;
-          b |= (keep ? 1u : 0u) << k;
+          b |= (keep ? 1u : 0u) << j;
         }
       }
-      uint32_t w = b << (8 * (lane & 3));
-      w |= __shfl_xor_sync(kFull, w, 1);
-      w |= __shfl_xor_sync(kFull, w, 2);
-      const int wi = (base >> 5) + (tid >> 2);
-      if ((lane & 3) == 0 && wi < nwords) words[wi] = w;
+      w |= b << (8 * q);
     }
+    words[lw] = w;
   }
 }
 
@@ -138,11 +140,16 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   pdl_trigger();
   pdl_wait();
 
-  // ---- 1. this CTA's slice [lo, hi) of the kept-row list ---------------
-  int lo = 0, hi = 0, nwords = 0;
+  // ---- 1. this CTA's rows [lo, hi) of its kept-row list -----------------
+  // threshold modes: the kept inputs of the slice's own 8-input groups, in
+  // ascending order; index and dense modes: the s-th of S equal slices of the
+  // index list / of all rows
+  int lo = 0, hi = 0, nwords = 0, K = 0;
   if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED) {
-    nwords = (d_in + 31) >> 5;
-    build_words<MODE>(a, nwords, words);
+    const int ngroups = (d_in + 7) >> 3;
+    K = s < ngroups ? (ngroups - 1 - s) / S + 1 : 0;
+    nwords = (K + 3) >> 2;
+    build_local_words<MODE>(a, s, K, nwords, words);
     __syncthreads();
     // exclusive prefix of the words' popcounts, thread-contiguous word ranges
     const int per = (nwords + kThreads - 1) / kThreads;
@@ -169,10 +176,15 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
       wpre[w] = r;
       r += __popc(words[w]);
     }
-    lo = (int)(((long long)s * total) / S);
-    hi = (int)(((long long)(s + 1) * total) / S);
-    if (a.mask_out != nullptr && cg == 0 && s == 0)
-      for (int w = tid; w < nwords; w += kThreads) a.mask_out[w] = words[w];
+    lo = 0;
+    hi = total;
+    if (a.mask_out != nullptr && cg == 0) {
+      // byte g of the mask words holds group g's bits; the slice writes its
+      // own groups, slice 0 also the padding bytes of the last word
+      uint8_t* mb = reinterpret_cast<uint8_t*>(a.mask_out);
+      for (int k = tid; k < K; k += kThreads) mb[s + k * S] = (uint8_t)(words[k >> 2] >> (8 * (k & 3)));
+      if (s == 0 && tid < 4 * ((d_in + 31) >> 5) - ngroups) mb[ngroups + tid] = 0;
+    }
     __syncthreads();
   } else if (MODE == MASK_IDX) {
     const int total = min(max(__ldg(a.nnz), 0), d_in);
@@ -184,25 +196,19 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   }
   const int n_rows = hi - lo;
 
-  // first word that can hold rank lo: the last one whose prefix is <= lo
-  int w_first = 0;
-  if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED) {
-    int a1 = nwords - 1;
-    while (w_first < a1) {
-      const int mid = (w_first + a1 + 1) >> 1;
-      if (wpre[mid] <= lo) w_first = mid; else a1 = mid - 1;
-    }
-  }
-
   // ---- 2. stream the slice's rows of this column tile ------------------
-  int pm = 0;                                  // the weight this tile belongs to
-  if (MULTI)
-    while (pm + 1 < a.n_mat && cg >= a.tile0[pm + 1]) ++pm;
-  const int c = cg - a.tile0[pm];              // tile within that weight
-  const int d_out = a.d_out[pm];
-  const int col = c * kTile + lane * 8;
+  // the weight this tile belongs to (static indices only: the arguments stay
+  // in the parameter bank)
+  const uint16_t* wsel = a.WT[0];
+  int d_out = a.d_out[0], t_first = 0;
+  if (MULTI) {
+#pragma unroll
+    for (int i = 1; i < kGemvMaxMat; ++i)
+      if (i < a.n_mat && cg >= a.tile0[i]) { wsel = a.WT[i]; d_out = a.d_out[i]; t_first = a.tile0[i]; }
+  }
+  const int col = (cg - t_first) * kTile + lane * 8;
   const bool col_ok = col < d_out;
-  const uint16_t* wp = a.WT[pm] + col;
+  const uint16_t* wp = wsel + col;
   const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
   const uint64_t pol = l2_evict_first_policy();
   float acc[8], acc2[8];
@@ -220,14 +226,15 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
           sidx[j] = (unsigned)i < (unsigned)d_in ? i : -1;
         }
       } else {
-        // one word per warp, one bit per lane: rank = word's first rank +
-        // popcount of the word's lower bits
-        for (int w = w_first + warp; w < nwords; w += kWarps) {
+        // one local word per warp, one bit per lane: rank = word's first
+        // rank + popcount of the word's lower bits
+        for (int w = warp; w < nwords; w += kWarps) {
           const int base = wpre[w];
           if (base >= c_hi) break;                     // uniform across the warp
           const uint32_t bits = words[w];
           const int rk = base + __popc(bits & ((1u << lane) - 1u));
-          if (((bits >> lane) & 1u) && rk >= c_lo && rk < c_hi) sidx[rk - c_lo] = w * 32 + lane;
+          if (((bits >> lane) & 1u) && rk >= c_lo && rk < c_hi)
+            sidx[rk - c_lo] = (s + (w * 4 + (lane >> 3)) * S) * 8 + (lane & 7);
         }
       }
       __syncthreads();
@@ -281,12 +288,17 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     if (DUAL) p2 += red[kWarps * kTile + w * kTile + tid];
   }
   // the tile's weight again (kept out of registers through the main loop)
-  int pe = 0;
-  if (MULTI)
-    while (pe + 1 < a.n_mat && cg >= a.tile0[pe + 1]) ++pe;
-  const int colr = (cg - a.tile0[pe]) * kTile + tid;
-  const bool colr_ok = colr < a.d_out[pe];
-  uint16_t* __restrict__ Y = a.y[pe];
+  uint16_t* __restrict__ Y = a.y[0];
+  int e_dout = a.d_out[0], e_first = 0, e_col0 = 0;
+  if (MULTI) {
+#pragma unroll
+    for (int i = 1; i < kGemvMaxMat; ++i)
+      if (i < a.n_mat && cg >= a.tile0[i]) {
+        Y = a.y[i]; e_dout = a.d_out[i]; e_first = a.tile0[i]; e_col0 = a.col0[i];
+      }
+  }
+  const int colr = (cg - e_first) * kTile + tid;
+  const bool colr_ok = colr < e_dout;
   const int dtot = a.d_out_total;
 
   auto finish = [&](float g, float u) {
@@ -302,7 +314,7 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     if (colr_ok) finish(p, p2);
     return;
   }
-  const size_t pcol = (size_t)a.col0[pe] + colr;   // column in the partial-sum space
+  const size_t pcol = (size_t)e_col0 + colr;       // column in the partial-sum space
   if (colr_ok) {
     a.partials[(size_t)s * dtot + pcol] = p;
     if (DUAL) a.partials[(size_t)S * dtot + (size_t)s * dtot + pcol] = p2;
@@ -314,9 +326,9 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   if (!s_last) return;
   __threadfence();
   if (colr_ok) {
-    // the partials of the column in flight together (all of them for S <= 16
-    // single, 8 per batch for the dual product), then added in slice order
-    constexpr int B = DUAL ? 8 : 16;
+    // the partials of the column in flight together (all of them for the
+    // single product, 8 per batch for the dual one), then added in slice order
+    constexpr int B = DUAL ? 8 : kMaxS;
     const float* pp = a.partials + pcol;
     float g = 0.f, u = 0.f;
     for (int q0 = 0; q0 < S; q0 += B) {
@@ -360,7 +372,10 @@ GemvPlan plan_gemv_multi(int64_t d_in, const int64_t* d_out, int n_mat, bool dua
     total += d_out[i];
   }
   p.S = std::max(1, std::min(kMaxS, (kNumSMs * kGemvCtasPerSM) / std::max(1, p.C)));
-  p.chunk = (int)std::max<int64_t>(1, std::min<int64_t>((d_in + p.S - 1) / p.S, kIdxCap));
+  // rows per slice: at most ceil(d_in / S) for an index or dense slice, at
+  // most 8 ceil(ceil(d_in / 8) / S) for a threshold slice's own groups
+  const int64_t groups = (d_in + 7) / 8;
+  p.chunk = (int)std::max<int64_t>(1, std::min<int64_t>((groups + p.S - 1) / p.S * 8, kIdxCap));
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)kWarps * kTile * 4 * (dual ? 2 : 1);
   p.smem = std::max(2 * words, red) + round_up((size_t)p.chunk * 4, 16);

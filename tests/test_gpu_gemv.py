@@ -57,15 +57,22 @@ def test_empty_and_full_masks(sig):
     assert np.all(y2.view(np.uint16) == 0)
 
 
-def test_index_path_matches_fused_path_bit_for_bit(sig):
+def test_index_path_and_fused_path_agree(sig):
+    # the two paths split the kept rows differently (interleaved 8-input groups
+    # under a threshold, equal runs of an index list), so they agree within the
+    # bound, each one bit for bit with itself
     p = workloads.projection("i", 4096, 4096, sigma=0.02, dist="laplace", seed=11,
                              sparsities=(0.5,))
     dW, dx = to_dev(p.WT), to_dev(p.x)
     t = p.thresholds[0.5]
+    ref = oracle.sparse_linear(p.WT, p.x, oracle.threshold_mask(p.x, t))
     y_fused = to_host(sig.sparse_gemv(dW, dx, t=t))
     _, idx, nnz = sig.sparsify_threshold(dx, t)
     y_idx = to_host(sig.sparse_gemv(dW, dx, idx=idx, nnz=nnz))
-    assert np.array_equal(y_fused.view(np.uint16), y_idx.view(np.uint16))
+    assert_within(y_fused, ref["y64"], ref["bound"], "fused")
+    assert_within(y_idx, ref["y64"], ref["bound"], "index list")
+    assert np.array_equal(y_idx.view(np.uint16),
+                          to_host(sig.sparse_gemv(dW, dx, idx=idx, nnz=nnz)).view(np.uint16))
 
 
 def test_out_of_range_indices_are_skipped(sig):
