@@ -20,6 +20,15 @@ __device__ __forceinline__ void pdl_trigger() {
 // L2 policy for data read exactly once (weight rows): evict first, so that
 // the stream does not push the small reused buffers (x, index lists, split-K
 // partials, counters) out of L2.
+// Atomic add with acquire-release semantics at GPU scope: publishes the
+// writes that the CTA made before a preceding __syncthreads, and makes the
+// writes published by earlier arrivers visible to the CTA after the next one.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
   asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));

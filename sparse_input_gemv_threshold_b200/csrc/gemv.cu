@@ -23,9 +23,9 @@
 //      16-byte non-allocating loads with an L2 evict-first policy, the
 //      activation value riding along as a broadcast load, fp32 FMA;
 //   3. the warps' sums meet in shared memory (fixed order), the CTA writes one
-//      partial per column, and the CTA that arrives last for the tile (an
-//      atomic counter) loads the S partials in one batch, adds them in slice
-//      order and stores fp16.
+//      partial per column, and the CTA that arrives last for the tile (one
+//      acquire-release atomic per CTA) loads the S partials in one batch, adds
+//      them in slice order and stores fp16.
 // No floating-point atomics and no spin-waits; y is bit-identical from run to
 // run.
 #include "common.cuh"
@@ -319,12 +319,13 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     a.partials[(size_t)s * dtot + pcol] = p;
     if (DUAL) a.partials[(size_t)S * dtot + (size_t)s * dtot + pcol] = p2;
   }
-  __threadfence();
+  // one release-acquire arrival per CTA: the barrier orders every thread's
+  // partial store before thread 0's release, and thread 0's acquire before
+  // the last arriver's loads
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(a.counters + cg, 1u) == (unsigned)(S - 1));
+  if (tid == 0) s_last = atomic_add_acq_rel_gpu(a.counters + cg, 1u) == (unsigned)(S - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   if (colr_ok) {
     // the partials of the column in flight together (all of them for the
     // single product, 8 per batch for the dual one), then added in slice order
