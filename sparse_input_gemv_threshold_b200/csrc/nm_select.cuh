@@ -77,6 +77,21 @@ __device__ __forceinline__ uint32_t nm_word_bits(const uint4 (&q)[4], int n, int
   return bits;
 }
 
+// Keep-bits of the 8 entries of one 16-byte vector, for M dividing 8 (blocks
+// never straddle the vector).
+template <int M>
+__device__ __forceinline__ uint32_t nm_vec_bits(const uint4& v, int n) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int b0 = 0; b0 < 8; b0 += M) {
+    uint32_t comp[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) comp[j] = (mag_key(lane_half(v, b0 + j)) << 5) | (uint32_t)(31 - j);
+    bits |= select_top_n<M>(comp, n) << b0;
+  }
+  return bits;
+}
+
 // The 16-byte vector `v` (entries 8i .. 8i+7 of the word) with the entries
 // whose keep-bit is clear set to +0.
 __device__ __forceinline__ uint4 nm_apply(const uint4& v, uint32_t bits, int i) {

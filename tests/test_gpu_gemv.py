@@ -173,7 +173,7 @@ def _check_topk(sig, x, k, what):
     return mb, idx, nnz
 
 
-@pytest.mark.parametrize("d", [1, 2, 31, 33, 1000, 8192, 28672])
+@pytest.mark.parametrize("d", [1, 2, 31, 33, 1000, 8192, 12288, 12289, 28672, 32767, 65537, 131072])
 def test_topk_masks_random(sig, d):
     x = workloads.draw_vector(np.random.default_rng(d), d, "student_t4")
     for k in sorted({0, 1, d // 3, d // 2, workloads.topk_count(0.6, d), d - 1, d}):
@@ -198,6 +198,13 @@ def test_topk_heavy_ties_and_specials(sig):
     x[[12]] = np.float16(6e-8)     # subnormal
     for k in (1, 3, 4, 100, 597, 598, 600):
         _check_topk(sig, x, k, f"specials k={k}")
+    # ties that span the CTAs of the cluster path
+    x = rng.choice([0.5, -1.0, 1.0, 2.0, -0.0], size=40000).astype(np.float16)
+    for k in (1, 7999, 8000, 13333, 20000, 31999, 39999, 40000):
+        _check_topk(sig, x, k, f"cluster ties k={k}")
+    x = np.full(70001, -7.0, dtype=np.float16)
+    for k in (1, 35000, 70000):
+        _check_topk(sig, x, k, f"cluster all equal k={k}")
 
 
 @pytest.mark.parametrize("name", ["up", "down"])

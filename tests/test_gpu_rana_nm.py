@@ -115,6 +115,10 @@ def test_nm_mask_ragged_and_ties(sig):
             for n in sorted({1, max(1, m // 2), m}):
                 _check_nm(sig, X, n, m, f"d={d} {n}:{m}")
     _check_nm(sig, np.zeros((0, 64), np.float16), 2, 4, "zero rows")
+    # several vectors per thread, rows whose last word is partial
+    X = workloads.draw_vector(rng, (37, 1000), "laplace")
+    for n, m in ((1, 1), (1, 2), (2, 4), (1, 4), (3, 8), (8, 8)):
+        _check_nm(sig, X, n, m, f"37x1000 {n}:{m}")
 
 
 # ---------------------------------------------------------------------------
