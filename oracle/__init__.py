@@ -24,8 +24,11 @@ Sources, cited by page title and section:
          states that feed each matrix multiplication.
 * [RaNA] "Adaptive Rank Allocation: Speeding Up Modern Transformers with RaNA
          Adapters" (OpenReview rebuttal): Q3, Eqn. 12 (RaNA neuron masker) and
-         the CATS masker beside it; Q5.1, the masked product A(m(x) . Bx) that
-         skips the columns whose mask entry is 0.
+         the CATS masker beside it; Q5.1, the linear-layer rank adapter
+         Linear(x) ~ A(m(x) . Bx), whose masked product skips the columns of A
+         whose mask entry is 0; Q4, its masker squares Bx element-wise and
+         compares with a threshold (eqn. 9); Q2 to the fourth reviewer, one
+         plain GEMV for v = Bx and one masked GEMV for A(m(x) . v).
 * [NM]   "Motivating Next-Gen Accelerators with Flexible (N:M) Activation
          Sparsity ..." (summary), Methodology: in blocks of size M, N non-zero
          elements are kept; selection criterion ACT = absolute activation size.
@@ -44,6 +47,9 @@ Readings where the pages are silent or disagree (each one is a choice):
   once to float32.
 * Eqn. 12 precision: g and u in float64 from the fp16 inputs, h rounded once to
   fp16, ``s_i = float32(|h_i|) * norm_i`` as one float32 multiply, ``s_i >= t``.
+* Rank adapter precision: v = Bx in float64 from the fp16 inputs, rounded once
+  to fp16 (the intermediate activation of an fp16 model); the score is
+  ``float32(v_i) * float32(v_i)`` as one float32 multiply; ``score >= t``.
 * Outputs: y in float64 (used for the error bound) and rounded once to fp16.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
@@ -59,6 +65,7 @@ __all__ = [
     "compact", "pack_bits", "unpack_bits", "sparsity", "flops",
     "masked_matvec", "sparse_linear", "silu", "row_norms", "rana_hidden",
     "rana_scores", "rana_mask", "gated_mlp", "nm_gemm",
+    "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
 ]
 
 
@@ -248,6 +255,41 @@ def gated_mlp(x, WgT, WuT, WdT, norms32, t: float, cols=None) -> dict:
     m = rana_mask(s32, t)
     out = sparse_linear(WdT, h16, m, cols)
     out.update({"g": g, "u": u, "h16": h16, "s32": s32})
+    return out
+
+
+# ---------------------------------------------------------------------------
+# RaNA linear-layer rank adapter A (m(x) . Bx)
+# ---------------------------------------------------------------------------
+
+def rank_adapter_hidden(x, BT):
+    """v = Bx in float64 from the fp16 inputs, and v rounded once to fp16.
+
+    ``BT`` is B transposed, (d_in, r): row i multiplies input i.  This is the
+    plain GEMV of [RaNA] Q2 (fourth reviewer).
+    """
+    v64 = np.asarray(x, dtype=np.float64) @ np.asarray(BT).astype(np.float64)
+    return v64, fp16(v64)
+
+
+def rank_adapter_scores(v16) -> np.ndarray:
+    """s_i = v_i^2 as one float32 multiply ([RaNA] Q4: the masker squares Bx
+    element-wise, eqn. 9)."""
+    v32 = np.asarray(v16, dtype=np.float16).astype(np.float32)
+    return (v32 * v32).astype(np.float32)
+
+
+def rank_adapter(x, BT, AT, t: float, cols=None) -> dict:
+    """[RaNA] Q5.1: Linear(x) ~ A (m(x) . Bx) with m_i = (Bx)_i^2 >= t.
+
+    ``AT`` is A transposed, (r, d_out): row i multiplies v_i, so the masked
+    product skips the rows of AT (columns of A) whose mask entry is 0.
+    """
+    v64, v16 = rank_adapter_hidden(x, BT)
+    s32 = rank_adapter_scores(v16)
+    m = rana_mask(s32, t)
+    out = sparse_linear(AT, v16, m, cols)
+    out.update({"v64": v64, "v16": v16, "s32": s32})
     return out
 
 

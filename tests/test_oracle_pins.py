@@ -469,3 +469,71 @@ def test_workloads_are_seeded_and_chunking_invariant():
     direct = rng.normal(0.0, 0.02, 1024 * 1024).astype(np.float16).reshape(1024, 1024)
     assert np.array_equal(direct, a.WT)
     assert a.thresholds[0.5] == workloads.quantile_threshold(a.x, 0.5)
+
+
+# ---------------------------------------------------------------------------
+# RaNA linear-layer rank adapter
+# ---------------------------------------------------------------------------
+
+def _rank_adapter_fixture():
+    x, B, A, v, cases = None, [], [], None, []
+    for ln in _read_lines("rank_adapter_tiny.txt"):
+        if ln.startswith("x:"):
+            x = _floats(ln[2:])
+        elif ln.startswith("B:"):
+            B.append(_floats(ln[2:]))
+        elif ln.startswith("A:"):
+            A.append(_floats(ln[2:]))
+        elif ln.startswith("v:"):
+            v = _floats(ln[2:])
+        else:
+            t, m, y = ln.split("|")
+            cases.append((float(t), [int(c) for c in m.split()], _floats(y)))
+    return (np.array(x, np.float16), np.array(B, np.float16), np.array(A, np.float16),
+            np.array(v), cases)
+
+
+def test_rank_adapter_golden():
+    x, B, A, v, cases = _rank_adapter_fixture()
+    v64, v16 = oracle.rank_adapter_hidden(x, B.T)
+    assert v64.tolist() == v.tolist() and v16.astype(np.float64).tolist() == v.tolist()
+    assert oracle.rank_adapter_scores(v16).tolist() == (v * v).tolist()
+    for t, m, y in cases:
+        out = oracle.rank_adapter(x, B.T, A.T, t)
+        assert out["mask"].astype(int).tolist() == m, t
+        assert out["y64"].tolist() == y, t
+
+
+def test_rank_adapter_identity_b_is_the_threshold_layer():
+    """B = I makes v = x exactly; the square of an fp16 value is exact in fp32,
+    so v_i^2 >= c^2 is |x_i| >= c and the adapter is the threshold layer on A."""
+    rng = np.random.default_rng(21)
+    d, d_out = 300, 40
+    x = rng.laplace(0, 1, d).astype(np.float16)
+    AT = rng.normal(0, 0.02, (d, d_out)).astype(np.float16)
+    eye = np.eye(d, dtype=np.float16)
+    for c in (0.0, 0.25, float(np.sort(np.abs(x))[150]), 3.0):
+        out = oracle.rank_adapter(x, eye, AT, c * c)
+        ref = oracle.sparse_linear(AT, x, oracle.threshold_mask(x, c))
+        assert np.array_equal(out["mask"], ref["mask"])
+        assert np.array_equal(out["y64"], ref["y64"])
+
+
+def test_rank_adapter_masked_rows_do_not_matter():
+    """Rows of A^T whose mask entry is 0 never reach y ([RaNA] Q5.1)."""
+    rng = np.random.default_rng(22)
+    d_in, r, d_out = 64, 48, 24
+    x = rng.normal(0, 1, d_in).astype(np.float16)
+    BT = rng.normal(0, 0.2, (d_in, r)).astype(np.float16)
+    AT = rng.normal(0, 0.2, (r, d_out)).astype(np.float16)
+    out = oracle.rank_adapter(x, BT, AT, 1.0)
+    assert 0 < out["nnz"] < r
+    AT2 = AT.copy()
+    AT2[~out["mask"]] = np.float16(1000.0)
+    assert np.array_equal(oracle.rank_adapter(x, BT, AT2, 1.0)["y64"], out["y64"])
+    # t = 0 keeps every finite v: the unmasked two-GEMV product
+    dense = oracle.rank_adapter(x, BT, AT, 0.0)
+    assert dense["nnz"] == r
+    v16 = dense["v16"].astype(np.float64)
+    want = [sum(v16[i] * float(AT[i, j]) for i in range(r)) for j in range(d_out)]
+    assert np.allclose(dense["y64"], want, rtol=0, atol=1e-12)
