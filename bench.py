@@ -16,7 +16,7 @@ no step finds its weights in L2 (580 MB of kept rows per rotation, > 4x L2).
 Steps are replayed CUDA graphs, timed with CUDA events on the launching stream.
 
 The JSON line also carries the sparsity sweep, the top-k (Q-Sparse 70B), RaNA
-gated-MLP and N:M GEMM rows, cuBLAS dense baselines at the same shapes, the
+gated-MLP, RaNA rank-adapter and N:M GEMM rows, cuBLAS dense baselines at the same shapes, the
 roofline of the sparse GEMV kernel, the oracle's CPU baseline and the SM
 clocks sampled during the timed region.
 
@@ -413,6 +413,7 @@ def run_ours(args, rank, world, local):
         extras["topk_qsparse_70b"] = bench_topk(args, stream, sig, hbm_peak)
         extras["rana_gated_mlp"] = bench_rana(args, stream, sig, hbm_peak)
         extras["nm_gemm"] = bench_nm(args, stream, sig, bf16_peak)
+        extras["rana_rank_adapter"] = bench_rank_adapter(args, stream, sig, hbm_peak)
         result["extras"] = extras
         result["cpu_baseline"] = cpu_baseline(groups)
     return result
@@ -552,6 +553,58 @@ def bench_rana(args, stream, sig, hbm_peak):
            "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
            "l2": "2 rotating weight copies of 258 MB"}
     del Ws, sg
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_rank_adapter(args, stream, sig, hbm_peak):
+    """RaNA rank adapter A (m . Bx) replacing one 4096 x 4096 projection, r = 2048."""
+    import torch
+    ra = workloads.rank_adapter(args.seed)
+    d_in, r = ra.BT.shape
+    d_out = ra.AT.shape[1]
+    copies = 16                      # 16 x 33.6 MB of factors rotate, > 4x L2
+    Bs = [torch.from_numpy(ra.BT).cuda()]
+    As = [torch.from_numpy(ra.AT).cuda()]
+    Bs += [Bs[0].clone() for _ in range(copies - 1)]
+    As += [As[0].clone() for _ in range(copies - 1)]
+    x = torch.from_numpy(ra.x).cuda()
+    y = torch.empty(d_out, dtype=torch.float16, device="cuda")
+    v = torch.empty(r, dtype=torch.float16, device="cuda")
+    ws = torch.zeros(sig.workspace_bytes(sig.OP_RANK_ADAPTER, d_in, d_out, r), dtype=torch.uint8,
+                     device="cuda")
+    # threshold: 50 % quantile of this path's own scores v_i^2 (timing only)
+    sig.rank_adapter_sparse(x, Bs[0], As[0], 0.0, y=y, v_out=v, ws=ws)
+    sc = v.float().square().cpu().numpy()
+    t = float(np.sort(sc)[r // 2])
+    nnz = int((sc >= t).sum())
+
+    def f(c):
+        def g():
+            sig.rank_adapter_sparse(x, Bs[c], As[c], t, y=y, v_out=v, ws=ws, stream=stream)
+        return g
+    sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies)
+    steps = 320
+    sec = time_steps(sg, steps, copies, stream)
+    us = sec / steps * 1e6
+    b = 2 * d_in * r + nnz * 2 * d_out + 2 * d_in + 4 * r + 2 * d_out
+    # the dense projection the adapter stands in for, through torch (cuBLAS)
+    W = [torch.empty((d_in, d_out), dtype=torch.float16, device="cuda").normal_(0, 0.02)
+         for _ in range(copies)]
+    yd = torch.empty((1, d_out), dtype=torch.float16, device="cuda")
+
+    def dn(c):
+        def g():
+            torch.matmul(x.view(1, -1), W[c], out=yd)
+        return g
+    sd = StepGraphs([dn(c) for c in range(copies)], stream, per_graph=copies)
+    us_dense = time_steps(sd, steps, copies, stream) / steps * 1e6
+    res = {"shapes": f"B {r}x{d_in} dense, A {d_out}x{r} masked", "sparsity": round(1 - nnz / r, 4),
+           "us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+           "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
+           "cublas_dense_4096x4096_us": round(us_dense, 2),
+           "l2": f"{copies} rotating copies of the factors (538 MB)"}
+    del Bs, As, W, sg, sd
     torch.cuda.empty_cache()
     return res
 

@@ -73,7 +73,8 @@ typedef enum {
   SIG_OP_SPARSE_GEMV = 1,  /* sparse_gemv(d_in, d_out)                 */
   SIG_OP_TOPK = 2,         /* sparsify_topk(d = d_in)                  */
   SIG_OP_GATED_MLP = 3,    /* gated_mlp_sparse(d_model = d_in, d_ff = d_out) */
-  SIG_OP_NM_GEMM = 4       /* nm_act_gemm(K = d_in, N = d_out, rows)   */
+  SIG_OP_NM_GEMM = 4,      /* nm_act_gemm(K = d_in, N = d_out, rows)   */
+  SIG_OP_RANK_ADAPTER = 5  /* rank_adapter_sparse(d_in, d_out, rows = r) */
 } sig_op;
 
 /* Largest activation length the fused mask prologue accepts. */
@@ -223,6 +224,28 @@ SIG_API int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint1
                      int64_t d_model, int64_t d_ff, float t,
                      uint16_t* y, uint16_t* h_out, uint32_t* mask_out,
                      void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * RaNA linear-layer rank adapter (RaNA rebuttal, Q5.1: Linear(x) ~ A (m(x) . Bx),
+ * whose masked product skips the columns of A with a zero mask entry; Q4: the
+ * masker squares Bx element-wise against a threshold (eqn. 9); Q2 to the fourth
+ * reviewer: one plain GEMV for v = Bx and one masked GEMV):
+ *   v = fp16(B x)                        (dense GEMV, float32 accumulation)
+ *   m_i = float32(v_i) * float32(v_i) >= t          (one float32 multiply)
+ *   y = A (m . v)                        (sparse GEMV as in sparse_gemv)
+ *   x [d_in] fp16.  BT [d_in x r] fp16 (B transposed: row i multiplies x_i).
+ *   AT [r x d_out] fp16 (A transposed: row i multiplies v_i).
+ *   y [d_out] fp16 out.  v_out [r] fp16 out, nullable.
+ *   mask_out [ceil(r/32)] uint32 out, nullable.
+ *   ws sig_workspace_bytes(SIG_OP_RANK_ADAPTER, d_in, d_out, r) bytes.
+ * d_in, r, d_out: multiples of 8 (r and d_out as output widths), each
+ * <= SIG_MAX_D_IN.  Two launches on `stream`; the caller owns every buffer.
+ * Errors: as sparse_gemv.
+ */
+SIG_API int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uint16_t* AT,
+                                int64_t d_in, int64_t r, int64_t d_out, float t,
+                                uint16_t* y, uint16_t* v_out, uint32_t* mask_out,
+                                void* ws, size_t ws_bytes, sig_stream_t stream);
 
 /*
  * l2 norm of every row of a row-major fp16 matrix, accumulated in float64 and

@@ -22,12 +22,12 @@ __all__ = [
     "MAX_D_IN", "abi_version", "workspace_bytes", "workspace", "sparsify_threshold",
     "sparsify_topk", "sparsify_nm", "sparse_gemv", "gated_mlp_sparse", "row_norms",
     "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
-    "sparse_gemv_multi", "workspace_bytes_multi",
+    "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
 
-OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM = 1, 2, 3, 4
+OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM, OP_RANK_ADAPTER = 1, 2, 3, 4, 5
 MAX_D_IN = 131072
 
 _p, _i64, _i32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
@@ -49,6 +49,7 @@ _SIGNATURES = {
     "gated_mlp_sparse_noalloc": (_i32, [_p, _p, _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p]),
     "sparse_gemv_multi": (_i32, [_i32, _p, _p, _i64, _p, _f32, _p, _p, _p, _p, _sz, _p]),
     "sig_workspace_bytes_multi": (_sz, [_i32, _p, _i64]),
+    "rank_adapter_sparse": (_i32, [_p, _p, _p, _i64, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
 }
 
 
@@ -238,6 +239,28 @@ def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
     _check("gated_mlp_sparse", _lib.gated_mlp_sparse(
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
         _ptr(y), _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def rank_adapter_sparse(x, BT, AT, t: float, y=None, v_out=None, mask_out=None, ws=None,
+                        stream=None):
+    """RaNA rank adapter y = A (m . v), v = fp16(B x), m_i = v_i^2 >= t.  Returns y.
+
+    ``BT`` is B transposed (d_in x r), ``AT`` is A transposed (r x d_out).
+    """
+    for name, w in (("BT", BT), ("AT", AT), ("x", x)):
+        _need(w, torch.float16, name, x.device)
+    d_in, r = BT.shape
+    if AT.shape[0] != r or x.numel() != d_in:
+        raise ValueError("shapes: x (d_in), BT (d_in, r), AT (r, d_out)")
+    d_out = AT.shape[1]
+    if y is None:
+        y = torch.empty(d_out, dtype=torch.float16, device=x.device)
+    if ws is None:
+        ws = workspace(OP_RANK_ADAPTER, d_in, d_out, r, device=x.device, stream=stream)
+    _check("rank_adapter_sparse", _lib.rank_adapter_sparse(
+        _ptr(x), _ptr(BT), _ptr(AT), d_in, r, d_out, float(t), _ptr(y), _ptr(v_out),
+        _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
     return y
 
 

@@ -62,6 +62,10 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
       if (check_gemv_shape(d_in, d_out) != SIG_OK || check_gemv_shape(d_out, d_in) != SIG_OK)
         return 0;
       return plan_gated(d_in, d_out).total;
+    case SIG_OP_RANK_ADAPTER:
+      if (check_gemv_shape(d_in, rows) != SIG_OK || check_gemv_shape(rows, d_out) != SIG_OK)
+        return 0;
+      return plan_rank(d_in, rows, d_out).total;
     case SIG_OP_NM_GEMM:
       if (rows < 1 || d_in < 1) return 0;
       return round_up((size_t)rows * (size_t)d_in * 2, 256);   // the masked activation block
@@ -195,6 +199,35 @@ int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT
   dn.x = h; dn.scale = down_norms; dn.t = t; dn.d_in = (int)d_ff; dn.mask_out = mask_out;
   dn.ws = base + g.off_down;
   return cuda_status(launch_gemv(MASK_THRESH_SCALED, EPI_STORE, g.down, dn, (cudaStream_t)stream));
+}
+
+int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uint16_t* AT, int64_t d_in,
+                        int64_t r, int64_t d_out, float t, uint16_t* y, uint16_t* v_out,
+                        uint32_t* mask_out, void* ws, size_t ws_bytes, sig_stream_t stream) {
+  if (x == nullptr || BT == nullptr || AT == nullptr || y == nullptr) return SIG_ERR_NULL;
+  int sh = check_gemv_shape(d_in, r);
+  if (sh == SIG_OK) sh = check_gemv_shape(r, d_out);
+  if (sh != SIG_OK) return sh;
+  if (!aligned16(x) || !aligned16(BT) || !aligned16(AT) || !aligned16(y) ||
+      (v_out != nullptr && !aligned16(v_out)))
+    return SIG_ERR_ALIGN;
+  const RankPlan g = plan_rank(d_in, r, d_out);
+  if (ws == nullptr || ws_bytes < g.total) return SIG_ERR_WORKSPACE;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  char* base = reinterpret_cast<char*>(ws);
+  uint16_t* v = v_out != nullptr ? v_out : reinterpret_cast<uint16_t*>(base + g.off_v);
+
+  GemvLaunch in{};
+  in.WT[0] = BT; in.y[0] = v; in.d_out[0] = (int)r;
+  in.x = x; in.d_in = (int)d_in; in.ws = base;
+  cudaError_t e = launch_gemv(MASK_DENSE, EPI_STORE, g.in, in, (cudaStream_t)stream);
+  if (e != cudaSuccess) return SIG_ERR_CUDA;
+
+  GemvLaunch out{};
+  out.WT[0] = AT; out.y[0] = y; out.d_out[0] = (int)d_out;
+  out.x = v; out.t = t; out.d_in = (int)r; out.mask_out = mask_out;
+  out.ws = base + g.off_out;
+  return cuda_status(launch_gemv(MASK_SQUARE, EPI_STORE, g.out, out, (cudaStream_t)stream));
 }
 
 int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float* norms,

@@ -40,7 +40,7 @@ namespace {
 constexpr int kThreads = kGemvThreads;        // 256
 constexpr int kWarps = kThreads / 32;         // 8
 constexpr int kTile = kGemvTile;              // 256 outputs per CTA
-constexpr int kMaxS = kGemvMaxSplits;         // 32
+constexpr int kMaxS = kGemvMaxSplits;         // 64
 
 struct KArgs {
   // weights that share the input and its mask: column tiles [tile0[p],
@@ -112,6 +112,7 @@ __device__ __forceinline__ void build_local_words(const KArgs& a, int s, int K, 
           if (i >= d_in) break;
           const float m = fabsf(h2f(e0 + 8 <= d_in ? lane_half(v[q], j) : a.x[i]));
           const bool keep = MODE == MASK_THRESH_SCALED ? __fmul_rn(m, __ldg(a.scale + i)) >= t
+                            : MODE == MASK_SQUARE      ? __fmul_rn(m, m) >= t
                                                        : m >= t;
           b |= (keep ? 1u : 0u) << j;
         }
@@ -145,7 +146,7 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   // ascending order; index and dense modes: the s-th of S equal slices of the
   // index list / of all rows
   int lo = 0, hi = 0, nwords = 0, K = 0;
-  if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED) {
+  if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED || MODE == MASK_SQUARE) {
     const int ngroups = (d_in + 7) >> 3;
     K = s < ngroups ? (ngroups - 1 - s) / S + 1 : 0;
     nwords = (K + 3) >> 2;
@@ -327,9 +328,9 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   __syncthreads();
   if (!s_last) return;
   if (colr_ok) {
-    // the partials of the column in flight together (all of them for the
-    // single product, 8 per batch for the dual one), then added in slice order
-    constexpr int B = DUAL ? 8 : kMaxS;
+    // the partials of the column in flight together (32 per batch for the
+    // single product, 8 for the dual one), then added in slice order
+    constexpr int B = DUAL ? 8 : 32;
     const float* pp = a.partials + pcol;
     float g = 0.f, u = 0.f;
     for (int q0 = 0; q0 < S; q0 += B) {
@@ -372,7 +373,10 @@ GemvPlan plan_gemv_multi(int64_t d_in, const int64_t* d_out, int n_mat, bool dua
     p.C += (int)((d_out[i] + kTile - 1) / kTile);
     total += d_out[i];
   }
-  p.S = std::max(1, std::min(kMaxS, (kNumSMs * kGemvCtasPerSM) / std::max(1, p.C)));
+  // narrow launches (fewer than 16 column tiles) may cut the rows finer to
+  // fill the GPU; wider ones stop at 32 slices (one batch of partial loads)
+  const int cap = p.C >= 16 ? 32 : kMaxS;
+  p.S = std::max(1, std::min(cap, (kNumSMs * kGemvCtasPerSM) / std::max(1, p.C)));
   // rows per slice: at most ceil(d_in / S) for an index or dense slice, at
   // most 8 ceil(ceil(d_in / 8) / S) for a threshold slice's own groups
   const int64_t groups = (d_in + 7) / 8;
@@ -430,6 +434,7 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   switch (mode) {
     case MASK_THRESH: return launch_t<MASK_THRESH, false, EPI_STORE>(p, k, stream);
     case MASK_THRESH_SCALED: return launch_t<MASK_THRESH_SCALED, false, EPI_STORE>(p, k, stream);
+    case MASK_SQUARE: return launch_t<MASK_SQUARE, false, EPI_STORE>(p, k, stream);
     case MASK_IDX: return launch_t<MASK_IDX, false, EPI_STORE>(p, k, stream);
     case MASK_DENSE: return launch_t<MASK_DENSE, false, EPI_STORE>(p, k, stream);
   }

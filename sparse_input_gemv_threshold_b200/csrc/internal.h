@@ -13,7 +13,7 @@ constexpr int kNumSMs = 148;         // B200: 2 dies x 74 SMs
 constexpr int kGemvThreads = 256;    // 8 warps
 constexpr int kGemvCtasPerSM = 4;    // residency the grid is sized for
 constexpr int kGemvTile = 256;       // output columns per CTA (one warp spans them)
-constexpr int kGemvMaxSplits = 32;   // K-splits per column tile (one batch of partial loads)
+constexpr int kGemvMaxSplits = 64;   // K-splits per column tile (32 unless fewer than 16 tiles)
 constexpr int kIdxCap = 4096;        // rows of a slice staged in shared memory at once
 constexpr int kGemvMaxMat = 4;       // weights that can share one input in one launch
 constexpr int kMaxDIn = 131072;
@@ -24,7 +24,8 @@ enum MaskMode : int {
   MASK_THRESH = 0,         // |x_i| >= t, computed in the prologue
   MASK_THRESH_SCALED = 1,  // |x_i| * scale_i >= t (RaNA Eqn. 12 with scale = norms)
   MASK_IDX = 2,            // rows idx[0 .. *nnz) given by the caller
-  MASK_DENSE = 3           // every row
+  MASK_DENSE = 3,          // every row
+  MASK_SQUARE = 4          // x_i * x_i >= t (RaNA rank adapter masker, one float32 multiply)
 };
 
 // What happens to a finished output column.
@@ -78,6 +79,24 @@ inline GatedPlan plan_gated(int64_t d_model, int64_t d_ff) {
   g.off_down = up256(g.up.ws_bytes());
   g.off_h = g.off_down + up256(g.down.ws_bytes());
   g.total = g.off_h + up256((size_t)d_ff * 2);
+  return g;
+}
+
+// Rank adapter y = A (m . v), v = fp16(B x): a dense GEMV into v, then the
+// masked GEMV on A; one workspace holds both plans' scratch and v.
+struct RankPlan {
+  GemvPlan in, out;
+  size_t off_out, off_v, total;
+};
+
+inline RankPlan plan_rank(int64_t d_in, int64_t r, int64_t d_out) {
+  auto up256 = [](size_t v) { return (v + 255) / 256 * 256; };
+  RankPlan g;
+  g.in = plan_gemv(d_in, r, false);
+  g.out = plan_gemv(r, d_out, false);
+  g.off_out = up256(g.in.ws_bytes());
+  g.off_v = g.off_out + up256(g.out.ws_bytes());
+  g.total = g.off_v + up256((size_t)r * 2);
   return g;
 }
 

@@ -140,6 +140,20 @@ def test_multi_validation(lib):
     assert lib.sig_workspace_bytes_multi(0, D, 64) == 0
 
 
+def test_rank_adapter_validation(lib):
+    f = lib.rank_adapter_sparse
+    big = 1 << 30
+    assert f(None, FAKE, FAKE, 64, 32, 16, 0.0, FAKE, None, None, FAKE, big, None) == NULL
+    assert f(FAKE, FAKE, FAKE, 64, 30, 16, 0.0, FAKE, None, None, FAKE, big, None) == SHAPE
+    assert f(FAKE, FAKE, FAKE, 64, 32, 12, 0.0, FAKE, None, None, FAKE, big, None) == SHAPE
+    assert f(FAKE, FAKE_ODD, FAKE, 64, 32, 16, 0.0, FAKE, None, None, FAKE, big, None) == ALIGN
+    need = lib.sig_workspace_bytes(5, 64, 16, 32)
+    assert need > 0
+    assert f(FAKE, FAKE, FAKE, 64, 32, 16, 0.0, FAKE, None, None, FAKE, need - 1, None) == WORKSPACE
+    assert f(FAKE, FAKE, FAKE, 64, 32, 16, 0.0, FAKE, None, None, None, need, None) == WORKSPACE
+    assert lib.sig_workspace_bytes(5, 64, 16, 30) == 0
+
+
 def test_gated_and_gemm_validation(lib):
     g = lib.gated_mlp_sparse
     big = 1 << 30

@@ -36,6 +36,7 @@ __all__ = [
     "LLAMA2_SPARSITIES", "QSPARSE_KEEP_FRACTIONS",
     "draw_weight", "draw_vector", "quantile_threshold", "topk_count",
     "Projection", "projection", "rana_mlp", "nm_tokens", "tiny_gemv", "llama2_7b_layer",
+    "rank_adapter",
 ]
 
 # Llama-2-7B decode projections at batch 1: (name, d_in, d_out).
@@ -177,6 +178,26 @@ def rana_mlp(seed: int = 0, d_model: int = 4096, d_ff: int = 11008,
     WdT = draw_weight(rng, d_ff, d_model, sigma)
     x = draw_vector(rng, d_model, "normal")
     return RanaMLP(WgT, WuT, WdT, x)
+
+
+@dataclass
+class RankAdapter:
+    BT: np.ndarray    # (d_in, r) fp16: B transposed
+    AT: np.ndarray    # (r, d_out) fp16: A transposed
+    x: np.ndarray     # (d_in,) fp16
+
+
+def rank_adapter(seed: int = 0, d_in: int = 4096, r: int = 2048, d_out: int = 4096,
+                 sigma_a: float = 0.02) -> RankAdapter:
+    """Rank adapter factors (B then A) and x ~ Laplace(0, 1).
+
+    B ~ N(0, 1/d_in), so that v = Bx has entries of order one; A ~ N(0, sigma_a^2).
+    """
+    rng = np.random.default_rng(seed)
+    BT = draw_weight(rng, d_in, r, 1.0 / math.sqrt(d_in))
+    AT = draw_weight(rng, r, d_out, sigma_a)
+    x = draw_vector(rng, d_in, "laplace")
+    return RankAdapter(BT, AT, x)
 
 
 def nm_tokens(seed: int = 0, rows: int = 4096, d: int = 1024, d_out: int = 1024,
