@@ -29,6 +29,9 @@ Sources, cited by page title and section:
          whose mask entry is 0; Q4, its masker squares Bx element-wise and
          compares with a threshold (eqn. 9); Q2 to the fourth reviewer, one
          plain GEMV for v = Bx and one masked GEMV for A(m(x) . v).
+* [RaNA] Q6 (batched inference with inconsistent masks) leaves a masked GEMV
+         for batch sizes above one, where every token has its own mask, to
+         future work; the batched product below is that operation.
 * [NM]   "Motivating Next-Gen Accelerators with Flexible (N:M) Activation
          Sparsity ..." (summary), Methodology: in blocks of size M, N non-zero
          elements are kept; selection criterion ACT = absolute activation size.
@@ -66,6 +69,7 @@ __all__ = [
     "masked_matvec", "sparse_linear", "silu", "row_norms", "rana_hidden",
     "rana_scores", "rana_mask", "gated_mlp", "nm_gemm",
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
+    "union_mask", "batched_sparse_linear",
 ]
 
 
@@ -291,6 +295,27 @@ def rank_adapter(x, BT, AT, t: float, cols=None) -> dict:
     out = sparse_linear(AT, v16, m, cols)
     out.update({"v64": v64, "v16": v16, "s32": s32})
     return out
+
+
+# ---------------------------------------------------------------------------
+# A few tokens, each with its own mask ([RaNA] Q6)
+# ---------------------------------------------------------------------------
+
+def union_mask(masks) -> np.ndarray:
+    """Rows any token keeps: the weight rows a batched product must read."""
+    return np.asarray(masks, dtype=bool).any(axis=0)
+
+
+def batched_sparse_linear(WT, X, masks, cols=None) -> dict:
+    """y_b = W (m_b . x_b) for every token b: the single-token product of
+    [RaNA] Q5.1 with token b's own mask ([RaNA] Q6).  Returns stacked
+    ``y64``, ``bound`` (tokens x outputs) and the union of the masks."""
+    X = np.asarray(X)
+    masks = np.asarray(masks, dtype=bool)
+    outs = [masked_matvec(WT, X[b], masks[b], cols) for b in range(X.shape[0])]
+    y64 = np.stack([o[0] for o in outs]) if outs else np.zeros((0, 0))
+    bound = np.stack([o[1] for o in outs]) if outs else np.zeros((0, 0))
+    return {"y64": y64, "y16": fp16(y64), "bound": bound, "union": union_mask(masks)}
 
 
 # ---------------------------------------------------------------------------

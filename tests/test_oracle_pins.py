@@ -537,3 +537,54 @@ def test_rank_adapter_masked_rows_do_not_matter():
     v16 = dense["v16"].astype(np.float64)
     want = [sum(v16[i] * float(AT[i, j]) for i in range(r)) for j in range(d_out)]
     assert np.allclose(dense["y64"], want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# A few tokens with their own masks
+# ---------------------------------------------------------------------------
+
+def test_batched_tokens_golden():
+    WT, xs, ms, ys, t, union = [], [], [], [], None, None
+    for ln in _read_lines("batched_tokens_tiny.txt"):
+        if ln.startswith("WT:"):
+            WT.append(_floats(ln[3:]))
+        elif ln.startswith("t:"):
+            t = float(ln[2:])
+        elif ln.startswith("union:"):
+            union = [int(v) for v in ln[6:].split()]
+        elif ln.startswith("x:"):
+            x, m, y = ln[2:].split("|")
+            xs.append(_floats(x)); ms.append([int(v) for v in m.split()]); ys.append(_floats(y))
+    WT = np.array(WT, np.float16)
+    X = np.array(xs, np.float16)
+    masks = np.stack([oracle.threshold_mask(x, t) for x in X])
+    assert masks.astype(int).tolist() == ms
+    out = oracle.batched_sparse_linear(WT, X, masks)
+    assert out["y64"].tolist() == ys
+    assert out["union"].astype(int).tolist() == union
+
+
+def test_batched_tokens_properties():
+    """One token is the single-token product; permuting tokens permutes the
+    outputs; rows outside the union never matter; identical tokens agree."""
+    rng = np.random.default_rng(31)
+    d_in, d_out, B = 96, 40, 5
+    WT = rng.normal(0, 0.05, (d_in, d_out)).astype(np.float16)
+    X = rng.laplace(0, 1, (B, d_in)).astype(np.float16)
+    t = 1.2
+    masks = np.stack([oracle.threshold_mask(x, t) for x in X])
+    out = oracle.batched_sparse_linear(WT, X, masks)
+    one = oracle.sparse_linear(WT, X[2], masks[2])
+    assert np.array_equal(out["y64"][2], one["y64"])
+    perm = np.array([3, 0, 4, 1, 2])
+    outp = oracle.batched_sparse_linear(WT, X[perm], masks[perm])
+    assert np.array_equal(outp["y64"], out["y64"][perm])
+    assert 0 < out["union"].sum() < d_in
+    WT2 = WT.copy()
+    WT2[~out["union"]] = np.float16(500.0)
+    assert np.array_equal(oracle.batched_sparse_linear(WT2, X, masks)["y64"], out["y64"])
+    Xs = np.repeat(X[:1], 3, axis=0)
+    ms = np.repeat(masks[:1], 3, axis=0)
+    same = oracle.batched_sparse_linear(WT, Xs, ms)["y64"]
+    assert np.array_equal(same[0], same[1]) and np.array_equal(same[1], same[2])
+    assert np.array_equal(oracle.union_mask(ms), masks[0])
