@@ -16,7 +16,7 @@ no step finds its weights in L2 (580 MB of kept rows per rotation, > 4x L2).
 Steps are replayed CUDA graphs, timed with CUDA events on the launching stream.
 
 The JSON line also carries the sparsity sweep, the top-k (Q-Sparse 70B), RaNA
-gated-MLP, RaNA rank-adapter and N:M GEMM rows, cuBLAS dense baselines at the same shapes, the
+gated-MLP, RaNA rank-adapter, per-token-mask batch and N:M GEMM rows, cuBLAS dense baselines at the same shapes, the
 roofline of the sparse GEMV kernel, the oracle's CPU baseline and the SM
 clocks sampled during the timed region.
 
@@ -414,6 +414,7 @@ def run_ours(args, rank, world, local):
         extras["rana_gated_mlp"] = bench_rana(args, stream, sig, hbm_peak)
         extras["nm_gemm"] = bench_nm(args, stream, sig, bf16_peak)
         extras["rana_rank_adapter"] = bench_rank_adapter(args, stream, sig, hbm_peak)
+        extras["batched_per_token_masks"] = bench_batch(args, stream, sig, hbm_peak)
         result["extras"] = extras
         result["cpu_baseline"] = cpu_baseline(groups)
     return result
@@ -607,6 +608,53 @@ def bench_rank_adapter(args, stream, sig, hbm_peak):
     del Bs, As, W, sg, sd
     torch.cuda.empty_cache()
     return res
+
+
+def bench_batch(args, stream, sig, hbm_peak):
+    """A few tokens with their own 50 % threshold masks through the gate-shaped
+    weight (4096 -> 11008): one batched launch that reads the union of the
+    kept rows once, against one single-token launch per token."""
+    import torch
+    out = {"shape": "4096->11008", "l2": "6 rotating weight copies (541 MB)"}
+    copies = 6
+    for B in (2, 4, 8):
+        WT, X, t = workloads.batch_tokens(seed=args.seed + B, B=B)
+        Ws = [torch.from_numpy(WT).cuda()]
+        Ws += [Ws[0].clone() for _ in range(copies - 1)]
+        Xd = torch.from_numpy(X).cuda()
+        Y = torch.empty((B, WT.shape[1]), dtype=torch.float16, device="cuda")
+        ws = torch.zeros(max(256, sig.workspace_bytes(sig.OP_SPARSE_GEMV_BATCH, WT.shape[0],
+                                                      WT.shape[1], B)), dtype=torch.uint8, device="cuda")
+        m = np.abs(X.astype(np.float32)) >= t
+        union = int(m.any(axis=0).sum())
+
+        def f(c, B=B):
+            def g():
+                sig.sparse_gemv_batch(Ws[c], Xd, t, Y=Y, ws=ws, stream=stream)
+            return g
+        sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies * 2)
+        steps = 240
+        us = time_steps(sg, steps, copies, stream) / steps * 1e6
+        d_in, d_out = WT.shape
+        b = union * 2 * d_out + B * (2 * d_in + 2 * d_out)
+        ys = [torch.empty(d_out, dtype=torch.float16, device="cuda") for _ in range(B)]
+        wss = [torch.zeros(max(256, sig.workspace_bytes(sig.OP_SPARSE_GEMV, d_in, d_out)),
+                           dtype=torch.uint8, device="cuda") for _ in range(B)]
+
+        def h(c, B=B):
+            def g():
+                for j in range(B):
+                    sig.sparse_gemv(Ws[c], Xd[j], t=t, y=ys[j], ws=wss[j], stream=stream)
+            return g
+        sh = StepGraphs([h(c) for c in range(copies)], stream, per_graph=copies * 2)
+        us_sep = time_steps(sh, steps, copies, stream) / steps * 1e6
+        out[f"B={B}"] = {"union_density": round(union / d_in, 4), "us": round(us, 2),
+                         "GBps": round(b / (us * 1e-6) / 1e9, 1),
+                         "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
+                         "separate_single_token_launches_us": round(us_sep, 2)}
+        del Ws, sg, sh
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_nm(args, stream, sig, bf16_peak):

@@ -74,7 +74,8 @@ typedef enum {
   SIG_OP_TOPK = 2,         /* sparsify_topk(d = d_in)                  */
   SIG_OP_GATED_MLP = 3,    /* gated_mlp_sparse(d_model = d_in, d_ff = d_out) */
   SIG_OP_NM_GEMM = 4,      /* nm_act_gemm(K = d_in, N = d_out, rows)   */
-  SIG_OP_RANK_ADAPTER = 5  /* rank_adapter_sparse(d_in, d_out, rows = r) */
+  SIG_OP_RANK_ADAPTER = 5, /* rank_adapter_sparse(d_in, d_out, rows = r) */
+  SIG_OP_SPARSE_GEMV_BATCH = 6 /* sparse_gemv_batch(d_in, d_out, rows = tokens) */
 } sig_op;
 
 /* Largest activation length the fused mask prologue accepts. */
@@ -224,6 +225,28 @@ SIG_API int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint1
                      int64_t d_model, int64_t d_ff, float t,
                      uint16_t* y, uint16_t* h_out, uint32_t* mask_out,
                      void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * A few tokens, each with its own threshold mask, through one weight:
+ *   y_b = W (m_b . x_b),  m_b,i = |x_b,i| >= t,  b < B.
+ * The product is the single-token one of sparse_gemv (RaNA rebuttal, Q5.1);
+ * batches with inconsistent masks are the open case of the same rebuttal (Q6).
+ * One launch reads every weight row that any token keeps (the union of the
+ * masks) once and applies each token's own mask to it; same tolerance and
+ * determinism as sparse_gemv for every token.
+ *   WT [d_in x d_out] fp16.  X [B x d_in] fp16, row-major.  Y [B x d_out] fp16 out.
+ *   ws sig_workspace_bytes(SIG_OP_SPARSE_GEMV_BATCH, d_in, d_out, B) bytes
+ *      (0 means none is needed and ws may be NULL), 256-byte aligned, zeroed
+ *      once before first use; every call leaves it ready for the next.
+ * 1 <= B <= SIG_MAX_BATCH; d_in % 8 == 0 (whole 16-byte groups per token row),
+ * d_in <= SIG_MAX_D_IN; d_out % 8 == 0.
+ * Errors: SIG_ERR_NULL, SIG_ERR_ARG (B), SIG_ERR_SHAPE, SIG_ERR_ALIGN,
+ *         SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
+ */
+#define SIG_MAX_BATCH 8
+SIG_API int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out,
+                              const uint16_t* X, int64_t B, float t, uint16_t* Y,
+                              void* ws, size_t ws_bytes, sig_stream_t stream);
 
 /*
  * RaNA linear-layer rank adapter (RaNA rebuttal, Q5.1: Linear(x) ~ A (m(x) . Bx),

@@ -23,11 +23,14 @@ __all__ = [
     "sparsify_topk", "sparsify_nm", "sparse_gemv", "gated_mlp_sparse", "row_norms",
     "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
     "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
+    "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
 
 OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM, OP_RANK_ADAPTER = 1, 2, 3, 4, 5
+OP_SPARSE_GEMV_BATCH = 6
+MAX_BATCH = 8
 MAX_D_IN = 131072
 
 _p, _i64, _i32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
@@ -50,6 +53,7 @@ _SIGNATURES = {
     "sparse_gemv_multi": (_i32, [_i32, _p, _p, _i64, _p, _f32, _p, _p, _p, _p, _sz, _p]),
     "sig_workspace_bytes_multi": (_sz, [_i32, _p, _i64]),
     "rank_adapter_sparse": (_i32, [_p, _p, _p, _i64, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
+    "sparse_gemv_batch": (_i32, [_p, _i64, _i64, _p, _i64, _f32, _p, _p, _sz, _p]),
 }
 
 
@@ -240,6 +244,24 @@ def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
         _ptr(y), _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
     return y
+
+
+def sparse_gemv_batch(WT, X, t: float, Y=None, ws=None, stream=None):
+    """Y[b] = W (m_b . X[b]), m_b = |X[b]| >= t, for B <= MAX_BATCH tokens in one launch."""
+    _need(WT, torch.float16, "WT")
+    _need(X, torch.float16, "X", WT.device)
+    if X.dim() != 2 or X.shape[1] != WT.shape[0]:
+        raise ValueError("X must be (B, d_in) with d_in = WT.shape[0]")
+    B, d_in = X.shape
+    d_out = WT.shape[1]
+    if Y is None:
+        Y = torch.empty((B, d_out), dtype=torch.float16, device=WT.device)
+    if ws is None:
+        ws = workspace(OP_SPARSE_GEMV_BATCH, d_in, d_out, B, device=WT.device, stream=stream)
+    _check("sparse_gemv_batch", _lib.sparse_gemv_batch(
+        _ptr(WT), d_in, d_out, _ptr(X), B, float(t), _ptr(Y), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return Y
 
 
 def rank_adapter_sparse(x, BT, AT, t: float, y=None, v_out=None, mask_out=None, ws=None,

@@ -66,6 +66,11 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
       if (check_gemv_shape(d_in, rows) != SIG_OK || check_gemv_shape(rows, d_out) != SIG_OK)
         return 0;
       return plan_rank(d_in, rows, d_out).total;
+    case SIG_OP_SPARSE_GEMV_BATCH:
+      if (check_gemv_shape(d_in, d_out) != SIG_OK || d_in % 8 != 0 || rows < 1 ||
+          rows > kGemvMaxBatch)
+        return 0;
+      return plan_gemv_batch(d_in, d_out, (int)rows).ws_bytes();
     case SIG_OP_NM_GEMM:
       if (rows < 1 || d_in < 1) return 0;
       return round_up((size_t)rows * (size_t)d_in * 2, 256);   // the masked activation block
@@ -129,6 +134,22 @@ int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t*
   a.x = x; a.t = t; a.idx = idx; a.nnz = nnz; a.d_in = (int)d_in; a.ws = ws;
   return cuda_status(launch_gemv(idx == nullptr ? MASK_THRESH : MASK_IDX, EPI_STORE, p, a,
                                  (cudaStream_t)stream));
+}
+
+int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t* X,
+                      int64_t B, float t, uint16_t* Y, void* ws, size_t ws_bytes,
+                      sig_stream_t stream) {
+  if (WT == nullptr || X == nullptr || Y == nullptr) return SIG_ERR_NULL;
+  if (B < 1 || B > kGemvMaxBatch) return SIG_ERR_ARG;
+  const int sh = check_gemv_shape(d_in, d_out);
+  if (sh != SIG_OK) return sh;
+  if (d_in % 8 != 0) return SIG_ERR_SHAPE;
+  if (!aligned16(WT) || !aligned16(X) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  const GemvPlan p = plan_gemv_batch(d_in, d_out, (int)B);
+  if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
+  return cuda_status(launch_gemv_batch(p, WT, X, Y, (int)B, (int)d_in, (int)d_out, t, ws,
+                                       (cudaStream_t)stream));
 }
 
 size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in) {

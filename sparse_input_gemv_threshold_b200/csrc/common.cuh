@@ -17,9 +17,6 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// L2 policy for data read exactly once (weight rows): evict first, so that
-// the stream does not push the small reused buffers (x, index lists, split-K
-// partials, counters) out of L2.
 // Atomic add with acquire-release semantics at GPU scope: publishes the
 // writes that the CTA made before a preceding __syncthreads, and makes the
 // writes published by earlier arrivers visible to the CTA after the next one.
@@ -29,6 +26,9 @@ __device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned
   return old;
 }
 
+// L2 policy for data read exactly once (weight rows): evict first, so that
+// the stream does not push the small reused buffers (x, index lists, split-K
+// partials, counters) out of L2.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
   asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -61,6 +61,25 @@ __device__ __forceinline__ void fma8(float (&acc)[8], const uint4& v, float xv) 
     acc[2 * k] = fmaf(f.x, xv, acc[2 * k]);
     acc[2 * k + 1] = fmaf(f.y, xv, acc[2 * k + 1]);
   }
+}
+
+// 8 mask bits for the 8 fp16 values in v: |x| >= th (th = t rounded up to
+// fp16, exact for fp16 inputs; NaN never passes an ordered compare).
+__device__ __forceinline__ uint32_t thresh_bits8(const uint4& v, __half2 th2) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t b = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t m = __hge2_mask(__habs2(*reinterpret_cast<const __half2*>(&w[q])), th2);
+    b |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
+  }
+  return b;
+}
+
+// The threshold as the fp16 pair thresh_bits8 compares against: t rounded up
+// to fp16, or 0 for t <= 0 (every number passes).
+__device__ __forceinline__ __half2 thresh_half2(float t) {
+  return __half2half2(t <= 0.f ? __float2half(0.f) : __float2half_ru(t));
 }
 
 // fp16 element k (0..7) of a 16-byte vector.

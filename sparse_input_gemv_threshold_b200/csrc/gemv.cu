@@ -66,19 +66,6 @@ struct KArgs {
   float* partials;        // [S][d_out_total] (then the same again for the second product)
 };
 
-// 8 mask bits for the 8 fp16 values in v: |x| >= th (th = t rounded up to
-// fp16; NaN never passes an ordered compare).
-__device__ __forceinline__ uint32_t thresh_bits8(const uint4& v, __half2 th2) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t b = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t m = __hge2_mask(__habs2(*reinterpret_cast<const __half2*>(&w[q])), th2);
-    b |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
-  }
-  return b;
-}
-
 // Mask bits of the 8-input groups this slice owns.  Group g covers inputs
 // 8g .. 8g+7; slice s owns groups s, s + S, s + 2S, ... (K of them), four to
 // a local word: bit 8q + b of local word lw is input 8 (s + (4 lw + q) S) + b.
@@ -87,7 +74,7 @@ __device__ __forceinline__ void build_local_words(const KArgs& a, int s, int K, 
                                                   uint32_t* words) {
   const int d_in = a.d_in, S = a.S;
   const float t = a.t;
-  const __half2 th2 = __half2half2(t <= 0.f ? __float2half(0.f) : __float2half_ru(t));
+  const __half2 th2 = thresh_half2(t);
   for (int lw = threadIdx.x; lw < nlw; lw += kThreads) {
     uint4 v[4];
 #pragma unroll

@@ -140,6 +140,23 @@ def test_multi_validation(lib):
     assert lib.sig_workspace_bytes_multi(0, D, 64) == 0
 
 
+def test_batch_validation(lib):
+    f = lib.sparse_gemv_batch
+    big = 1 << 30
+    assert f(None, 64, 64, FAKE, 2, 0.0, FAKE, FAKE, big, None) == NULL
+    assert f(FAKE, 64, 64, FAKE, 0, 0.0, FAKE, FAKE, big, None) == ARG
+    assert f(FAKE, 64, 64, FAKE, 9, 0.0, FAKE, FAKE, big, None) == ARG
+    assert f(FAKE, 60, 64, FAKE, 2, 0.0, FAKE, FAKE, big, None) == SHAPE     # d_in % 8
+    assert f(FAKE, 64, 60, FAKE, 2, 0.0, FAKE, FAKE, big, None) == SHAPE     # d_out % 8
+    assert f(FAKE, 64, 64, FAKE_ODD, 2, 0.0, FAKE, FAKE, big, None) == ALIGN
+    need = lib.sig_workspace_bytes(6, 64, 64, 2)
+    assert need > 0
+    assert f(FAKE, 64, 64, FAKE, 2, 0.0, FAKE, FAKE, need - 1, None) == WORKSPACE
+    assert f(FAKE, 64, 64, FAKE, 2, 0.0, FAKE, None, need, None) == WORKSPACE
+    assert lib.sig_workspace_bytes(6, 64, 64, 9) == 0
+    assert lib.sig_workspace_bytes(6, 60, 64, 2) == 0
+
+
 def test_rank_adapter_validation(lib):
     f = lib.rank_adapter_sparse
     big = 1 << 30

@@ -36,7 +36,7 @@ __all__ = [
     "LLAMA2_SPARSITIES", "QSPARSE_KEEP_FRACTIONS",
     "draw_weight", "draw_vector", "quantile_threshold", "topk_count",
     "Projection", "projection", "rana_mlp", "nm_tokens", "tiny_gemv", "llama2_7b_layer",
-    "rank_adapter",
+    "rank_adapter", "batch_tokens",
 ]
 
 # Llama-2-7B decode projections at batch 1: (name, d_in, d_out).
@@ -178,6 +178,17 @@ def rana_mlp(seed: int = 0, d_model: int = 4096, d_ff: int = 11008,
     WdT = draw_weight(rng, d_ff, d_model, sigma)
     x = draw_vector(rng, d_model, "normal")
     return RanaMLP(WgT, WuT, WdT, x)
+
+
+def batch_tokens(seed: int = 0, B: int = 4, d_in: int = 4096, d_out: int = 11008,
+                 sigma: float = 0.02, sparsity: float = 0.5):
+    """A weight WT (d_in, d_out) then B Laplace tokens X (B, d_in), and one
+    threshold shared by the tokens: the ``sparsity`` quantile of the pooled
+    |X| (a per-layer calibrated threshold, as TEAL uses for every token)."""
+    rng = np.random.default_rng(seed)
+    WT = draw_weight(rng, d_in, d_out, sigma)
+    X = draw_vector(rng, (B, d_in), "laplace")
+    return WT, X, quantile_threshold(X, sparsity)
 
 
 @dataclass
