@@ -8,20 +8,23 @@
 // the masks) once from HBM and applies each token's own mask to it in
 // registers: a row that token b drops contributes x_b,i = 0 to y_b.
 //
-// Launch shape, as the single-token kernel: C x S CTAs of 256 threads, a CTA
-// owns a 256-output column tile (one warp spans it with 16-byte lanes) and
-// the union rows of its interleaved 8-input groups (slice s owns groups s,
-// s+S, s+2S, ...), staged in shared memory with the tokens' masked values:
-//   1. the CTA loads its groups of every token's x (from L2), ballots the
-//      union of their fp16 threshold compares into shared words, prefix-sums
-//      the words' popcounts and places the union rows in ascending order,
-//      each with the NB masked token values (0 where that token drops it);
-//   2. 8 warps stream the rows of the tile, 6 or 8 in flight per warp, FMA
-//      into NB x 8 float32 accumulators per lane;
-//   3. per token, the warps' sums meet in shared memory, the CTA writes one
-//      partial per column, and the last CTA to arrive for the tile (one
-//      acquire-release atomic per CTA) adds the S partials of every token in
-//      slice order and stores fp16.
+// Launch shape: C x S CTAs of 256 threads (three per SM), a CTA owns a
+// 256-output column tile and the union rows of its interleaved 8-input
+// groups (slice s owns groups s, s+S, s+2S, ...):
+//   1. one thread per group loads that group of every token's x (from L2,
+//      all tokens' loads in flight together) and ORs their fp16 threshold
+//      compares into a union byte; the popcounts are prefix-summed and the
+//      union rows placed in ascending order, with the tokens' masked values
+//      staged token-major (0 where a token drops the row);
+//   2. for a column tile the work is a small dense contraction,
+//      Y^T (256 outputs x 8 tokens) += W^T rows (256 x 16) . Xm (16 x 8) per
+//      step of 16 union rows, which the warp-level mma.m16n8k16 (fp16 in,
+//      float32 accumulate) takes directly: the weight rows reach shared
+//      memory through a multi-stage cp.async pipeline, each warp owns 32
+//      output columns and runs every row of the slice, so warps never meet;
+//   3. the CTA writes one partial per (token, column), and the last CTA to
+//      arrive for the tile (one acquire-release atomic per CTA) adds the S
+//      partials of every token in slice order and stores fp16.
 // Deterministic: no floating-point atomics, no spin-waits.
 #include "common.cuh"
 #include "internal.h"
@@ -41,20 +44,54 @@ struct BArgs {
   const uint16_t* X;      // B x d_in, row-major
   uint16_t* Y;            // B x d_out, row-major
   float t;
-  int B, d_in, d_out, S, chunk;
+  int B, d_in, d_out, S;
   uint32_t words_bytes;   // shared bytes of the union words (and again of their prefixes)
-  uint32_t union_bytes;   // shared bytes of words + prefixes / the warp-sum buffer
+  uint32_t union_bytes;   // shared bytes of words + prefixes; the stages follow
   unsigned* counters;     // [C]
   float* partials;        // [S][B][d_out]
 };
 
-// CTAs per SM each width is sized for (registers: NB x 8 accumulators).
-template <int NB>
-constexpr int ctas_per_sm() { return NB <= 2 ? 4 : NB <= 4 ? 3 : 2; }
+// Shared-memory staging: weight rows padded to 528 bytes so that the
+// transposing ldmatrix reads are free of bank conflicts; padding rows of a
+// step and columns past d_out are written as zeros by plain shared stores.
+// Tokens' masked values are staged token-major, padded rows apart likewise.
 
-template <int NB>
-__global__ void __launch_bounds__(kThreads, ctas_per_sm<NB>())
-batch_gemv_kernel(const __grid_constant__ BArgs a) {
+constexpr int kMmaStages = 5;
+constexpr int kMmaRows = 16;                      // union rows per step
+constexpr int kMmaRowBytes = kTile * 2 + 16;      // 528: padded shared row
+constexpr int kMmaStageBytes = kMmaRows * kMmaRowBytes;
+constexpr int kMmaChunk = 1024;                   // union rows staged per chunk
+constexpr int kMmaXtStride = kMmaChunk * 2 + 16;  // bytes between token rows of staged values
+constexpr int kMmaCtasPerSM = 3;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+               "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__global__ void __launch_bounds__(kThreads, kMmaCtasPerSM)
+batch_mma_kernel(const __grid_constant__ BArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_tot[kWarps];
   __shared__ int s_last;
@@ -62,34 +99,39 @@ batch_gemv_kernel(const __grid_constant__ BArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, s = blockIdx.y;
   const int d_in = a.d_in, d_out = a.d_out, S = a.S, B = a.B;
+  constexpr int xt_stride = kMmaXtStride;
 
   uint32_t* words = reinterpret_cast<uint32_t*>(smem);
   int* wpre = reinterpret_cast<int*>(smem + a.words_bytes);
-  int* sidx = reinterpret_cast<int*>(smem + a.union_bytes);
-  uint16_t* sxv = reinterpret_cast<uint16_t*>(smem + a.union_bytes + (size_t)a.chunk * 4);
+  unsigned char* stages = smem + a.union_bytes;
+  int* sidx = reinterpret_cast<int*>(stages + kMmaStages * kMmaStageBytes);
+  unsigned char* sxt = reinterpret_cast<unsigned char*>(sidx + kMmaChunk);   // 8 x kMmaXtStride bytes
 
   pdl_trigger();
   pdl_wait();
 
-  // ---- 1. the union of the tokens' masks over this slice's groups -------
+  // ---- 1. union of the tokens' masks over this slice's groups ----------
   const __half2 th2 = thresh_half2(a.t);
-  const int ngroups = (d_in + 7) >> 3;    // d_in % 8 == 0: whole groups
+  const float th = __half2float(__low2half(th2));
+  const int ngroups = (d_in + 7) >> 3;
   const int K = s < ngroups ? (ngroups - 1 - s) / S + 1 : 0;
   const int nwords = (K + 3) >> 2;
-  for (int lw = tid; lw < nwords; lw += kThreads) {
-    uint32_t w = 0;
+  // one thread per group: every token's loads in flight together
+  uint8_t* wbytes = reinterpret_cast<uint8_t*>(words);
+  for (int k = tid; k < nwords * 4; k += kThreads) {
+    uint32_t u = 0;
+    if (k < K) {
+      const int e0 = (s + k * S) * 8;
+      uint4 v[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int k = lw * 4 + q;
-      if (k < K) {
-        const int e0 = (s + k * S) * 8;
-        uint32_t u = 0;
-        for (int b = 0; b < B; ++b)
-          u |= thresh_bits8(__ldg(reinterpret_cast<const uint4*>(a.X + (size_t)b * d_in + e0)), th2);
-        w |= u << (8 * q);
-      }
+      for (int b = 0; b < 8; ++b)
+        v[b] = b < B ? __ldg(reinterpret_cast<const uint4*>(a.X + (size_t)b * d_in + e0))
+                     : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (b < B) u |= thresh_bits8(v[b], th2);
     }
-    words[lw] = w;
+    wbytes[k] = (uint8_t)u;
   }
   __syncthreads();
   const int per = (nwords + kThreads - 1) / kThreads;
@@ -118,22 +160,43 @@ batch_gemv_kernel(const __grid_constant__ BArgs a) {
   }
   __syncthreads();
 
-  // ---- 2. stream the union rows of this column tile ---------------------
-  const int col = c * kTile + lane * 8;
-  const bool col_ok = col < d_out;
-  const uint16_t* wp = a.WT + col;
-  const uint64_t pol = l2_evict_first_policy();
-  float acc[NB][8];
+  // ---- 2. the contraction over the union rows ---------------------------
+  const int tile0 = c * kTile;
+  float acc[2][4];
 #pragma unroll
-  for (int b = 0; b < NB; ++b)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[b][k] = 0.f;
-  constexpr int U = NB == 8 ? 8 : 6;   // rows in flight per warp (registers: NB x 8 accumulators)
+    for (int k = 0; k < 4; ++k) acc[mt][k] = 0.f;
 
-  for (int cb = 0; cb < total; cb += a.chunk) {
-    const int c_lo = cb, c_hi = min(total, cb + a.chunk), cn = c_hi - c_lo;
-    if (cb > 0) __syncthreads();   // the previous chunk's rows are no longer read
-    // one word per warp, one bit per lane; the row's masked token values beside it
+  // this thread's two 16-byte pieces of every staged step (row, 16-byte column)
+  int cp_row[2], cp_col[2];
+  bool cp_in[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int q = tid + kThreads * e;
+    cp_row[e] = q >> 5;
+    cp_col[e] = q & 31;
+    cp_in[e] = tile0 + cp_col[e] * 8 < d_out;
+  }
+  // rows past the chunk's end and columns past d_out are zeros in shared memory
+  auto issue_step = [&](int step, int cn) {
+    unsigned char* st = stages + (step % kMmaStages) * kMmaStageBytes;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = step * kMmaRows + cp_row[e];
+      unsigned char* dst = st + cp_row[e] * kMmaRowBytes + cp_col[e] * 16;
+      if (j < cn && cp_in[e])
+        cp_async16(smem_u32(dst), a.WT + (size_t)sidx[j] * d_out + tile0 + cp_col[e] * 8);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+  };
+
+  for (int cb = 0; cb < total; cb += kMmaChunk) {
+    const int c_lo = cb, c_hi = min(total, cb + kMmaChunk), cn = c_hi - c_lo;
+    const int nsteps = (cn + kMmaRows - 1) / kMmaRows;
+    if (cb > 0) __syncthreads();   // every read of the previous chunk is over
+    // union rows of this chunk, and the tokens' masked values token-major
     for (int w = warp; w < nwords; w += kWarps) {
       const int base = wpre[w];
       if (base >= c_hi) break;                       // uniform across the warp
@@ -141,120 +204,123 @@ batch_gemv_kernel(const __grid_constant__ BArgs a) {
       const int rk = base + __popc(bits & ((1u << lane) - 1u));
       if (((bits >> lane) & 1u) && rk >= c_lo && rk < c_hi) {
         const int i = (s + (w * 4 + (lane >> 3)) * S) * 8 + (lane & 7);
-        sidx[rk - c_lo] = i;
-        uint16_t* dst = sxv + (size_t)(rk - c_lo) * NB;
+        const int j = rk - c_lo;
+        sidx[j] = i;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
+        for (int b = 0; b < 8; ++b) {
           uint16_t h = 0;
           if (b < B) {
             h = a.X[(size_t)b * d_in + i];
-            if (!(fabsf(h2f(h)) >= __half2float(__low2half(th2)))) h = 0;
+            if (!(fabsf(h2f(h)) >= th)) h = 0;
           }
-          dst[b] = h;
+          *reinterpret_cast<uint16_t*>(sxt + b * xt_stride + j * 2) = h;
         }
       }
+    }
+    // zero values for the padding rows of the last step
+    for (int q = tid; q < 8 * kMmaRows; q += kThreads) {
+      const int j = cn + (q % kMmaRows);
+      if (j < nsteps * kMmaRows) *reinterpret_cast<uint16_t*>(sxt + (q / kMmaRows) * xt_stride + j * 2) = 0;
     }
     __syncthreads();
-    if (col_ok) {
-      for (int j0 = warp; j0 < cn; j0 += kWarps * U) {
-        uint4 v[U];
+
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int j = j0 + kWarps * u;
-          v[u] = j < cn ? ld_stream_v4(wp + (size_t)sidx[j] * d_out, pol) : make_uint4(0, 0, 0, 0);
-        }
+    for (int st = 0; st < kMmaStages - 1; ++st) {
+      if (st < nsteps) issue_step(st, cn);
+      cp_async_commit();
+    }
+    for (int ks = 0; ks < nsteps; ++ks) {
+      cp_async_wait<kMmaStages - 2>();
+      __syncthreads();                 // step ks has landed; step ks-1's stage is free
+      if (ks + kMmaStages - 1 < nsteps) issue_step(ks + kMmaStages - 1, cn);
+      cp_async_commit();
+      __syncwarp();                    // the fragment loads and MMAs below are warp-wide
+      const unsigned char* stg = stages + (ks % kMmaStages) * kMmaStageBytes;
+      uint32_t bf[2];
+      {
+        const int n = lane & 7, kh = (lane >> 3) & 1;
+        ldsm_x2(bf, smem_u32(sxt + n * xt_stride + (ks * kMmaRows + kh * 8) * 2));
+      }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int j = j0 + kWarps * u;
-          if (j < cn) {
-            const uint16_t* xs = sxv + (size_t)j * NB;
-#pragma unroll
-            for (int b = 0; b < NB; ++b) fma8(acc[b], v[u], h2f(xs[b]));
-          }
-        }
+      for (int mt = 0; mt < 2; ++mt) {
+        const int q = lane >> 3, r = lane & 7;
+        const int m = warp * 32 + mt * 16 + (q & 1) * 8;
+        uint32_t af[4];
+        ldsm_x4_trans(af, smem_u32(stg + ((q >> 1) * 8 + r) * kMmaRowBytes + m * 2));
+        mma_16816(acc[mt], af, bf);
       }
     }
+    cp_async_wait<0>();
   }
 
-  // ---- 3. per token: CTA partial; the last arriver finishes the tile ----
-  float* red = reinterpret_cast<float*>(smem);
-  const int colr = c * kTile + tid;
-  const bool colr_ok = colr < d_out;
-  float p[NB];
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    __syncthreads();   // the previous use of the buffer is over
-    float4* r4 = reinterpret_cast<float4*>(red + warp * kTile + lane * 8);
-    r4[0] = make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
-    r4[1] = make_float4(acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
-    __syncthreads();
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) sum += red[w * kTile + tid];
-    p[b] = sum;
-  }
+  // ---- 3. this CTA's partials; the last arriver finishes the tile -------
+  const int g = lane >> 2, t4 = lane & 3;
   if (S == 1) {
-    if (colr_ok) {
 #pragma unroll
-      for (int b = 0; b < NB; ++b)
-        if (b < B) a.Y[(size_t)b * d_out + colr] = f2h_rn(p[b]);
-    }
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = tile0 + warp * 32 + mt * 16 + g + h * 8;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int n = t4 * 2 + e;
+          if (col < d_out && n < B) a.Y[(size_t)n * d_out + col] = f2h_rn(acc[mt][h * 2 + e]);
+        }
+      }
     return;
   }
-  if (colr_ok) {
 #pragma unroll
-    for (int b = 0; b < NB; ++b)
-      if (b < B) a.partials[((size_t)s * B + b) * d_out + colr] = p[b];
-  }
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int col = tile0 + warp * 32 + mt * 16 + g + h * 8;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = t4 * 2 + e;
+        if (col < d_out && n < B)
+          a.partials[((size_t)s * B + n) * d_out + col] = acc[mt][h * 2 + e];
+      }
+    }
   __syncthreads();
   if (tid == 0) s_last = atomic_add_acq_rel_gpu(a.counters + c, 1u) == (unsigned)(S - 1);
   __syncthreads();
   if (!s_last) return;
-  if (colr_ok) {
-    for (int b = 0; b < B; ++b) {
-      const float* pp = a.partials + (size_t)b * d_out + colr;
-      float g = 0.f;
-      for (int q0 = 0; q0 < S; q0 += 32) {
-        float pg[32];
+  const int colr = tile0 + tid;
+  if (colr < d_out) {
+    // every token's partials of a slice in flight together, two slices at a
+    // time; each token's sum still runs in slice order
+    float sum[8];
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          pg[k] = q0 + k < S ? __ldcg(pp + (size_t)(q0 + k) * B * d_out) : 0.f;
+    for (int b = 0; b < 8; ++b) sum[b] = 0.f;
+    const size_t slice_stride = (size_t)B * d_out;
+    const float* pp = a.partials + colr;
+#pragma unroll 2
+    for (int q = 0; q < S; ++q) {
+      float v[8];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) g += pg[k];
-      }
-      a.Y[(size_t)b * d_out + colr] = f2h_rn(g);
+      for (int b = 0; b < 8; ++b) v[b] = b < B ? __ldcg(pp + q * slice_stride + (size_t)b * d_out) : 0.f;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) sum[b] += v[b];
     }
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+      if (b < B) a.Y[(size_t)b * d_out + colr] = f2h_rn(sum[b]);
   }
   if (tid == 0) a.counters[c] = 0u;  // ready for the next call on this workspace
 }
 
 size_t round_up(size_t v, size_t al) { return (v + al - 1) / al * al; }
 
-int width_for(int B) { return B <= 2 ? 2 : B <= 4 ? 4 : 8; }
-
-template <int NB>
-cudaError_t launch_nb(const GemvPlan& p, const BArgs& k, cudaStream_t stream) {
-  auto fn = batch_gemv_kernel<NB>;
-  cudaError_t e =
-      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(fn, dim3(p.C, p.S), dim3(kThreads), p.smem, stream, k);
-}
-
 }  // namespace
 
 GemvPlan plan_gemv_batch(int64_t d_in, int64_t d_out, int B) {
   GemvPlan p{};
-  const int nb = width_for(B);
-  const int cps = nb <= 2 ? 4 : nb <= 4 ? 3 : 2;
   p.C = (int)((d_out + kTile - 1) / kTile);
-  p.S = std::max(1, std::min(32, (kNumSMs * cps) / std::max(1, p.C)));
-  const int64_t groups = (d_in + 7) / 8;
-  p.chunk = (int)std::max<int64_t>(1, std::min<int64_t>((groups + p.S - 1) / p.S * 8, 2048));
+  p.S = std::max(1, std::min(32, (kNumSMs * kMmaCtasPerSM) / std::max(1, p.C)));
+  p.chunk = kMmaChunk;
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
-  const size_t red = (size_t)kWarps * kTile * 4;
-  p.smem = std::max(2 * words, red) + round_up((size_t)p.chunk * 4, 16) +
-           round_up((size_t)p.chunk * nb * 2, 16);
+  p.smem = 2 * words + (size_t)kMmaStages * kMmaStageBytes + (size_t)kMmaChunk * 4 +
+           (size_t)8 * kMmaXtStride;
   p.counters = p.S > 1 ? round_up((size_t)p.C * 4, 256) : 0;
   p.partials = p.S > 1 ? round_up((size_t)p.S * B * d_out * 4, 256) : 0;
   return p;
@@ -263,19 +329,17 @@ GemvPlan plan_gemv_batch(int64_t d_in, int64_t d_out, int B) {
 cudaError_t launch_gemv_batch(const GemvPlan& p, const uint16_t* WT, const uint16_t* X, uint16_t* Y,
                               int B, int d_in, int d_out, float t, void* ws, cudaStream_t stream) {
   BArgs k{};
-  k.WT = WT; k.X = X; k.Y = Y; k.t = t; k.B = B; k.d_in = d_in; k.d_out = d_out;
-  k.S = p.S; k.chunk = p.chunk;
+  k.WT = WT; k.X = X; k.Y = Y; k.t = t; k.B = B; k.d_in = d_in; k.d_out = d_out; k.S = p.S;
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
   k.words_bytes = (uint32_t)words;
-  k.union_bytes = (uint32_t)std::max(2 * words, (size_t)kWarps * kTile * 4);
+  k.union_bytes = (uint32_t)(2 * words);
   k.counters = reinterpret_cast<unsigned*>(ws);
   k.partials = ws != nullptr ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + p.counters)
                              : nullptr;
-  switch (width_for(B)) {
-    case 2: return launch_nb<2>(p, k, stream);
-    case 4: return launch_nb<4>(p, k, stream);
-    default: return launch_nb<8>(p, k, stream);
-  }
+  cudaError_t e = cudaFuncSetAttribute(batch_mma_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(batch_mma_kernel, dim3(p.C, p.S), dim3(kThreads), p.smem, stream, k);
 }
 
 }  // namespace sig
