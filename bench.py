@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--profile-case", default=None,
                     help="for ncu: run only this kernel case eagerly and exit "
                          "(a Llama-2-7B projection name or launch group such as 'q|k|v' or "
-                         "'gate|up' at 50%%, 'topk70b' or 'nm2:4')")
+                         "'gate|up' at 50%%, 'topk70b', 'batchB' (B tokens, 4096->11008) or 'nm2:4')")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     return ap.parse_args()
 
@@ -841,6 +841,18 @@ def profile_case(args):
             launch_group(sig, W[i % copies], x, grp[0].thresholds[HEADLINE_SPARSITY], ys, ws, None)
         info = {"case": case, "launches": args.launches, "copies": copies,
                 "algorithmic_bytes_per_launch": group_bytes(grp, kept_count(grp[0], HEADLINE_SPARSITY))}
+    elif case.startswith("batch"):
+        B = int(case[5:])
+        WT, X, t = workloads.batch_tokens(seed=args.seed + B, B=B)
+        copies = 6
+        Ws = [torch.from_numpy(WT).cuda()]
+        Ws += [Ws[0].clone() for _ in range(copies - 1)]
+        Xd = torch.from_numpy(X).cuda()
+        for i in range(args.launches):
+            sig.sparse_gemv_batch(Ws[i % copies], Xd, t)
+        union = int((np.abs(X.astype(np.float32)) >= t).any(axis=0).sum())
+        info = {"case": case, "launches": args.launches, "copies": copies,
+                "algorithmic_bytes_per_launch": union * 2 * WT.shape[1] + B * 2 * sum(WT.shape)}
     elif case == "nm2:4":
         WT, X = workloads.nm_tokens(args.seed)
         Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()
