@@ -32,6 +32,10 @@ Sources, cited by page title and section:
 * [RaNA] Q6 (batched inference with inconsistent masks) leaves a masked GEMV
          for batch sizes above one, where every token has its own mask, to
          future work; the batched product below is that operation.
+* [TEAL] Limitations: quantised sparse kernels are missing; [QS] A1 on
+         batched inference: quantisation, which shrinks the weight bytes
+         moved per decoding step, is orthogonal to activation sparsity.  The
+         weight-quantised product below is that combination.
 * [NM]   "Motivating Next-Gen Accelerators with Flexible (N:M) Activation
          Sparsity ..." (summary), Methodology: in blocks of size M, N non-zero
          elements are kept; selection criterion ACT = absolute activation size.
@@ -53,6 +57,9 @@ Readings where the pages are silent or disagree (each one is a choice):
 * Rank adapter precision: v = Bx in float64 from the fp16 inputs, rounded once
   to fp16 (the intermediate activation of an fp16 model); the score is
   ``float32(v_i) * float32(v_i)`` as one float32 multiply; ``score >= t``.
+* Weight-quantised product (the pages fix no format): int8 weights q with one
+  float32 scale per output column, ``W_ij = s_j * q_ij``; the activation and
+  its mask stay fp16, and ``y_j = s_j * sum_i q_ij (m_i x_i)``.
 * Outputs: y in float64 (used for the error bound) and rounded once to fp16.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
@@ -69,7 +76,7 @@ __all__ = [
     "masked_matvec", "sparse_linear", "silu", "row_norms", "rana_hidden",
     "rana_scores", "rana_mask", "gated_mlp", "nm_gemm",
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
-    "union_mask", "batched_sparse_linear",
+    "union_mask", "batched_sparse_linear", "q8_sparse_linear",
 ]
 
 
@@ -316,6 +323,31 @@ def batched_sparse_linear(WT, X, masks, cols=None) -> dict:
     y64 = np.stack([o[0] for o in outs]) if outs else np.zeros((0, 0))
     bound = np.stack([o[1] for o in outs]) if outs else np.zeros((0, 0))
     return {"y64": y64, "y16": fp16(y64), "bound": bound, "union": union_mask(masks)}
+
+
+# ---------------------------------------------------------------------------
+# Weight-quantised sparse product ([TEAL] Limitations, [QS] A1)
+# ---------------------------------------------------------------------------
+
+def q8_sparse_linear(QT, scale, x, mask, cols=None) -> dict:
+    """y_j = s_j * sum_i QT[i, j] * (m_i ? x_i : 0) in float64.
+
+    ``QT`` is the int8 weight transposed, (d_in, d_out); ``scale`` the float32
+    scale of each output column, so that W[j, i] = s_j * QT[i, j].  Returns
+    the same fields as :func:`sparse_linear`, with
+    ``bound_j = |s_j| * sum_i |QT[i, j] * m_i x_i|``.
+    """
+    QT = np.asarray(QT, dtype=np.int8)
+    s64 = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    if cols is not None:
+        QT, s64 = QT[:, np.asarray(cols)], s64[np.asarray(cols)]
+    xm = np.where(np.asarray(mask, dtype=bool), np.asarray(x, dtype=np.float64), 0.0)
+    Q64 = QT.astype(np.float64)
+    y64 = (xm @ Q64) * s64
+    bound = (np.abs(xm) @ np.abs(Q64)) * np.abs(s64)
+    idx = compact(mask)
+    return {"mask": np.asarray(mask, dtype=bool), "idx": idx, "nnz": int(idx.size),
+            "y64": y64, "y16": fp16(y64), "bound": bound}
 
 
 # ---------------------------------------------------------------------------

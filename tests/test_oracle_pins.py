@@ -588,3 +588,42 @@ def test_batched_tokens_properties():
     same = oracle.batched_sparse_linear(WT, Xs, ms)["y64"]
     assert np.array_equal(same[0], same[1]) and np.array_equal(same[1], same[2])
     assert np.array_equal(oracle.union_mask(ms), masks[0])
+
+
+# ---------------------------------------------------------------------------
+# Weight-quantised sparse product
+# ---------------------------------------------------------------------------
+
+def test_q8_golden():
+    Q, vals = [], {}
+    for ln in _read_lines("q8_tiny.txt"):
+        key, v = ln.split(":", 1)
+        if key == "Q":
+            Q.append([int(c) for c in v.split()])
+        else:
+            vals[key] = v
+    QT = np.array(Q, np.int8)
+    x = np.array(_floats(vals["x"]), np.float16)
+    m = oracle.threshold_mask(x, float(vals["t"]))
+    assert m.astype(int).tolist() == [int(c) for c in vals["mask"].split()]
+    out = oracle.q8_sparse_linear(QT, np.array(_floats(vals["scale"]), np.float32), x, m)
+    assert out["y64"].tolist() == _floats(vals["y"])
+
+
+def test_q8_is_the_fp16_product_on_exact_dequantised_weights():
+    """With power-of-two scales, s_j * q_ij is exact in fp16, and the
+    quantised product equals the fp16 product on those weights exactly."""
+    rng = np.random.default_rng(41)
+    d_in, d_out = 200, 48
+    QT = rng.integers(-127, 128, (d_in, d_out)).astype(np.int8)
+    scale = (2.0 ** -rng.integers(6, 10, d_out)).astype(np.float32)
+    WT = (QT.astype(np.float64) * scale.astype(np.float64)).astype(np.float16)
+    assert np.array_equal(WT.astype(np.float64), QT.astype(np.float64) * scale.astype(np.float64))
+    x = rng.laplace(0, 1, d_in).astype(np.float16)
+    m = oracle.threshold_mask(x, 0.8)
+    a = oracle.q8_sparse_linear(QT, scale, x, m)
+    b = oracle.sparse_linear(WT, x, m)
+    assert np.array_equal(a["y64"], b["y64"]) and np.array_equal(a["bound"], b["bound"])
+    cols = np.array([0, 7, 47])
+    c = oracle.q8_sparse_linear(QT, scale, x, m, cols=cols)
+    assert np.array_equal(c["y64"], a["y64"][cols])

@@ -36,7 +36,7 @@ __all__ = [
     "LLAMA2_SPARSITIES", "QSPARSE_KEEP_FRACTIONS",
     "draw_weight", "draw_vector", "quantile_threshold", "topk_count",
     "Projection", "projection", "rana_mlp", "nm_tokens", "tiny_gemv", "llama2_7b_layer",
-    "rank_adapter", "batch_tokens",
+    "rank_adapter", "batch_tokens", "q8_projection",
 ]
 
 # Llama-2-7B decode projections at batch 1: (name, d_in, d_out).
@@ -189,6 +189,26 @@ def batch_tokens(seed: int = 0, B: int = 4, d_in: int = 4096, d_out: int = 11008
     WT = draw_weight(rng, d_in, d_out, sigma)
     X = draw_vector(rng, (B, d_in), "laplace")
     return WT, X, quantile_threshold(X, sparsity)
+
+
+def q8_projection(seed: int = 0, d_in: int = 4096, d_out: int = 11008, q_sigma: float = 40.0,
+                  w_sigma: float = 0.02, sparsities=(0.5,)):
+    """An int8 weight as a quantised checkpoint holds it, then x ~ Laplace(0, 1).
+
+    QT (d_in, d_out) int8: N(0, q_sigma^2) rounded to the nearest integer and
+    clipped to [-127, 127]; scale (d_out,) float32: w_sigma / q_sigma times
+    U(0.9, 1.1), so that s_j * q has the spread of the fp16 weights.  Returns
+    (QT, scale, x, {sparsity: t}).
+    """
+    rng = np.random.default_rng(seed)
+    QT = np.empty((d_in, d_out), dtype=np.int8)
+    flat = QT.reshape(-1)
+    for lo in range(0, flat.size, _CHUNK):
+        hi = min(flat.size, lo + _CHUNK)
+        flat[lo:hi] = np.clip(np.rint(rng.normal(0.0, q_sigma, hi - lo)), -127, 127).astype(np.int8)
+    scale = (w_sigma / q_sigma * rng.uniform(0.9, 1.1, d_out)).astype(np.float32)
+    x = draw_vector(rng, d_in, "laplace")
+    return QT, scale, x, {s: quantile_threshold(x, s) for s in sparsities}
 
 
 @dataclass
