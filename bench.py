@@ -16,7 +16,7 @@ no step finds its weights in L2 (580 MB of kept rows per rotation, > 4x L2).
 Steps are replayed CUDA graphs, timed with CUDA events on the launching stream.
 
 The JSON line also carries the sparsity sweep, the top-k (Q-Sparse 70B), RaNA
-gated-MLP, RaNA rank-adapter, per-token-mask batch and N:M GEMM rows, cuBLAS dense baselines at the same shapes, the
+gated-MLP, RaNA rank-adapter, per-token-mask batch, int8-weight and N:M GEMM rows, cuBLAS dense baselines at the same shapes, the
 roofline of the sparse GEMV kernel, the oracle's CPU baseline and the SM
 clocks sampled during the timed region.
 
@@ -415,6 +415,7 @@ def run_ours(args, rank, world, local):
         extras["nm_gemm"] = bench_nm(args, stream, sig, bf16_peak)
         extras["rana_rank_adapter"] = bench_rank_adapter(args, stream, sig, hbm_peak)
         extras["batched_per_token_masks"] = bench_batch(args, stream, sig, hbm_peak)
+        extras["int8_weights"] = bench_q8(args, stream, sig, hbm_peak)
         result["extras"] = extras
         result["cpu_baseline"] = cpu_baseline(groups)
     return result
@@ -653,6 +654,53 @@ def bench_batch(args, stream, sig, hbm_peak):
                          "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
                          "separate_single_token_launches_us": round(us_sep, 2)}
         del Ws, sg, sh
+        torch.cuda.empty_cache()
+    return out
+
+
+def bench_q8(args, stream, sig, hbm_peak):
+    """int8 weights (one scale per column) at the Llama-2-7B shapes, 50 % threshold,
+    against the fp16 sparse GEMV on the same shapes."""
+    import torch
+    out = {"note": "int8 kept rows cost d_out bytes; fp16 rows 2 d_out"}
+    for name, d_in, d_out in (("q", 4096, 4096), ("gate", 4096, 11008), ("down", 11008, 4096)):
+        QT, scale, x, ts = workloads.q8_projection(seed=args.seed + d_in + d_out, d_in=d_in,
+                                                   d_out=d_out)
+        t = ts[0.5]
+        copies = max(2, math.ceil(4 * 126e6 / (d_in * d_out)))
+        Qs = [torch.from_numpy(QT).cuda()]
+        Qs += [Qs[0].clone() for _ in range(copies - 1)]
+        sd = torch.from_numpy(scale).cuda()
+        xd = torch.from_numpy(x).cuda()
+        y = torch.empty(d_out, dtype=torch.float16, device="cuda")
+        ws = torch.zeros(max(256, sig.workspace_bytes(sig.OP_SPARSE_GEMV_Q8, d_in, d_out)),
+                         dtype=torch.uint8, device="cuda")
+
+        def f(c):
+            def g():
+                sig.sparse_gemv_q8(Qs[c], sd, xd, t, y=y, ws=ws, stream=stream)
+            return g
+        sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies * 4)
+        steps = 400
+        us = time_steps(sg, steps, copies, stream) / steps * 1e6
+        nnz = int((np.abs(x.astype(np.float32)) >= t).sum())
+        b = nnz * d_out + 2 * d_in + 2 * d_out
+        # the fp16 sparse GEMV on a weight of the same shape
+        Ws = [torch.empty((d_in, d_out), dtype=torch.float16, device="cuda").normal_(0, 0.02)
+              for _ in range(max(2, math.ceil(4 * 126e6 / (2 * d_in * d_out))))]
+        ws16 = torch.zeros(max(256, sig.workspace_bytes(sig.OP_SPARSE_GEMV, d_in, d_out)),
+                           dtype=torch.uint8, device="cuda")
+
+        def h(c):
+            def g():
+                sig.sparse_gemv(Ws[c], xd, t=t, y=y, ws=ws16, stream=stream)
+            return g
+        sh = StepGraphs([h(c) for c in range(len(Ws))], stream, per_graph=len(Ws) * 4)
+        us16 = time_steps(sh, steps, len(Ws), stream) / steps * 1e6
+        out[f"{name} {d_in}->{d_out}"] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+                                          "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
+                                          "fp16_sparse_us": round(us16, 2)}
+        del Qs, Ws, sg, sh
         torch.cuda.empty_cache()
     return out
 

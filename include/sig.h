@@ -75,7 +75,8 @@ typedef enum {
   SIG_OP_GATED_MLP = 3,    /* gated_mlp_sparse(d_model = d_in, d_ff = d_out) */
   SIG_OP_NM_GEMM = 4,      /* nm_act_gemm(K = d_in, N = d_out, rows)   */
   SIG_OP_RANK_ADAPTER = 5, /* rank_adapter_sparse(d_in, d_out, rows = r) */
-  SIG_OP_SPARSE_GEMV_BATCH = 6 /* sparse_gemv_batch(d_in, d_out, rows = tokens) */
+  SIG_OP_SPARSE_GEMV_BATCH = 6, /* sparse_gemv_batch(d_in, d_out, rows = tokens) */
+  SIG_OP_SPARSE_GEMV_Q8 = 7     /* sparse_gemv_q8(d_in, d_out)              */
 } sig_op;
 
 /* Largest activation length the fused mask prologue accepts. */
@@ -247,6 +248,24 @@ SIG_API int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint1
 SIG_API int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out,
                               const uint16_t* X, int64_t B, float t, uint16_t* Y,
                               void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * Weight-quantised sparse GEMV: y = W (m . x), m_i = |x_i| >= t, with the weight
+ * held as int8 q and one float32 scale per output column, W[j, i] = s_j q[i, j]:
+ *   y_j = fp16( s_j * sum_{i: m_i} q[i, j] x_i )      (float32 accumulation)
+ * The pages leave quantised sparse kernels open (TEAL README, Limitations) and
+ * call quantisation orthogonal to activation sparsity (Q-Sparse rebuttal, A1 on
+ * batched inference); a kept input costs d_out bytes instead of 2 d_out.
+ *   QT [d_in x d_out] int8 (transposed: row i multiplies x_i), 16-byte aligned.
+ *   scale [d_out] float32.  x [d_in] fp16.  y [d_out] fp16 out.
+ *   ws sig_workspace_bytes(SIG_OP_SPARSE_GEMV_Q8, d_in, d_out, 0) bytes
+ *      (0 means none is needed), 256-byte aligned, zeroed once before first use.
+ * d_out % 16 == 0 (whole 16-byte lanes of a row), d_in <= SIG_MAX_D_IN.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
+ */
+SIG_API int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+                           const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                           sig_stream_t stream);
 
 /*
  * RaNA linear-layer rank adapter (RaNA rebuttal, Q5.1: Linear(x) ~ A (m(x) . Bx),

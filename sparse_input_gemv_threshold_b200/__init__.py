@@ -23,13 +23,15 @@ __all__ = [
     "sparsify_topk", "sparsify_nm", "sparse_gemv", "gated_mlp_sparse", "row_norms",
     "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
     "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
-    "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch",
+    "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch", "OP_SPARSE_GEMV_Q8",
+    "sparse_gemv_q8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
 
 OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM, OP_RANK_ADAPTER = 1, 2, 3, 4, 5
 OP_SPARSE_GEMV_BATCH = 6
+OP_SPARSE_GEMV_Q8 = 7
 MAX_BATCH = 8
 MAX_D_IN = 131072
 
@@ -54,6 +56,7 @@ _SIGNATURES = {
     "sig_workspace_bytes_multi": (_sz, [_i32, _p, _i64]),
     "rank_adapter_sparse": (_i32, [_p, _p, _p, _i64, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
     "sparse_gemv_batch": (_i32, [_p, _i64, _i64, _p, _i64, _f32, _p, _p, _sz, _p]),
+    "sparse_gemv_q8": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
 }
 
 
@@ -243,6 +246,24 @@ def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
     _check("gated_mlp_sparse", _lib.gated_mlp_sparse(
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
         _ptr(y), _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def sparse_gemv_q8(QT, scale, x, t: float, y=None, ws=None, stream=None):
+    """y = W (m . x) with int8 weights QT (d_in x d_out) and float32 column scales."""
+    _need(QT, torch.int8, "QT")
+    _need(scale, torch.float32, "scale", QT.device)
+    _need(x, torch.float16, "x", QT.device)
+    d_in, d_out = QT.shape
+    if x.numel() != d_in or scale.numel() != d_out:
+        raise ValueError("shapes: QT (d_in, d_out), scale (d_out), x (d_in)")
+    if y is None:
+        y = torch.empty(d_out, dtype=torch.float16, device=QT.device)
+    if ws is None:
+        ws = workspace(OP_SPARSE_GEMV_Q8, d_in, d_out, device=QT.device, stream=stream)
+    _check("sparse_gemv_q8", _lib.sparse_gemv_q8(
+        _ptr(QT), _ptr(scale), d_in, d_out, _ptr(x), float(t), _ptr(y), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return y
 
 

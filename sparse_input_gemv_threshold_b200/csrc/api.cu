@@ -4,6 +4,7 @@
 // returns at once.
 #include "../../include/sig.h"
 #include "internal.h"
+#include "gemv_q8.h"
 
 #include <cuda_runtime.h>
 
@@ -71,6 +72,9 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
           rows > kGemvMaxBatch)
         return 0;
       return plan_gemv_batch(d_in, d_out, (int)rows).ws_bytes();
+    case SIG_OP_SPARSE_GEMV_Q8:
+      if (check_gemv_shape(d_in, d_out) != SIG_OK || d_out % 16 != 0) return 0;
+      return plan_gemv_q8(d_in, d_out).ws_bytes();
     case SIG_OP_NM_GEMM:
       if (rows < 1 || d_in < 1) return 0;
       return round_up((size_t)rows * (size_t)d_in * 2, 256);   // the masked activation block
@@ -150,6 +154,23 @@ int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out, const uin
   if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
   return cuda_status(launch_gemv_batch(p, WT, X, Y, (int)B, (int)d_in, (int)d_out, t, ws,
                                        (cudaStream_t)stream));
+}
+
+int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+                   const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                   sig_stream_t stream) {
+  if (QT == nullptr || scale == nullptr || x == nullptr || y == nullptr) return SIG_ERR_NULL;
+  const int sh = check_gemv_shape(d_in, d_out);
+  if (sh != SIG_OK) return sh;
+  if (d_out % 16 != 0) return SIG_ERR_SHAPE;
+  if (!aligned16(QT) || !aligned16(x) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return SIG_ERR_ALIGN;
+  const GemvPlan p = plan_gemv_q8(d_in, d_out);
+  if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
+  return cuda_status(launch_gemv_q8(p, QT, scale, x, t, y, (int)d_in, (int)d_out, ws,
+                                    (cudaStream_t)stream));
 }
 
 size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in) {

@@ -140,6 +140,21 @@ def test_multi_validation(lib):
     assert lib.sig_workspace_bytes_multi(0, D, 64) == 0
 
 
+def test_q8_validation(lib):
+    f = lib.sparse_gemv_q8
+    big = 1 << 30
+    assert f(None, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == NULL
+    assert f(FAKE, None, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == NULL
+    assert f(FAKE, FAKE, 64, 24, FAKE, 0.0, FAKE, FAKE, big, None) == SHAPE    # d_out % 16
+    assert f(FAKE, FAKE, 0, 64, FAKE, 0.0, FAKE, FAKE, big, None) == SHAPE
+    assert f(FAKE_ODD, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == ALIGN
+    assert f(FAKE, FAKE + 1, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == ALIGN   # scale alignment
+    need = lib.sig_workspace_bytes(7, 64, 64, 0)
+    assert need > 0
+    assert f(FAKE, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, need - 1, None) == WORKSPACE
+    assert lib.sig_workspace_bytes(7, 64, 24, 0) == 0
+
+
 def test_batch_validation(lib):
     f = lib.sparse_gemv_batch
     big = 1 << 30
