@@ -60,6 +60,14 @@ Readings where the pages are silent or disagree (each one is a choice):
 * Weight-quantised product (the pages fix no format): int8 weights q with one
   float32 scale per output column, ``W_ij = s_j * q_ij``; the activation and
   its mask stay fp16, and ``y_j = s_j * sum_i q_ij (m_i x_i)``.
+* N:M mitigation variants ([NM] Methodology: selection criteria ACT and WT,
+  error mitigation D-/S-/L-PTS and VAR): a per-token shift mu gives
+  ``x' = fp16(float32(x) - mu)`` (the product adds back ``mu * r_j`` with
+  ``r_j = sum_i WT[i, j]``); the WT criterion scores ``float32(|x'_i|) *
+  norm_i`` (one float32 multiply, ``norm_i`` the l2 norm of the weights that
+  multiply input i) in place of ``|x'_i|``; VAR scales a token's kept values
+  by ``gamma = sqrt(sum x'^2 / sum (m x')^2)`` so that the masked activation
+  keeps the token's l2 norm (gamma = 1 when either sum is 0).
 * Outputs: y in float64 (used for the error bound) and rounded once to fp16.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
@@ -77,6 +85,7 @@ __all__ = [
     "rana_scores", "rana_mask", "gated_mlp", "nm_gemm",
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
     "union_mask", "batched_sparse_linear", "q8_sparse_linear",
+    "pts_shift", "wt_scores", "nm_mask_by_score", "var_gamma", "nm_variant", "nm_variant_gemm",
 ]
 
 
@@ -323,6 +332,79 @@ def batched_sparse_linear(WT, X, masks, cols=None) -> dict:
     y64 = np.stack([o[0] for o in outs]) if outs else np.zeros((0, 0))
     bound = np.stack([o[1] for o in outs]) if outs else np.zeros((0, 0))
     return {"y64": y64, "y16": fp16(y64), "bound": bound, "union": union_mask(masks)}
+
+
+# ---------------------------------------------------------------------------
+# N:M selection and error-mitigation variants ([NM] Methodology)
+# ---------------------------------------------------------------------------
+
+def pts_shift(X, shift) -> np.ndarray:
+    """Per-token shift (PTS): x' = fp16(float32(x) - mu_row), one rounding."""
+    X32 = np.asarray(X, dtype=np.float16).astype(np.float32)
+    mu = np.asarray(shift, dtype=np.float32).reshape(-1, 1)
+    return (X32 - mu).astype(np.float16)
+
+
+def wt_scores(Xs, norms) -> np.ndarray:
+    """WT criterion: float32(|x'_i|) * norm_i as one float32 multiply."""
+    a = np.abs(np.asarray(Xs, dtype=np.float16)).astype(np.float32)
+    return (a * np.asarray(norms, dtype=np.float32).reshape(1, -1)).astype(np.float32)
+
+
+def nm_mask_by_score(S, n: int, m: int) -> np.ndarray:
+    """Per row, in each block of m consecutive entries keep the n of largest
+    score; equal scores by lower index, a NaN score below every number."""
+    S = np.asarray(S, dtype=np.float64)
+    rows, d = S.shape
+    out = np.zeros((rows, d), dtype=bool)
+    for r in range(rows):
+        for b0 in range(0, d, m):
+            blk = S[r, b0:b0 + m]
+            key = np.where(np.isnan(blk), -np.inf, blk)
+            nan = np.isnan(blk)
+            # sort by (score desc, NaN last, index asc)
+            order = sorted(range(blk.size), key=lambda j: (nan[j], -key[j], j))
+            out[r, b0 + np.array(order[:n])] = True
+    return out
+
+
+def var_gamma(Xs, mask) -> np.ndarray:
+    """VAR: per row gamma = sqrt(sum x'^2 / sum (m x')^2) in float64 (1 when
+    either sum is 0), the scale that gives the masked row the l2 norm of x'."""
+    X64 = np.asarray(Xs, dtype=np.float16).astype(np.float64)
+    full = (X64 * X64).sum(axis=1)
+    kept = np.where(mask, X64 * X64, 0.0).sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        g = np.sqrt(full / kept)
+    return np.where((full > 0) & (kept > 0), g, 1.0)
+
+
+def nm_variant(X, n: int, m: int, shift=None, norms=None, var: bool = False) -> dict:
+    """The masked activation block of one N:M variant: shift (PTS), score
+    (|x'| for ACT, WT with norms), select n of m, then scale (VAR)."""
+    X = np.asarray(X, dtype=np.float16)
+    Xs = pts_shift(X, shift) if shift is not None else X
+    if norms is None:
+        mask = nm_mask(Xs, n, m)
+    else:
+        mask = nm_mask_by_score(wt_scores(Xs, norms), n, m)
+    gamma = var_gamma(Xs, mask) if var else np.ones(X.shape[0])
+    Xm64 = np.where(mask, Xs.astype(np.float64), 0.0) * gamma.reshape(-1, 1)
+    return {"xs": Xs, "mask": mask, "gamma": gamma, "xm64": Xm64, "xm16": fp16(Xm64)}
+
+
+def nm_variant_gemm(Xm, WT, shift=None, rows=None):
+    """Y = Xm WT + mu r^T (r_j = sum_i WT[i, j], the shift added back), float64.
+    ``Xm`` is the masked (and scaled) activation block.  Returns (Y64, bound)
+    with bound = |Xm| |WT| + |mu| sum_i |WT[i, j]|."""
+    Xm = np.asarray(Xm, dtype=np.float64)
+    W64 = np.asarray(WT).astype(np.float64)
+    mu = np.zeros(Xm.shape[0]) if shift is None else np.asarray(shift, dtype=np.float32).astype(np.float64)
+    if rows is not None:
+        Xm, mu = Xm[np.asarray(rows)], mu[np.asarray(rows)]
+    Y = Xm @ W64 + np.outer(mu, W64.sum(axis=0))
+    bound = np.abs(Xm) @ np.abs(W64) + np.outer(np.abs(mu), np.abs(W64).sum(axis=0))
+    return Y, bound
 
 
 # ---------------------------------------------------------------------------

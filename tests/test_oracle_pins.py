@@ -627,3 +627,65 @@ def test_q8_is_the_fp16_product_on_exact_dequantised_weights():
     cols = np.array([0, 7, 47])
     c = oracle.q8_sparse_linear(QT, scale, x, m, cols=cols)
     assert np.array_equal(c["y64"], a["y64"][cols])
+
+
+# ---------------------------------------------------------------------------
+# N:M selection and mitigation variants
+# ---------------------------------------------------------------------------
+
+def _nmv_fixture():
+    f = {}
+    for ln in _read_lines("nm_variants_tiny.txt"):
+        k, v = ln.split(":", 1)
+        f[k] = [part.strip() for part in v.split("|")]
+    return f
+
+
+def test_nm_variants_golden():
+    f = _nmv_fixture()
+    x = np.array([_floats(f["act"][0])], np.float16)
+    assert oracle.nm_variant(x, 2, 4)["mask"].astype(int)[0].tolist() == [int(v) for v in f["act"][1].split()]
+    norms = np.array(_floats(f["wt"][1]), np.float32)
+    out = oracle.nm_variant(x, 2, 4, norms=norms)
+    assert out["mask"].astype(int)[0].tolist() == [int(v) for v in f["wt"][2].split()]
+    xp = np.array([_floats(f["pts"][0])], np.float16)
+    mu = np.array([float(f["pts"][1])], np.float32)
+    out = oracle.nm_variant(xp, 2, 4, shift=mu, var=True)
+    assert out["xs"].astype(np.float64)[0].tolist() == _floats(f["pts"][2])
+    assert out["mask"].astype(int)[0].tolist() == [int(v) for v in f["pts"][3].split()]
+    full, kept = _floats(f["var"][0])
+    assert out["gamma"][0] == pytest.approx(math.sqrt(full / kept), rel=1e-15)
+    WT = np.array([[1, 0], [0, 1], [1, 1], [2, -1]], np.float16)
+    all_kept = oracle.nm_variant(xp, 4, 4, shift=mu)
+    Y, _ = oracle.nm_variant_gemm(all_kept["xm64"], WT, shift=mu)
+    assert Y[0].tolist() == _floats(f["gemm"][0])
+    assert Y[0].tolist() == (xp.astype(np.float64) @ WT.astype(np.float64))[0].tolist()
+
+
+def test_nm_variants_reduce_to_plain_nm():
+    rng = np.random.default_rng(51)
+    X = rng.choice([0.0, 0.5, -0.5, 1.0, -2.0, 3.0], size=(6, 64)).astype(np.float16)
+    X[0, :5] = np.nan
+    for n, m in ((2, 4), (1, 4), (3, 8), (8, 16), (16, 32)):
+        plain = oracle.nm_mask(X, n, m)
+        out = oracle.nm_variant(X, n, m)
+        assert np.array_equal(out["mask"], plain)
+        assert np.array_equal(out["xm16"].view(np.uint16), np.where(plain, X, np.float16(0)).view(np.uint16))
+        # scoring by |x| itself, or WT with equal power-of-two norms, is ACT
+        by_score = oracle.nm_mask_by_score(np.abs(X.astype(np.float32)), n, m)
+        assert np.array_equal(by_score, plain)
+        wt = oracle.nm_variant(X, n, m, norms=np.full(64, 2.0, np.float32))
+        assert np.array_equal(wt["mask"], plain)
+        # a zero shift changes nothing
+        z = oracle.nm_variant(X, n, m, shift=np.zeros(6, np.float32))
+        assert np.array_equal(z["mask"], plain)
+
+
+def test_var_restores_the_row_norm():
+    rng = np.random.default_rng(52)
+    X = rng.laplace(0, 1, (5, 128)).astype(np.float16)
+    out = oracle.nm_variant(X, 2, 4, shift=rng.normal(0, 0.1, 5).astype(np.float32), var=True)
+    xs = out["xs"].astype(np.float64)
+    assert np.allclose(np.linalg.norm(out["xm64"], axis=1), np.linalg.norm(xs, axis=1), rtol=1e-13)
+    zero = oracle.var_gamma(np.zeros((1, 8), np.float16), np.ones((1, 8), bool))
+    assert zero.tolist() == [1.0]
