@@ -751,6 +751,23 @@ def bench_nm(args, stream, sig, bf16_peak):
     sec = time_steps(sg, steps, copies, stream)
     us = sec / steps * 1e6
     out["cublas_dense"] = {"us": round(us, 2), "TFLOPs": round(flops_dense / (us * 1e-6) / 1e12, 1)}
+    # the mitigation variants on 2:4: per-token shift (mean of the token), WT
+    # scores with the weight's row norms, VAR; the shift added back in the GEMM
+    shifts = [x.float().mean(dim=1).contiguous() for x in Xs[:2]]
+    norms = sig.row_norms(Ws[0])
+    csum = sig.col_sums_of(Ws[0])
+    for label, kw in (("2:4 WT", {"norms": norms}), ("2:4 PTS+VAR", {"var": True}),
+                      ("2:4 WT+PTS+VAR", {"norms": norms, "var": True})):
+        use_shift = "PTS" in label
+
+        def fv(c, kw=kw, use_shift=use_shift):
+            def g():
+                sig.nm_act_gemm_ex(Xs[c], Ws[c], 2, 4, shift=shifts[c % 2] if use_shift else None,
+                                   col_sums=csum if use_shift else None, Y=Y, ws=ws, stream=stream, **kw)
+            return g
+        sv = StepGraphs([fv(c) for c in range(copies)], stream, per_graph=copies)
+        usv = time_steps(sv, steps, copies, stream) / steps * 1e6
+        out[label] = {"us": round(usv, 2), "TFLOPs_executed": round(flops_dense / (usv * 1e-6) / 1e12, 1)}
     out["tensor_peak_tflops"] = bf16_peak
     return out
 

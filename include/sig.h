@@ -290,6 +290,54 @@ SIG_API int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uin
                                 void* ws, size_t ws_bytes, sig_stream_t stream);
 
 /*
+ * N:M activation mask with the selection and error-mitigation variants of
+ * "Motivating Next-Gen Accelerators with Flexible (N:M) Activation Sparsity
+ * ..." (summary, Methodology: criteria ACT and WT, mitigation PTS and VAR),
+ * per row r of X:
+ *   x' = fp16(float32(x) - shift[r])            (PTS; shift NULL: x' = x)
+ *   score_i = |x'_i|                            (ACT, norms NULL)
+ *           = float32(|x'_i|) * norms[i]        (WT: one float32 multiply;
+ *                                                norms = ||W_i||, see sig_row_norms)
+ *   m: in each block of m, the n of largest score (lower index first among
+ *      equals, NaN last), as sparsify_nm
+ *   X_masked = fp16(gamma_r * m . x')           (VAR: gamma_r = sqrt(sum x'^2 /
+ *                                                sum (m x')^2), float32, 1 when
+ *                                                either sum is 0; var = 0: gamma 1)
+ *   X [rows x d] fp16, row-major.  shift [rows] float32, nullable.
+ *   norms [d] float32, nullable.  X_masked [rows x d] fp16 out (required).
+ *   mask_bits [rows x ceil(d/32)] uint32 out, nullable.  gamma_out [rows] float32 out, nullable.
+ * 1 <= n <= m, m in {1, 2, 4, 8, 16, 32}, d % m == 0, d % 8 == 0.
+ * Errors: SIG_ERR_ARG (n, m), SIG_ERR_SHAPE, SIG_ERR_NULL, SIG_ERR_ALIGN, SIG_ERR_CUDA.
+ */
+SIG_API int sparsify_nm_ex(const uint16_t* X, int64_t rows, int64_t d, int n, int m,
+                           const float* shift, const float* norms, int var,
+                           uint16_t* X_masked, uint32_t* mask_bits, float* gamma_out,
+                           sig_stream_t stream);
+
+/*
+ * N:M activation GEMM with the variants of sparsify_nm_ex:
+ *   Y = X_masked WT + shift col_sums^T       (the shift added back: col_sums[j] =
+ *                                             sum_i WT[i, j], see sig_col_sums)
+ * on the tensor cores as nm_act_gemm.  shift NULL: no added term (col_sums may
+ * be NULL); otherwise col_sums [N] float32 is required.  Shapes, workspace
+ * (sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows)) and errors as nm_act_gemm.
+ */
+SIG_API int nm_act_gemm_ex(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT,
+                           int64_t N, int n, int m, const float* shift, const float* norms,
+                           int var, const float* col_sums, uint16_t* Y, void* ws,
+                           size_t ws_bytes, sig_stream_t stream);
+
+/*
+ * Column sums of a row-major fp16 matrix, accumulated in float64 and rounded
+ * once to float32: for WT, r_j = sum_i W[j, i], the vector a per-token shift
+ * mu brings back as mu * r (x W = (x - mu) W + mu r).
+ *   WT [rows x cols] fp16.  sums [cols] float32 out.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE.
+ */
+SIG_API int sig_col_sums(const uint16_t* WT, int64_t rows, int64_t cols, float* sums,
+                         sig_stream_t stream);
+
+/*
  * l2 norm of every row of a row-major fp16 matrix, accumulated in float64 and
  * rounded once to float32.  For WdT it yields the ||W^down_i|| of RaNA Eqn. 12.
  *   WT [rows x cols] fp16 (16-byte aligned, cols % 8 == 0).  norms [rows] float32 out.

@@ -24,7 +24,7 @@ __all__ = [
     "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
     "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
     "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch", "OP_SPARSE_GEMV_Q8",
-    "sparse_gemv_q8",
+    "sparse_gemv_q8", "sparsify_nm_ex", "nm_act_gemm_ex", "col_sums",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -57,6 +57,10 @@ _SIGNATURES = {
     "rank_adapter_sparse": (_i32, [_p, _p, _p, _i64, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
     "sparse_gemv_batch": (_i32, [_p, _i64, _i64, _p, _i64, _f32, _p, _p, _sz, _p]),
     "sparse_gemv_q8": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
+    "sparsify_nm_ex": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _p]),
+    "nm_act_gemm_ex": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _sz,
+                              _p]),
+    "sig_col_sums": (_i32, [_p, _i64, _i64, _p, _p]),
 }
 
 
@@ -247,6 +251,61 @@ def gated_mlp_sparse(x, WgT, WuT, WdT, down_norms, t: float, y=None, h_out=None,
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), _ptr(down_norms), d_model, d_ff, float(t),
         _ptr(y), _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
     return y
+
+
+def sparsify_nm_ex(X, n: int, m: int, shift=None, norms=None, var: bool = False,
+                   X_masked=None, want_bits=True, want_gamma=False, stream=None):
+    """N:M mask with the per-token shift (PTS), the weight-aware score (WT:
+    norms = ||W_i||) and the variance correction (VAR).  Returns
+    (X_masked, mask_bits or None, gamma or None)."""
+    _need(X, torch.float16, "X")
+    rows, d = X.shape
+    for name, v, size in (("shift", shift, rows), ("norms", norms, d)):
+        if v is not None:
+            _need(v, torch.float32, name, X.device)
+            if v.numel() != size:
+                raise ValueError(f"{name} must have {size} entries")
+    if X_masked is None:
+        X_masked = torch.empty_like(X)
+    bits = (torch.empty((rows, (d + 31) // 32), dtype=torch.int32, device=X.device)
+            if want_bits else None)
+    gamma = torch.empty(rows, dtype=torch.float32, device=X.device) if want_gamma else None
+    _check("sparsify_nm_ex", _lib.sparsify_nm_ex(
+        _ptr(X), rows, d, n, m, _ptr(shift), _ptr(norms), int(bool(var)), _ptr(X_masked),
+        _ptr(bits), _ptr(gamma), _stream(stream)))
+    return X_masked, bits, gamma
+
+
+def nm_act_gemm_ex(X, WT, n: int, m: int, shift=None, norms=None, var: bool = False,
+                   col_sums=None, Y=None, ws=None, stream=None):
+    """Y = X_masked WT + shift col_sums^T on the tensor cores (see sparsify_nm_ex)."""
+    _need(X, torch.float16, "X")
+    _need(WT, torch.float16, "WT", X.device)
+    rows, K = X.shape
+    N = WT.shape[1]
+    if shift is not None and col_sums is None:
+        col_sums = col_sums_of(WT, stream=stream)
+    if Y is None:
+        Y = torch.empty((rows, N), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(OP_NM_GEMM, K, N, rows, device=X.device, stream=stream)
+    _check("nm_act_gemm_ex", _lib.nm_act_gemm_ex(
+        _ptr(X), rows, K, _ptr(WT), N, n, m, _ptr(shift), _ptr(norms), int(bool(var)),
+        _ptr(col_sums), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
+def col_sums_of(WT, sums=None, stream=None):
+    """r_j = sum_i WT[i, j] (float64 accumulation, float32 out)."""
+    _need(WT, torch.float16, "WT")
+    rows, cols = WT.shape
+    if sums is None:
+        sums = torch.empty(cols, dtype=torch.float32, device=WT.device)
+    _check("sig_col_sums", _lib.sig_col_sums(_ptr(WT), rows, cols, _ptr(sums), _stream(stream)))
+    return sums
+
+
+col_sums = col_sums_of
 
 
 def sparse_gemv_q8(QT, scale, x, t: float, y=None, ws=None, stream=None):

@@ -5,6 +5,7 @@
 #include "../../include/sig.h"
 #include "internal.h"
 #include "gemv_q8.h"
+#include "nm_ex.h"
 
 #include <cuda_runtime.h>
 
@@ -270,6 +271,47 @@ int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uint16_t* A
   out.x = v; out.t = t; out.d_in = (int)r; out.mask_out = mask_out;
   out.ws = base + g.off_out;
   return cuda_status(launch_gemv(MASK_SQUARE, EPI_STORE, g.out, out, (cudaStream_t)stream));
+}
+
+int sparsify_nm_ex(const uint16_t* X, int64_t rows, int64_t d, int n, int m, const float* shift,
+                   const float* norms, int var, uint16_t* X_masked, uint32_t* mask_bits,
+                   float* gamma_out, sig_stream_t stream) {
+  if (!nm_pattern_ok(n, m)) return SIG_ERR_ARG;
+  if (rows < 0 || d < 1 || d % m != 0 || d > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
+  if (rows == 0) return SIG_OK;
+  if (X == nullptr || X_masked == nullptr) return SIG_ERR_NULL;
+  if (d % 8 != 0 || !aligned16(X) || !aligned16(X_masked)) return SIG_ERR_ALIGN;
+  return cuda_status(launch_nm_ex(X, rows, (int)d, n, m, shift, norms, var != 0, X_masked,
+                                  mask_bits, gamma_out, (cudaStream_t)stream));
+}
+
+int nm_act_gemm_ex(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT, int64_t N,
+                   int n, int m, const float* shift, const float* norms, int var,
+                   const float* col_sums, uint16_t* Y, void* ws, size_t ws_bytes,
+                   sig_stream_t stream) {
+  if (X == nullptr || WT == nullptr || Y == nullptr) return SIG_ERR_NULL;
+  if (shift != nullptr && col_sums == nullptr) return SIG_ERR_NULL;
+  if (!nm_pattern_ok(n, m)) return SIG_ERR_ARG;
+  if (rows < 128 || rows % 128 != 0 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0 ||
+      K % m != 0 || rows > (1 << 24) || K > (1 << 20) || N > (1 << 20))
+    return SIG_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(WT) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  const size_t need = sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows);
+  if (ws == nullptr || ws_bytes < need) return SIG_ERR_WORKSPACE;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  uint16_t* Xm = reinterpret_cast<uint16_t*>(ws);
+  cudaError_t e = launch_nm_ex(X, rows, (int)K, n, m, shift, norms, var != 0, Xm, nullptr, nullptr,
+                               (cudaStream_t)stream);
+  if (e != cudaSuccess) return SIG_ERR_CUDA;
+  return cuda_status(launch_gemm_f16_shift(Xm, WT, Y, (int)rows, (int)N, (int)K, shift, col_sums,
+                                           (cudaStream_t)stream));
+}
+
+int sig_col_sums(const uint16_t* WT, int64_t rows, int64_t cols, float* sums,
+                 sig_stream_t stream) {
+  if (WT == nullptr || sums == nullptr) return SIG_ERR_NULL;
+  if (rows < 1 || cols < 1 || cols > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
+  return cuda_status(launch_col_sums(WT, rows, (int)cols, sums, (cudaStream_t)stream));
 }
 
 int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float* norms,

@@ -11,6 +11,7 @@
 //  - row norms (||W^down_i|| of RaNA Eqn. 12), float64 accumulation.
 #include "common.cuh"
 #include "internal.h"
+#include "nm_ex.h"
 #include "nm_select.cuh"
 
 #include <cooperative_groups.h>
@@ -482,6 +483,150 @@ nm_vec_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, uint16
   }
 }
 
+// N:M variants, one warp per row ("Motivating Next-Gen Accelerators with
+// Flexible (N:M) Activation Sparsity ...", Methodology: selection criteria
+// ACT and WT, error mitigation PTS and VAR).  For every 32-entry word of the
+// row the lane shifts the entries (x' = fp16(float32(x) - mu); without a
+// shift x' is x, bit for bit), ranks each block of M by |x'| (ACT) or by float32(|x'|) * norm_i
+// (WT) with lower indices first among equals and NaN last, and keeps n.
+// With VAR the warp sums x'^2 and kept x'^2 over the row (float32, fixed
+// order), gamma = sqrt(full / kept) (1 when either is 0), and a second pass
+// writes fp16(gamma * x') for the kept entries.
+template <int M>
+__device__ __forceinline__ uint32_t nm_ex_word(const uint16_t* src, int cnt, bool shifted, float mu,
+                                               const float* norms, int e0, int n,
+                                               uint32_t (&xs)[16]) {
+  uint4 q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    q[i] = i * 8 < cnt ? __ldg(reinterpret_cast<const uint4*>(src) + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (shifted) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        const __half2 h = __floats2half2_rn(__fsub_rn(f.x, mu), __fsub_rn(f.y, mu));
+        xs[i * 4 + k] = *reinterpret_cast<const uint32_t*>(&h);
+      } else {
+        xs[i * 4 + k] = w[k];   // no shift: the input bits as they are
+      }
+    }
+  }
+  uint32_t bits = 0;
+#pragma unroll
+  for (int b0 = 0; b0 < 32; b0 += M) {
+    if (b0 < cnt) {
+      uint64_t comp[M];
+#pragma unroll
+      for (int j = 0; j < M; ++j) {
+        const int e = b0 + j;
+        const uint16_t h = (uint16_t)(xs[e >> 1] >> (16 * (e & 1)));
+        uint64_t key;
+        if (norms == nullptr) {
+          key = mag_key(h);
+        } else {
+          const float sc = __fmul_rn(fabsf(h2f(h)), __ldg(norms + e0 + e));
+          key = isnan(sc) ? 0ull : (uint64_t)__float_as_uint(sc) + 1ull;
+        }
+        comp[j] = (key << 5) | (uint64_t)(31 - j);
+      }
+      bits |= select_top_n<M>(comp, n) << b0;
+    }
+  }
+  return bits;
+}
+
+template <int M>
+__global__ void __launch_bounds__(256)
+nm_ex_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, const float* shift,
+             const float* norms, int var, uint16_t* X_masked, uint32_t* mask_bits,
+             float* gamma_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  pdl_trigger();
+  pdl_wait();
+  if (row >= rows) return;                      // uniform across the warp
+  const int wpr = (d + 31) >> 5;
+  const float mu = shift != nullptr ? __ldg(shift + row) : 0.f;
+  const uint16_t* xrow = X + row * (int64_t)d;
+  uint16_t* orow = X_masked + row * (int64_t)d;
+  float full = 0.f, kept = 0.f;
+  for (int w = lane; w < wpr; w += 32) {
+    const int e0 = w * 32, cnt = min(32, d - e0);
+    uint32_t xs[16];
+    const uint32_t bits = nm_ex_word<M>(xrow + e0, cnt, shift != nullptr, mu, norms, e0, n, xs);
+    if (mask_bits != nullptr) mask_bits[row * wpr + w] = bits;
+    if (var) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float v = h2f((uint16_t)(xs[e >> 1] >> (16 * (e & 1))));
+        const float v2 = e < cnt ? v * v : 0.f;
+        full += v2;
+        kept += ((bits >> e) & 1u) ? v2 : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (i * 8 < cnt) {
+          uint32_t p[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = i * 8 + 2 * k;
+            const uint32_t lo = ((bits >> e) & 1u) ? (xs[i * 4 + k] & 0xffffu) : 0u;
+            const uint32_t hi = ((bits >> (e + 1)) & 1u) ? (xs[i * 4 + k] & 0xffff0000u) : 0u;
+            p[k] = lo | hi;
+          }
+          reinterpret_cast<uint4*>(orow + e0)[i] = make_uint4(p[0], p[1], p[2], p[3]);
+        }
+    }
+  }
+  if (!var) {
+    if (gamma_out != nullptr && lane == 0) gamma_out[row] = 1.f;
+    return;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    full += __shfl_xor_sync(kFull, full, o);
+    kept += __shfl_xor_sync(kFull, kept, o);
+  }
+  const float gamma = (full > 0.f && kept > 0.f) ? __fsqrt_rn(__fdiv_rn(full, kept)) : 1.f;
+  if (gamma_out != nullptr && lane == 0) gamma_out[row] = gamma;
+  for (int w = lane; w < wpr; w += 32) {
+    const int e0 = w * 32, cnt = min(32, d - e0);
+    uint32_t xs[16];
+    const uint32_t bits = nm_ex_word<M>(xrow + e0, cnt, shift != nullptr, mu, norms, e0, n, xs);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i * 8 < cnt) {
+        uint32_t p[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = i * 8 + 2 * k;
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xs[i * 4 + k]));
+          const float a = ((bits >> e) & 1u) ? __fmul_rn(gamma, f.x) : 0.f;
+          const float b = ((bits >> (e + 1)) & 1u) ? __fmul_rn(gamma, f.y) : 0.f;
+          const __half2 h = __floats2half2_rn(a, b);
+          p[k] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        reinterpret_cast<uint4*>(orow + e0)[i] = make_uint4(p[0], p[1], p[2], p[3]);
+      }
+  }
+}
+
+// One thread per column: sum over the rows in float64, one rounding to float32.
+__global__ void __launch_bounds__(256)
+col_sums_kernel(const uint16_t* __restrict__ WT, int64_t rows, int cols, float* sums) {
+  pdl_trigger();
+  pdl_wait();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= cols) return;
+  double s = 0.0;
+  for (int64_t i = 0; i < rows; ++i) s += (double)h2f(WT[i * cols + j]);
+  sums[j] = __double2float_rn(s);
+}
+
 // One warp per row: sum of squares in float64, sqrt, one rounding to float32.
 __global__ void __launch_bounds__(256)
 row_norms_kernel(const uint16_t* __restrict__ WT, int64_t rows, int cols, float* norms) {
@@ -571,6 +716,30 @@ cudaError_t launch_nm_mask(const uint16_t* X, int64_t rows, int d, int n, int m,
     default: return cudaErrorInvalidValue;
   }
   return e;
+}
+
+cudaError_t launch_nm_ex(const uint16_t* X, int64_t rows, int d, int n, int m, const float* shift,
+                         const float* norms, bool var, uint16_t* X_masked, uint32_t* mask_bits,
+                         float* gamma_out, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  const int v = var ? 1 : 0;
+  switch (m) {
+    case 1: return launch_pdl(nm_ex_kernel<1>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+    case 2: return launch_pdl(nm_ex_kernel<2>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+    case 4: return launch_pdl(nm_ex_kernel<4>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+    case 8: return launch_pdl(nm_ex_kernel<8>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+    case 16: return launch_pdl(nm_ex_kernel<16>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+    case 32: return launch_pdl(nm_ex_kernel<32>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_col_sums(const uint16_t* WT, int64_t rows, int cols, float* sums,
+                            cudaStream_t stream) {
+  if (cols == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((cols + 255) / 256);
+  return launch_pdl(col_sums_kernel, dim3(blocks), dim3(256), 0, stream, WT, rows, cols, sums);
 }
 
 cudaError_t launch_row_norms(const uint16_t* WT, int64_t rows, int cols, float* norms,

@@ -17,6 +17,7 @@
 // land (again with a limit), frees its tensor memory and returns.
 #include "common.cuh"
 #include "internal.h"
+#include "nm_ex.h"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -121,7 +122,8 @@ struct __align__(1024) GemmSmem {
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                uint16_t* __restrict__ Y, int M, int N, int K) {
+                uint16_t* __restrict__ Y, int M, int N, int K, const float* __restrict__ shift,
+                const float* __restrict__ colsum) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the dynamic window starts 1024-aligned only by request; align by hand
   GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
@@ -226,6 +228,7 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   if (have_acc) {
     const int row = m0 + warp * 32 + lane;
     uint16_t* yrow = Y + (size_t)row * N + n0;
+    const float mu = shift != nullptr ? __ldg(shift + row) : 0.f;   // the per-token shift added back
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t r[32];
@@ -245,7 +248,12 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       uint32_t p[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const __half2 h = __floats2half2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+        float v0 = __uint_as_float(r[2 * q]), v1 = __uint_as_float(r[2 * q + 1]);
+        if (shift != nullptr) {
+          v0 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q), v0);
+          v1 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q + 1), v1);
+        }
+        const __half2 h = __floats2half2_rn(v0, v1);
         p[q] = *reinterpret_cast<const uint32_t*>(&h);
       }
       uint4* dst = reinterpret_cast<uint4*>(yrow + c);
@@ -293,26 +301,33 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
 
 template <int BN>
 cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, uint16_t* Y, int M, int N,
-                      int K, cudaStream_t stream) {
+                      int K, const float* shift, const float* colsum, cudaStream_t stream) {
   const size_t smem = sizeof(GemmSmem<BN>) + 1024;
   auto fn = gemm_f16_kernel<BN>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(N / BN, M / kBM);
-  fn<<<grid, kThreads, smem, stream>>>(ma, mb, Y, M, N, K);
+  fn<<<grid, kThreads, smem, stream>>>(ma, mb, Y, M, N, K, shift, colsum);
   return cudaPeekAtLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
-                            int K, cudaStream_t stream) {
+cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
+                                  int K, const float* shift, const float* colsum,
+                                  cudaStream_t stream) {
   if (M % kBM != 0 || K % kBK != 0 || N % 128 != 0) return cudaErrorInvalidValue;
+  if (shift != nullptr && colsum == nullptr) return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kBK)) return cudaErrorInvalidValue;
-  if (N % 256 == 0) return launch_bn<256>(ma, mb, Y, M, N, K, stream);
-  return launch_bn<128>(ma, mb, Y, M, N, K, stream);
+  if (N % 256 == 0) return launch_bn<256>(ma, mb, Y, M, N, K, shift, colsum, stream);
+  return launch_bn<128>(ma, mb, Y, M, N, K, shift, colsum, stream);
+}
+
+cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
+                            int K, cudaStream_t stream) {
+  return launch_gemm_f16_shift(A, WT, Y, M, N, K, nullptr, nullptr, stream);
 }
 
 cudaError_t read_device_error(unsigned* out, cudaStream_t stream) {

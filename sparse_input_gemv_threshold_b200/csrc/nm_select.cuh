@@ -12,17 +12,19 @@
 namespace sig {
 
 // One bitonic stage (K = run length, J = partner distance) and the ones after
-// it; template recursion keeps every index a compile-time constant.
-template <int M, int K, int J>
-__device__ __forceinline__ void bitonic_stage(uint32_t (&s)[M]) {
+// it; template recursion keeps every index a compile-time constant.  T is an
+// unsigned composite type (uint32_t or uint64_t).
+template <int M, int K, int J, typename T>
+__device__ __forceinline__ void bitonic_stage(T (&s)[M]) {
 #pragma unroll
   for (int i = 0; i < M; ++i) {
     const int l = i ^ J;
     if (l > i) {
-      const uint32_t a = s[i], b = s[l];
+      const T a = s[i], b = s[l];
+      const T hi = a > b ? a : b, lo = a > b ? b : a;
       const bool desc = (i & K) == 0;      // the final merge leaves s descending
-      s[i] = desc ? max(a, b) : min(a, b);
-      s[l] = desc ? min(a, b) : max(a, b);
+      s[i] = desc ? hi : lo;
+      s[l] = desc ? lo : hi;
     }
   }
   if constexpr (J > 1) bitonic_stage<M, K, J / 2>(s);
@@ -33,8 +35,8 @@ __device__ __forceinline__ void bitonic_stage(uint32_t (&s)[M]) {
 // M <= 8: count, for each entry, the entries ranked above it.  M >= 16: sort a
 // copy descending with a bitonic network; the n-th largest is the minimum of
 // the first n, and an entry is kept when it is at least that.
-template <int M>
-__device__ __forceinline__ uint32_t select_top_n(const uint32_t (&c)[M], int n) {
+template <int M, typename T>
+__device__ __forceinline__ uint32_t select_top_n(const T (&c)[M], int n) {
   uint32_t bits = 0;
   if constexpr (M <= 8) {
 #pragma unroll
@@ -45,13 +47,13 @@ __device__ __forceinline__ uint32_t select_top_n(const uint32_t (&c)[M], int n) 
       bits |= (rank < n ? 1u : 0u) << j;
     }
   } else {
-    uint32_t s[M];
+    T s[M];
 #pragma unroll
     for (int j = 0; j < M; ++j) s[j] = c[j];
     bitonic_stage<M, 2, 1>(s);
-    uint32_t thr = 0xffffffffu;
+    T thr = ~T(0);
 #pragma unroll
-    for (int j = 0; j < M; ++j) thr = min(thr, j < n ? s[j] : 0xffffffffu);
+    for (int j = 0; j < M; ++j) thr = (j < n && s[j] < thr) ? s[j] : thr;
 #pragma unroll
     for (int j = 0; j < M; ++j) bits |= (c[j] >= thr ? 1u : 0u) << j;
   }
