@@ -304,7 +304,7 @@ SIG_API int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uin
  *                                                sum (m x')^2), float32, 1 when
  *                                                either sum is 0; var = 0: gamma 1)
  *   X [rows x d] fp16, row-major.  shift [rows] float32, nullable.
- *   norms [d] float32, nullable.  X_masked [rows x d] fp16 out (required).
+ *   norms [d] float32, 16-byte aligned, nullable.  X_masked [rows x d] fp16 out (required).
  *   mask_bits [rows x ceil(d/32)] uint32 out, nullable.  gamma_out [rows] float32 out, nullable.
  * 1 <= n <= m, m in {1, 2, 4, 8, 16, 32}, d % m == 0, d % 8 == 0.
  * Errors: SIG_ERR_ARG (n, m), SIG_ERR_SHAPE, SIG_ERR_NULL, SIG_ERR_ALIGN, SIG_ERR_CUDA.

@@ -280,7 +280,8 @@ int sparsify_nm_ex(const uint16_t* X, int64_t rows, int64_t d, int n, int m, con
   if (rows < 0 || d < 1 || d % m != 0 || d > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
   if (rows == 0) return SIG_OK;
   if (X == nullptr || X_masked == nullptr) return SIG_ERR_NULL;
-  if (d % 8 != 0 || !aligned16(X) || !aligned16(X_masked)) return SIG_ERR_ALIGN;
+  if (d % 8 != 0 || !aligned16(X) || !aligned16(X_masked) || (norms != nullptr && !aligned16(norms)))
+    return SIG_ERR_ALIGN;
   return cuda_status(launch_nm_ex(X, rows, (int)d, n, m, shift, norms, var != 0, X_masked,
                                   mask_bits, gamma_out, (cudaStream_t)stream));
 }
@@ -295,7 +296,8 @@ int nm_act_gemm_ex(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* W
   if (rows < 128 || rows % 128 != 0 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0 ||
       K % m != 0 || rows > (1 << 24) || K > (1 << 20) || N > (1 << 20))
     return SIG_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(WT) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  if (!aligned16(X) || !aligned16(WT) || !aligned16(Y) || (norms != nullptr && !aligned16(norms)))
+    return SIG_ERR_ALIGN;
   const size_t need = sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows);
   if (ws == nullptr || ws_bytes < need) return SIG_ERR_WORKSPACE;
   if (!aligned256(ws)) return SIG_ERR_ALIGN;

@@ -15,6 +15,7 @@
 #include "nm_select.cuh"
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 namespace sig {
 
@@ -492,7 +493,7 @@ nm_vec_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, uint16
 // With VAR the warp sums x'^2 and kept x'^2 over the row (float32, fixed
 // order), gamma = sqrt(full / kept) (1 when either is 0), and a second pass
 // writes fp16(gamma * x') for the kept entries.
-template <int M>
+template <int M, bool WT>
 __device__ __forceinline__ uint32_t nm_ex_word(const uint16_t* src, int cnt, bool shifted, float mu,
                                                const float* norms, int e0, int n,
                                                uint32_t (&xs)[16]) {
@@ -514,23 +515,33 @@ __device__ __forceinline__ uint32_t nm_ex_word(const uint16_t* src, int cnt, boo
       }
     }
   }
+  float nv[WT ? 32 : 1];
+  if constexpr (WT) {   // the word's 32 norms as eight 16-byte loads
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 f = i * 4 < cnt ? __ldg(reinterpret_cast<const float4*>(norms + e0) + i)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      nv[4 * i] = f.x; nv[4 * i + 1] = f.y; nv[4 * i + 2] = f.z; nv[4 * i + 3] = f.w;
+    }
+  }
   uint32_t bits = 0;
 #pragma unroll
   for (int b0 = 0; b0 < 32; b0 += M) {
     if (b0 < cnt) {
-      uint64_t comp[M];
+      using T = typename std::conditional<WT, uint64_t, uint32_t>::type;
+      T comp[M];
 #pragma unroll
       for (int j = 0; j < M; ++j) {
         const int e = b0 + j;
         const uint16_t h = (uint16_t)(xs[e >> 1] >> (16 * (e & 1)));
-        uint64_t key;
-        if (norms == nullptr) {
-          key = mag_key(h);
+        T key;
+        if constexpr (WT) {
+          const float sc = __fmul_rn(fabsf(h2f(h)), nv[e]);
+          key = isnan(sc) ? T(0) : (T)__float_as_uint(sc) + T(1);
         } else {
-          const float sc = __fmul_rn(fabsf(h2f(h)), __ldg(norms + e0 + e));
-          key = isnan(sc) ? 0ull : (uint64_t)__float_as_uint(sc) + 1ull;
+          key = (T)mag_key(h);
         }
-        comp[j] = (key << 5) | (uint64_t)(31 - j);
+        comp[j] = (key << 5) | (T)(31 - j);
       }
       bits |= select_top_n<M>(comp, n) << b0;
     }
@@ -538,51 +549,81 @@ __device__ __forceinline__ uint32_t nm_ex_word(const uint16_t* src, int cnt, boo
   return bits;
 }
 
-template <int M>
+// The fp16 words of gamma * (m . x') for one 32-entry word.
+__device__ __forceinline__ void nm_ex_store(uint16_t* dst, int cnt, const uint32_t (&xs)[16],
+                                            uint32_t bits, bool scale, float gamma) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (i * 8 < cnt) {
+      uint32_t p[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = i * 8 + 2 * k;
+        if (!scale) {
+          const uint32_t lo = ((bits >> e) & 1u) ? (xs[i * 4 + k] & 0xffffu) : 0u;
+          const uint32_t hi = ((bits >> (e + 1)) & 1u) ? (xs[i * 4 + k] & 0xffff0000u) : 0u;
+          p[k] = lo | hi;
+        } else {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xs[i * 4 + k]));
+          const float a = ((bits >> e) & 1u) ? __fmul_rn(gamma, f.x) : 0.f;
+          const float b = ((bits >> (e + 1)) & 1u) ? __fmul_rn(gamma, f.y) : 0.f;
+          const __half2 h = __floats2half2_rn(a, b);
+          p[k] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+      }
+      reinterpret_cast<uint4*>(dst)[i] = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+}
+
+// Up to kExKeep words per lane (rows up to 32 * 32 * kExKeep entries) stay in
+// registers between the VAR reduction and the scaled store; longer rows run
+// the word a second time.
+constexpr int kExKeep = 2;
+
+template <int M, bool WT, bool VAR>
 __global__ void __launch_bounds__(256)
 nm_ex_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, const float* shift,
-             const float* norms, int var, uint16_t* X_masked, uint32_t* mask_bits,
-             float* gamma_out) {
+             const float* norms, uint16_t* X_masked, uint32_t* mask_bits, float* gamma_out) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   pdl_trigger();
   pdl_wait();
   if (row >= rows) return;                      // uniform across the warp
   const int wpr = (d + 31) >> 5;
-  const float mu = shift != nullptr ? __ldg(shift + row) : 0.f;
+  const bool shifted = shift != nullptr;
+  const float mu = shifted ? __ldg(shift + row) : 0.f;
   const uint16_t* xrow = X + row * (int64_t)d;
   uint16_t* orow = X_masked + row * (int64_t)d;
+  const bool keep = wpr <= 32 * kExKeep;
+  uint32_t kx[VAR ? kExKeep : 1][16], kb[VAR ? kExKeep : 1];
   float full = 0.f, kept = 0.f;
-  for (int w = lane; w < wpr; w += 32) {
+  for (int w = lane, t = 0; w < wpr; w += 32, ++t) {
     const int e0 = w * 32, cnt = min(32, d - e0);
     uint32_t xs[16];
-    const uint32_t bits = nm_ex_word<M>(xrow + e0, cnt, shift != nullptr, mu, norms, e0, n, xs);
+    const uint32_t bits = nm_ex_word<M, WT>(xrow + e0, cnt, shifted, mu, norms, e0, n, xs);
     if (mask_bits != nullptr) mask_bits[row * wpr + w] = bits;
-    if (var) {
+    if constexpr (!VAR) {
+      nm_ex_store(orow + e0, cnt, xs, bits, false, 1.f);
+      continue;
+    }
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float v = h2f((uint16_t)(xs[e >> 1] >> (16 * (e & 1))));
-        const float v2 = e < cnt ? v * v : 0.f;
-        full += v2;
-        kept += ((bits >> e) & 1u) ? v2 : 0.f;
-      }
-    } else {
+    for (int e = 0; e < 32; ++e) {
+      const float v = h2f((uint16_t)(xs[e >> 1] >> (16 * (e & 1))));
+      const float v2 = e < cnt ? v * v : 0.f;
+      full += v2;
+      kept += ((bits >> e) & 1u) ? v2 : 0.f;
+    }
+    if (VAR && keep) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (i * 8 < cnt) {
-          uint32_t p[4];
+      for (int u = 0; u < (VAR ? kExKeep : 1); ++u)
+        if (u == t) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int e = i * 8 + 2 * k;
-            const uint32_t lo = ((bits >> e) & 1u) ? (xs[i * 4 + k] & 0xffffu) : 0u;
-            const uint32_t hi = ((bits >> (e + 1)) & 1u) ? (xs[i * 4 + k] & 0xffff0000u) : 0u;
-            p[k] = lo | hi;
-          }
-          reinterpret_cast<uint4*>(orow + e0)[i] = make_uint4(p[0], p[1], p[2], p[3]);
+          for (int k = 0; k < 16; ++k) kx[u][k] = xs[k];
+          kb[u] = bits;
         }
     }
   }
-  if (!var) {
+  if constexpr (!VAR) {
     if (gamma_out != nullptr && lane == 0) gamma_out[row] = 1.f;
     return;
   }
@@ -593,25 +634,19 @@ nm_ex_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, const f
   }
   const float gamma = (full > 0.f && kept > 0.f) ? __fsqrt_rn(__fdiv_rn(full, kept)) : 1.f;
   if (gamma_out != nullptr && lane == 0) gamma_out[row] = gamma;
+  if (keep) {
+#pragma unroll
+    for (int u = 0; u < (VAR ? kExKeep : 1); ++u) {
+      const int w = lane + 32 * u;
+      if (w < wpr) nm_ex_store(orow + w * 32, min(32, d - w * 32), kx[u], kb[u], true, gamma);
+    }
+    return;
+  }
   for (int w = lane; w < wpr; w += 32) {
     const int e0 = w * 32, cnt = min(32, d - e0);
     uint32_t xs[16];
-    const uint32_t bits = nm_ex_word<M>(xrow + e0, cnt, shift != nullptr, mu, norms, e0, n, xs);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (i * 8 < cnt) {
-        uint32_t p[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = i * 8 + 2 * k;
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xs[i * 4 + k]));
-          const float a = ((bits >> e) & 1u) ? __fmul_rn(gamma, f.x) : 0.f;
-          const float b = ((bits >> (e + 1)) & 1u) ? __fmul_rn(gamma, f.y) : 0.f;
-          const __half2 h = __floats2half2_rn(a, b);
-          p[k] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        reinterpret_cast<uint4*>(orow + e0)[i] = make_uint4(p[0], p[1], p[2], p[3]);
-      }
+    const uint32_t bits = nm_ex_word<M, WT>(xrow + e0, cnt, shifted, mu, norms, e0, n, xs);
+    nm_ex_store(orow + e0, cnt, xs, bits, true, gamma);
   }
 }
 
@@ -722,16 +757,18 @@ cudaError_t launch_nm_ex(const uint16_t* X, int64_t rows, int d, int n, int m, c
                          const float* norms, bool var, uint16_t* X_masked, uint32_t* mask_bits,
                          float* gamma_out, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)((rows + 7) / 8);
-  const int v = var ? 1 : 0;
-  switch (m) {
-    case 1: return launch_pdl(nm_ex_kernel<1>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
-    case 2: return launch_pdl(nm_ex_kernel<2>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
-    case 4: return launch_pdl(nm_ex_kernel<4>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
-    case 8: return launch_pdl(nm_ex_kernel<8>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
-    case 16: return launch_pdl(nm_ex_kernel<16>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
-    case 32: return launch_pdl(nm_ex_kernel<32>, dim3(blocks), dim3(256), 0, stream, X, rows, d, n, shift, norms, v, X_masked, mask_bits, gamma_out);
+  const dim3 grid((unsigned)((rows + 7) / 8)), block(256);
+#define SIG_NM_EX_V(MM, W, V)                                                                  \
+  launch_pdl(nm_ex_kernel<MM, W, V>, grid, block, 0, stream, X, rows, d, n, shift, norms,      \
+             X_masked, mask_bits, gamma_out)
+#define SIG_NM_EX(MM)                                                                           \
+  if (m == MM) {                                                                                \
+    if (norms != nullptr) return var ? SIG_NM_EX_V(MM, true, true) : SIG_NM_EX_V(MM, true, false); \
+    return var ? SIG_NM_EX_V(MM, false, true) : SIG_NM_EX_V(MM, false, false);                 \
   }
+  SIG_NM_EX(1) SIG_NM_EX(2) SIG_NM_EX(4) SIG_NM_EX(8) SIG_NM_EX(16) SIG_NM_EX(32)
+#undef SIG_NM_EX
+#undef SIG_NM_EX_V
   return cudaErrorInvalidValue;
 }
 
