@@ -659,11 +659,12 @@ def bench_batch(args, stream, sig, hbm_peak):
 
 
 def bench_q8(args, stream, sig, hbm_peak):
-    """int8 weights (one scale per column) at the Llama-2-7B shapes, 50 % threshold,
-    against the fp16 sparse GEMV on the same shapes."""
+    """int8 weights (one scale per column) at the Llama-2-7B shapes and a Llama-70B
+    MLP shape, 50 % threshold, against the fp16 sparse GEMV on the same shapes."""
     import torch
     out = {"note": "int8 kept rows cost d_out bytes; fp16 rows 2 d_out"}
-    for name, d_in, d_out in (("q", 4096, 4096), ("gate", 4096, 11008), ("down", 11008, 4096)):
+    for name, d_in, d_out in (("q", 4096, 4096), ("gate", 4096, 11008), ("down", 11008, 4096),
+                              ("70B up", 8192, 28672)):
         QT, scale, x, ts = workloads.q8_projection(seed=args.seed + d_in + d_out, d_in=d_in,
                                                    d_out=d_out)
         t = ts[0.5]
