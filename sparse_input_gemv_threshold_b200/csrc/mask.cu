@@ -604,49 +604,49 @@ nm_ex_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, const f
     if (mask_bits != nullptr) mask_bits[row * wpr + w] = bits;
     if constexpr (!VAR) {
       nm_ex_store(orow + e0, cnt, xs, bits, false, 1.f);
-      continue;
-    }
+    } else {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float v = h2f((uint16_t)(xs[e >> 1] >> (16 * (e & 1))));
-      const float v2 = e < cnt ? v * v : 0.f;
-      full += v2;
-      kept += ((bits >> e) & 1u) ? v2 : 0.f;
-    }
-    if (VAR && keep) {
+      for (int e = 0; e < 32; ++e) {
+        const float v = h2f((uint16_t)(xs[e >> 1] >> (16 * (e & 1))));
+        const float v2 = e < cnt ? v * v : 0.f;
+        full += v2;
+        kept += ((bits >> e) & 1u) ? v2 : 0.f;
+      }
+      if (keep) {
 #pragma unroll
-      for (int u = 0; u < (VAR ? kExKeep : 1); ++u)
-        if (u == t) {
+        for (int u = 0; u < kExKeep; ++u)
+          if (u == t) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) kx[u][k] = xs[k];
-          kb[u] = bits;
-        }
+            for (int k = 0; k < 16; ++k) kx[u][k] = xs[k];
+            kb[u] = bits;
+          }
+      }
     }
   }
   if constexpr (!VAR) {
     if (gamma_out != nullptr && lane == 0) gamma_out[row] = 1.f;
-    return;
-  }
+  } else {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    full += __shfl_xor_sync(kFull, full, o);
-    kept += __shfl_xor_sync(kFull, kept, o);
-  }
-  const float gamma = (full > 0.f && kept > 0.f) ? __fsqrt_rn(__fdiv_rn(full, kept)) : 1.f;
-  if (gamma_out != nullptr && lane == 0) gamma_out[row] = gamma;
-  if (keep) {
-#pragma unroll
-    for (int u = 0; u < (VAR ? kExKeep : 1); ++u) {
-      const int w = lane + 32 * u;
-      if (w < wpr) nm_ex_store(orow + w * 32, min(32, d - w * 32), kx[u], kb[u], true, gamma);
+    for (int o = 16; o > 0; o >>= 1) {
+      full += __shfl_xor_sync(kFull, full, o);
+      kept += __shfl_xor_sync(kFull, kept, o);
     }
-    return;
-  }
-  for (int w = lane; w < wpr; w += 32) {
-    const int e0 = w * 32, cnt = min(32, d - e0);
-    uint32_t xs[16];
-    const uint32_t bits = nm_ex_word<M, WT>(xrow + e0, cnt, shifted, mu, norms, e0, n, xs);
-    nm_ex_store(orow + e0, cnt, xs, bits, true, gamma);
+    const float gamma = (full > 0.f && kept > 0.f) ? __fsqrt_rn(__fdiv_rn(full, kept)) : 1.f;
+    if (gamma_out != nullptr && lane == 0) gamma_out[row] = gamma;
+    if (keep) {
+#pragma unroll
+      for (int u = 0; u < kExKeep; ++u) {
+        const int w = lane + 32 * u;
+        if (w < wpr) nm_ex_store(orow + w * 32, min(32, d - w * 32), kx[u], kb[u], true, gamma);
+      }
+    } else {
+      for (int w = lane; w < wpr; w += 32) {
+        const int e0 = w * 32, cnt = min(32, d - e0);
+        uint32_t xs[16];
+        const uint32_t bits = nm_ex_word<M, WT>(xrow + e0, cnt, shifted, mu, norms, e0, n, xs);
+        nm_ex_store(orow + e0, cnt, xs, bits, true, gamma);
+      }
+    }
   }
 }
 
