@@ -618,7 +618,7 @@ def bench_batch(args, stream, sig, hbm_peak):
     import torch
     out = {"shape": "4096->11008", "l2": "6 rotating weight copies (541 MB)"}
     copies = 6
-    for B in (2, 4, 8):
+    for B in (2, 4, 8, 16):
         WT, X, t = workloads.batch_tokens(seed=args.seed + B, B=B)
         Ws = [torch.from_numpy(WT).cuda()]
         Ws += [Ws[0].clone() for _ in range(copies - 1)]

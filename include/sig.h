@@ -239,12 +239,12 @@ SIG_API int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint1
  *   ws sig_workspace_bytes(SIG_OP_SPARSE_GEMV_BATCH, d_in, d_out, B) bytes
  *      (0 means none is needed and ws may be NULL), 256-byte aligned, zeroed
  *      once before first use; every call leaves it ready for the next.
- * 1 <= B <= SIG_MAX_BATCH; d_in % 8 == 0 (whole 16-byte groups per token row),
+ * 1 <= B <= SIG_MAX_BATCH (16); d_in % 8 == 0 (whole 16-byte groups per token row),
  * d_in <= SIG_MAX_D_IN; d_out % 8 == 0.
  * Errors: SIG_ERR_NULL, SIG_ERR_ARG (B), SIG_ERR_SHAPE, SIG_ERR_ALIGN,
  *         SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
  */
-#define SIG_MAX_BATCH 8
+#define SIG_MAX_BATCH 16
 SIG_API int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out,
                               const uint16_t* X, int64_t B, float t, uint16_t* Y,
                               void* ws, size_t ws_bytes, sig_stream_t stream);

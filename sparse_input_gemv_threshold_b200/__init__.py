@@ -32,7 +32,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
 OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM, OP_RANK_ADAPTER = 1, 2, 3, 4, 5
 OP_SPARSE_GEMV_BATCH = 6
 OP_SPARSE_GEMV_Q8 = 7
-MAX_BATCH = 8
+MAX_BATCH = 16
 MAX_D_IN = 131072
 
 _p, _i64, _i32, _f32, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,

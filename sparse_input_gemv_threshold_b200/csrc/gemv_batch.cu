@@ -1,5 +1,5 @@
 // A few tokens, each with its own threshold mask, through one weight:
-// y_b = W (m_b . x_b), m_b,i = |x_b,i| >= t, for b < B <= 8.
+// y_b = W (m_b . x_b), m_b,i = |x_b,i| >= t, for b < B <= 16.
 //
 // The pages define the single-token product ("Adaptive Rank Allocation ...
 // RaNA Adapters", rebuttal Q5.1: the columns of A that meet a zero mask entry
@@ -8,7 +8,8 @@
 // the masks) once from HBM and applies each token's own mask to it in
 // registers: a row that token b drops contributes x_b,i = 0 to y_b.
 //
-// Launch shape: C x S CTAs of 256 threads (three per SM), a CTA owns a
+// Launch shape: C x S CTAs of 256 threads (three per SM for up to 8 tokens,
+// two for up to 16), a CTA owns a
 // 256-output column tile and the union rows of its interleaved 8-input
 // groups (slice s owns groups s, s+S, s+2S, ...):
 //   1. one thread per group loads that group of every token's x (from L2,
@@ -17,7 +18,7 @@
 //      union rows placed in ascending order, with the tokens' masked values
 //      staged token-major (0 where a token drops the row);
 //   2. for a column tile the work is a small dense contraction,
-//      Y^T (256 outputs x 8 tokens) += W^T rows (256 x 16) . Xm (16 x 8) per
+//      Y^T (256 outputs x 8 or 16 tokens) += W^T rows (256 x 16) . Xm per
 //      step of 16 union rows, which the warp-level mma.m16n8k16 (fp16 in,
 //      float32 accumulate) takes directly: the weight rows reach shared
 //      memory through a multi-stage cp.async pipeline, each warp owns 32
@@ -62,7 +63,10 @@ constexpr int kMmaRowBytes = kTile * 2 + 16;      // 528: padded shared row
 constexpr int kMmaStageBytes = kMmaRows * kMmaRowBytes;
 constexpr int kMmaChunk = 1024;                   // union rows staged per chunk
 constexpr int kMmaXtStride = kMmaChunk * 2 + 16;  // bytes between token rows of staged values
-constexpr int kMmaCtasPerSM = 3;
+// CTAs per SM for a token width (8 or 16 tokens per MMA column block):
+// shared memory holds the tokens' staged values.
+template <int TOK>
+constexpr int mma_ctas_per_sm() { return TOK == 8 ? 3 : 2; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -90,7 +94,8 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
                : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-__global__ void __launch_bounds__(kThreads, kMmaCtasPerSM)
+template <int TOK>
+__global__ void __launch_bounds__(kThreads, mma_ctas_per_sm<TOK>())
 batch_mma_kernel(const __grid_constant__ BArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_tot[kWarps];
@@ -105,7 +110,7 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
   int* wpre = reinterpret_cast<int*>(smem + a.words_bytes);
   unsigned char* stages = smem + a.union_bytes;
   int* sidx = reinterpret_cast<int*>(stages + kMmaStages * kMmaStageBytes);
-  unsigned char* sxt = reinterpret_cast<unsigned char*>(sidx + kMmaChunk);   // 8 x kMmaXtStride bytes
+  unsigned char* sxt = reinterpret_cast<unsigned char*>(sidx + kMmaChunk);   // TOK x kMmaXtStride bytes
 
   pdl_trigger();
   pdl_wait();
@@ -122,14 +127,17 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
     uint32_t u = 0;
     if (k < K) {
       const int e0 = (s + k * S) * 8;
-      uint4 v[8];
 #pragma unroll
-      for (int b = 0; b < 8; ++b)
-        v[b] = b < B ? __ldg(reinterpret_cast<const uint4*>(a.X + (size_t)b * d_in + e0))
-                     : make_uint4(0, 0, 0, 0);
+      for (int b0 = 0; b0 < TOK; b0 += 8) {   // eight tokens' loads in flight at a time
+        uint4 v[8];
 #pragma unroll
-      for (int b = 0; b < 8; ++b)
-        if (b < B) u |= thresh_bits8(v[b], th2);
+        for (int b = 0; b < 8; ++b)
+          v[b] = b0 + b < B ? __ldg(reinterpret_cast<const uint4*>(a.X + (size_t)(b0 + b) * d_in + e0))
+                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+          if (b0 + b < B) u |= thresh_bits8(v[b], th2);
+      }
     }
     wbytes[k] = (uint8_t)u;
   }
@@ -162,11 +170,14 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
 
   // ---- 2. the contraction over the union rows ---------------------------
   const int tile0 = c * kTile;
-  float acc[2][4];
+  constexpr int NT = TOK / 8;               // n8 tiles of tokens
+  float acc[2][NT][4];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[mt][k] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[mt][nt][k] = 0.f;
 
   // this thread's two 16-byte pieces of every staged step (row, 16-byte column)
   int cp_row[2], cp_col[2];
@@ -207,7 +218,7 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
         const int j = rk - c_lo;
         sidx[j] = i;
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
+        for (int b = 0; b < TOK; ++b) {
           uint16_t h = 0;
           if (b < B) {
             h = a.X[(size_t)b * d_in + i];
@@ -218,7 +229,7 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
       }
     }
     // zero values for the padding rows of the last step
-    for (int q = tid; q < 8 * kMmaRows; q += kThreads) {
+    for (int q = tid; q < TOK * kMmaRows; q += kThreads) {
       const int j = cn + (q % kMmaRows);
       if (j < nsteps * kMmaRows) *reinterpret_cast<uint16_t*>(sxt + (q / kMmaRows) * xt_stride + j * 2) = 0;
     }
@@ -236,10 +247,11 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
       cp_async_commit();
       __syncwarp();                    // the fragment loads and MMAs below are warp-wide
       const unsigned char* stg = stages + (ks % kMmaStages) * kMmaStageBytes;
-      uint32_t bf[2];
-      {
-        const int n = lane & 7, kh = (lane >> 3) & 1;
-        ldsm_x2(bf, smem_u32(sxt + n * xt_stride + (ks * kMmaRows + kh * 8) * 2));
+      uint32_t bf[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = nt * 8 + (lane & 7), kh = (lane >> 3) & 1;
+        ldsm_x2(bf[nt], smem_u32(sxt + n * xt_stride + (ks * kMmaRows + kh * 8) * 2));
       }
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
@@ -247,7 +259,8 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
         const int m = warp * 32 + mt * 16 + (q & 1) * 8;
         uint32_t af[4];
         ldsm_x4_trans(af, smem_u32(stg + ((q >> 1) * 8 + r) * kMmaRowBytes + m * 2));
-        mma_16816(acc[mt], af, bf);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], af, bf[nt]);
       }
     }
     cp_async_wait<0>();
@@ -255,56 +268,53 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
 
   // ---- 3. this CTA's partials; the last arriver finishes the tile -------
   const int g = lane >> 2, t4 = lane & 3;
-  if (S == 1) {
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int col = tile0 + warp * 32 + mt * 16 + g + h * 8;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int n = t4 * 2 + e;
-          if (col < d_out && n < B) a.Y[(size_t)n * d_out + col] = f2h_rn(acc[mt][h * 2 + e]);
+          const int n = nt * 8 + t4 * 2 + e;
+          if (col < d_out && n < B) {
+            if (S == 1)
+              a.Y[(size_t)n * d_out + col] = f2h_rn(acc[mt][nt][h * 2 + e]);
+            else
+              a.partials[((size_t)s * B + n) * d_out + col] = acc[mt][nt][h * 2 + e];
+          }
         }
       }
-    return;
-  }
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int col = tile0 + warp * 32 + mt * 16 + g + h * 8;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int n = t4 * 2 + e;
-        if (col < d_out && n < B)
-          a.partials[((size_t)s * B + n) * d_out + col] = acc[mt][h * 2 + e];
-      }
-    }
+  if (S == 1) return;
   __syncthreads();
   if (tid == 0) s_last = atomic_add_acq_rel_gpu(a.counters + c, 1u) == (unsigned)(S - 1);
   __syncthreads();
   if (!s_last) return;
   const int colr = tile0 + tid;
   if (colr < d_out) {
-    // every token's partials of a slice in flight together, two slices at a
+    // eight tokens' partials of a slice in flight together, two slices at a
     // time; each token's sum still runs in slice order
-    float sum[8];
-#pragma unroll
-    for (int b = 0; b < 8; ++b) sum[b] = 0.f;
     const size_t slice_stride = (size_t)B * d_out;
     const float* pp = a.partials + colr;
+#pragma unroll
+    for (int b0 = 0; b0 < TOK; b0 += 8) {
+      float sum[8];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) sum[b] = 0.f;
 #pragma unroll 2
-    for (int q = 0; q < S; ++q) {
-      float v[8];
+      for (int q = 0; q < S; ++q) {
+        float v[8];
 #pragma unroll
-      for (int b = 0; b < 8; ++b) v[b] = b < B ? __ldcg(pp + q * slice_stride + (size_t)b * d_out) : 0.f;
+        for (int b = 0; b < 8; ++b)
+          v[b] = b0 + b < B ? __ldcg(pp + q * slice_stride + (size_t)(b0 + b) * d_out) : 0.f;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) sum[b] += v[b];
+        for (int b = 0; b < 8; ++b) sum[b] += v[b];
+      }
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (b0 + b < B) a.Y[(size_t)(b0 + b) * d_out + colr] = f2h_rn(sum[b]);
     }
-#pragma unroll
-    for (int b = 0; b < 8; ++b)
-      if (b < B) a.Y[(size_t)b * d_out + colr] = f2h_rn(sum[b]);
   }
   if (tid == 0) a.counters[c] = 0u;  // ready for the next call on this workspace
 }
@@ -316,11 +326,13 @@ size_t round_up(size_t v, size_t al) { return (v + al - 1) / al * al; }
 GemvPlan plan_gemv_batch(int64_t d_in, int64_t d_out, int B) {
   GemvPlan p{};
   p.C = (int)((d_out + kTile - 1) / kTile);
-  p.S = std::max(1, std::min(32, (kNumSMs * kMmaCtasPerSM) / std::max(1, p.C)));
+  const int tok = B <= 8 ? 8 : 16;
+  const int cps = tok == 8 ? mma_ctas_per_sm<8>() : mma_ctas_per_sm<16>();
+  p.S = std::max(1, std::min(32, (kNumSMs * cps) / std::max(1, p.C)));
   p.chunk = kMmaChunk;
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
   p.smem = 2 * words + (size_t)kMmaStages * kMmaStageBytes + (size_t)kMmaChunk * 4 +
-           (size_t)8 * kMmaXtStride;
+           (size_t)tok * kMmaXtStride;
   p.counters = p.S > 1 ? round_up((size_t)p.C * 4, 256) : 0;
   p.partials = p.S > 1 ? round_up((size_t)p.S * B * d_out * 4, 256) : 0;
   return p;
@@ -336,10 +348,10 @@ cudaError_t launch_gemv_batch(const GemvPlan& p, const uint16_t* WT, const uint1
   k.counters = reinterpret_cast<unsigned*>(ws);
   k.partials = ws != nullptr ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + p.counters)
                              : nullptr;
-  cudaError_t e = cudaFuncSetAttribute(batch_mma_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  auto fn = B <= 8 ? batch_mma_kernel<8> : batch_mma_kernel<16>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(batch_mma_kernel, dim3(p.C, p.S), dim3(kThreads), p.smem, stream, k);
+  return launch_pdl(fn, dim3(p.C, p.S), dim3(kThreads), p.smem, stream, k);
 }
 
 }  // namespace sig

@@ -82,8 +82,8 @@ inline GatedPlan plan_gated(int64_t d_model, int64_t d_ff) {
   return g;
 }
 
-// A few tokens with their own threshold masks through one weight (B <= 8).
-constexpr int kGemvMaxBatch = 8;
+// A few tokens with their own threshold masks through one weight (B <= 16).
+constexpr int kGemvMaxBatch = 16;
 GemvPlan plan_gemv_batch(int64_t d_in, int64_t d_out, int B);
 cudaError_t launch_gemv_batch(const GemvPlan& p, const uint16_t* WT, const uint16_t* X, uint16_t* Y,
                               int B, int d_in, int d_out, float t, void* ws, cudaStream_t stream);

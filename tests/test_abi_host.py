@@ -160,7 +160,7 @@ def test_batch_validation(lib):
     big = 1 << 30
     assert f(None, 64, 64, FAKE, 2, 0.0, FAKE, FAKE, big, None) == NULL
     assert f(FAKE, 64, 64, FAKE, 0, 0.0, FAKE, FAKE, big, None) == ARG
-    assert f(FAKE, 64, 64, FAKE, 9, 0.0, FAKE, FAKE, big, None) == ARG
+    assert f(FAKE, 64, 64, FAKE, 17, 0.0, FAKE, FAKE, big, None) == ARG
     assert f(FAKE, 60, 64, FAKE, 2, 0.0, FAKE, FAKE, big, None) == SHAPE     # d_in % 8
     assert f(FAKE, 64, 60, FAKE, 2, 0.0, FAKE, FAKE, big, None) == SHAPE     # d_out % 8
     assert f(FAKE, 64, 64, FAKE_ODD, 2, 0.0, FAKE, FAKE, big, None) == ALIGN
@@ -168,7 +168,8 @@ def test_batch_validation(lib):
     assert need > 0
     assert f(FAKE, 64, 64, FAKE, 2, 0.0, FAKE, FAKE, need - 1, None) == WORKSPACE
     assert f(FAKE, 64, 64, FAKE, 2, 0.0, FAKE, None, need, None) == WORKSPACE
-    assert lib.sig_workspace_bytes(6, 64, 64, 9) == 0
+    assert lib.sig_workspace_bytes(6, 64, 64, 17) == 0
+    assert lib.sig_workspace_bytes(6, 64, 64, 16) > 0
     assert lib.sig_workspace_bytes(6, 60, 64, 2) == 0
 
 
