@@ -208,3 +208,29 @@ def test_gated_and_gemm_validation(lib):
     assert lib.sig_workspace_init(None, 16, None) == NULL
     assert lib.sig_workspace_init(FAKE + 16, 16, None) == ALIGN
     assert lib.sig_workspace_init(None, 0, None) == OK
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """The product path has no fallback: with libsig.so absent, importing the
+    binding raises instead of computing anything elsewhere."""
+    import types
+    src = open(os.path.join(ROOT, "sparse_input_gemv_threshold_b200", "__init__.py")).read()
+    key = 'LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")'
+    assert key in src
+    missing = str(tmp_path / "libsig.so")
+    mod = types.ModuleType("sig_without_library")
+    with pytest.raises(ImportError):
+        exec(compile(src.replace(key, f"LIB_PATH = {missing!r}"), "sig_without_library", "exec"),
+             mod.__dict__)
+
+
+def test_product_never_touches_the_oracle():
+    """Neither the binding, the build script nor the CUDA sources name the
+    oracle package; only tests, the smoke check and the bench's CPU legs may."""
+    pkg = os.path.join(ROOT, "sparse_input_gemv_threshold_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "oracle/" not in text, f
