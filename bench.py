@@ -58,7 +58,8 @@ def parse():
     ap.add_argument("--profile-case", default=None,
                     help="for ncu: run only this kernel case eagerly and exit "
                          "(a Llama-2-7B projection name or launch group such as 'q|k|v' or "
-                         "'gate|up' at 50%%, 'topk70b', 'batchB' (B tokens, 4096->11008) or 'nm2:4')")
+                         "'gate|up' at 50%%, 'topk70b', 'batchB' (B tokens, 4096->11008), "
+                         "'q8up70b', 'nm2:4' or 'nmex2:4')")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     return ap.parse_args()
 
@@ -951,6 +952,25 @@ def profile_case(args):
         union = int((np.abs(X.astype(np.float32)) >= t).any(axis=0).sum())
         info = {"case": case, "launches": args.launches, "copies": copies,
                 "algorithmic_bytes_per_launch": union * 2 * WT.shape[1] + B * 2 * sum(WT.shape)}
+    elif case == "q8up70b":
+        QT, scale, x, ts = workloads.q8_projection(seed=args.seed, d_in=8192, d_out=28672)
+        copies = 3
+        Qs = [torch.from_numpy(QT).cuda()]
+        Qs += [Qs[0].clone() for _ in range(copies - 1)]
+        sd, xd = torch.from_numpy(scale).cuda(), torch.from_numpy(x).cuda()
+        for i in range(args.launches):
+            sig.sparse_gemv_q8(Qs[i % copies], sd, xd, ts[0.5])
+        nnz = int((np.abs(x.astype(np.float32)) >= ts[0.5]).sum())
+        info = {"case": case, "launches": args.launches, "copies": copies,
+                "algorithmic_bytes_per_launch": nnz * 28672 + 2 * 8192 + 2 * 28672}
+    elif case == "nmex2:4":
+        WT, X = workloads.nm_tokens(args.seed)
+        Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()
+        shift = Xd.float().mean(dim=1).contiguous()
+        norms = sig.row_norms(Wd)
+        for _ in range(args.launches):
+            sig.sparsify_nm_ex(Xd, 2, 4, shift=shift, norms=norms, var=True, want_bits=False)
+        info = {"case": case, "launches": args.launches}
     elif case == "nm2:4":
         WT, X = workloads.nm_tokens(args.seed)
         Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()
