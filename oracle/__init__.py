@@ -84,7 +84,7 @@ __all__ = [
     "masked_matvec", "sparse_linear", "silu", "row_norms", "rana_hidden",
     "rana_scores", "rana_mask", "gated_mlp", "nm_gemm",
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
-    "union_mask", "batched_sparse_linear", "q8_sparse_linear",
+    "union_mask", "batched_sparse_linear", "q8_sparse_linear", "teal_mlp",
     "pts_shift", "wt_scores", "nm_mask_by_score", "var_gamma", "nm_variant", "nm_variant_gemm",
 ]
 
@@ -430,6 +430,21 @@ def q8_sparse_linear(QT, scale, x, mask, cols=None) -> dict:
     idx = compact(mask)
     return {"mask": np.asarray(mask, dtype=bool), "idx": idx, "nnz": int(idx.size),
             "y64": y64, "y16": fp16(y64), "bound": bound}
+
+
+def teal_mlp(x, WgT, WuT, WdT, t_x: float, t_h: float, cols=None) -> dict:
+    """A gated MLP with TEAL's magnitude threshold on the input of every
+    product ([TEAL] Abstract: the hidden states that feed each matrix
+    multiplication): g and u from the kept entries of x (|x_i| >= t_x), float64;
+    h = fp16(SiLU(g) * u); y = W_down (m . h) with m_i = |h_i| >= t_h."""
+    m_x = threshold_mask(x, t_x)
+    g, _ = masked_matvec(WgT, x, m_x)
+    u, _ = masked_matvec(WuT, x, m_x)
+    h16 = fp16(silu(g) * u)
+    m_h = threshold_mask(h16, t_h)
+    out = sparse_linear(WdT, h16, m_h, cols)
+    out.update({"mask_x": m_x, "g": g, "u": u, "h16": h16})
+    return out
 
 
 # ---------------------------------------------------------------------------

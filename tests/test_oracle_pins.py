@@ -689,3 +689,35 @@ def test_var_restores_the_row_norm():
     assert np.allclose(np.linalg.norm(out["xm64"], axis=1), np.linalg.norm(xs, axis=1), rtol=1e-13)
     zero = oracle.var_gamma(np.zeros((1, 8), np.float16), np.ones((1, 8), bool))
     assert zero.tolist() == [1.0]
+
+
+# ---------------------------------------------------------------------------
+# Gated MLP with TEAL thresholds on both inputs
+# ---------------------------------------------------------------------------
+
+def test_teal_mlp_reductions():
+    """t_x = 0 keeps every input: g, u and h are those of the dense gated MLP;
+    t_h = 0 then makes y the dense down product of h; an empty input mask
+    gives g = u = 0, h = 0 and y = 0."""
+    rng = np.random.default_rng(61)
+    d_model, d_ff = 24, 40
+    x = rng.normal(0, 1, d_model).astype(np.float16)
+    WgT = rng.normal(0, 0.3, (d_model, d_ff)).astype(np.float16)
+    WuT = rng.normal(0, 0.3, (d_model, d_ff)).astype(np.float16)
+    WdT = rng.normal(0, 0.3, (d_ff, d_model)).astype(np.float16)
+    g, u, h = oracle.rana_hidden(x, WgT, WuT)
+    out = oracle.teal_mlp(x, WgT, WuT, WdT, 0.0, 0.0)
+    assert np.array_equal(out["g"], g) and np.array_equal(out["u"], u)
+    assert np.array_equal(out["h16"].view(np.uint16), h.view(np.uint16))
+    dense = oracle.sparse_linear(WdT, h, np.ones(d_ff, bool))
+    assert np.array_equal(out["y64"], dense["y64"])
+    none = oracle.teal_mlp(x, WgT, WuT, WdT, float("inf"), 0.0)
+    assert not none["mask_x"].any() and not np.any(none["h16"].astype(np.float64))
+    assert not np.any(none["y64"])
+    # the input mask acts on the rows of W_gate and W_up: dropping x_i equals zeroing it
+    t = float(np.sort(np.abs(x.astype(np.float64)))[12])
+    part = oracle.teal_mlp(x, WgT, WuT, WdT, t, 0.3)
+    x0 = np.where(oracle.threshold_mask(x, t), x, np.float16(0))
+    g0, u0, h0 = oracle.rana_hidden(x0, WgT, WuT)
+    assert np.array_equal(part["h16"].view(np.uint16), h0.view(np.uint16))
+    assert np.array_equal(part["mask"], oracle.threshold_mask(h0, 0.3))
