@@ -414,6 +414,7 @@ def run_ours(args, rank, world, local):
         extras["topk_qsparse_70b"] = bench_topk(args, stream, sig, hbm_peak)
         extras["rana_gated_mlp"] = bench_rana(args, stream, sig, hbm_peak)
         extras["nm_gemm"] = bench_nm(args, stream, sig, bf16_peak)
+        extras["teal_mlp"] = bench_teal_mlp(args, stream, sig, hbm_peak)
         extras["rana_rank_adapter"] = bench_rank_adapter(args, stream, sig, hbm_peak)
         extras["batched_per_token_masks"] = bench_batch(args, stream, sig, hbm_peak)
         extras["int8_weights"] = bench_q8(args, stream, sig, hbm_peak)
@@ -555,6 +556,46 @@ def bench_rana(args, stream, sig, hbm_peak):
            "us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
            "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
            "l2": "2 rotating weight copies of 258 MB"}
+    del Ws, sg
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_teal_mlp(args, stream, sig, hbm_peak):
+    """Gated MLP with the 50 % threshold on x (gate and up, one fused launch)
+    and the 50 % threshold on h (down), Llama-2-7B MLP shapes."""
+    import torch
+    mlp = workloads.rana_mlp(args.seed)
+    d_model, d_ff = mlp.WgT.shape
+    xh = workloads.draw_vector(np.random.default_rng(args.seed), d_model, "laplace")
+    t_x = workloads.quantile_threshold(xh, 0.5)
+    x = torch.from_numpy(xh).cuda()
+    Ws = [tuple(torch.from_numpy(a).cuda() for a in (mlp.WgT, mlp.WuT, mlp.WdT))]
+    Ws += [tuple(w.clone() for w in Ws[0]) for _ in range(2)]
+    h = torch.empty(d_ff, dtype=torch.float16, device="cuda")
+    y = torch.empty(d_model, dtype=torch.float16, device="cuda")
+    ws = torch.zeros(sig.workspace_bytes(sig.OP_GATED_MLP, d_model, d_ff), dtype=torch.uint8,
+                     device="cuda")
+    # t_h: 50 % quantile of this path's own h (timing only)
+    sig.teal_mlp_sparse(x, *Ws[0], t_x, 0.0, y=y, h_out=h, ws=ws)
+    hv = h.float().abs().cpu().numpy()
+    t_h = float(np.sort(hv)[d_ff // 2])
+    nnz_x = int((np.abs(xh.astype(np.float32)) >= t_x).sum())
+    nnz_h = int((hv >= t_h).sum())
+
+    def f(W):
+        def g():
+            sig.teal_mlp_sparse(x, *W, t_x, t_h, y=y, h_out=h, ws=ws, stream=stream)
+        return g
+    sg = StepGraphs([f(W) for W in Ws], stream, per_graph=12)
+    steps = 300
+    us = time_steps(sg, steps, 12, stream) / steps * 1e6
+    b = nnz_x * 2 * d_ff * 2 + nnz_h * 2 * d_model + 2 * d_model * 2 + 2 * d_ff * 2
+    res = {"shapes": "4096->11008 x2 (threshold on x), 11008->4096 (threshold on h)",
+           "sparsity_x": round(1 - nnz_x / d_model, 4), "sparsity_h": round(1 - nnz_h / d_ff, 4),
+           "us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+           "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
+           "l2": "3 rotating weight copies of 271 MB"}
     del Ws, sg
     torch.cuda.empty_cache()
     return res

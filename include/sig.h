@@ -338,6 +338,27 @@ SIG_API int sig_col_sums(const uint16_t* WT, int64_t rows, int64_t cols, float* 
                          sig_stream_t stream);
 
 /*
+ * Gated MLP with TEAL's magnitude threshold on the input of every product
+ * (TEAL README, Abstract: the hidden states that feed each matrix
+ * multiplication):
+ *   m_x = |x_i| >= t_x;  g = GateProj(m_x . x), u = UpProj(m_x . x)
+ *                                        (one fused sparse GEMV for both,
+ *                                         float32 accumulation)
+ *   h = fp16(SiLU(g) * u)                (SiLU(z) = z / (1 + exp(-z)), float32)
+ *   m_h = |h_i| >= t_h;  y = W_down (m_h . h)        (sparse GEMV as sparse_gemv)
+ *   x [d_model] fp16.  WgT, WuT [d_model x d_ff] fp16.  WdT [d_ff x d_model] fp16.
+ *   y [d_model] fp16 out.  h_out [d_ff] fp16 out, nullable.
+ *   mask_out [ceil(d_ff/32)] uint32 out (m_h), nullable.
+ *   ws sig_workspace_bytes(SIG_OP_GATED_MLP, d_model, d_ff, 0) bytes.
+ * d_model % 8 == 0, d_ff % 8 == 0, d_model and d_ff <= SIG_MAX_D_IN.
+ * Errors: as sparse_gemv.
+ */
+SIG_API int teal_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                            const uint16_t* WdT, int64_t d_model, int64_t d_ff, float t_x,
+                            float t_h, uint16_t* y, uint16_t* h_out, uint32_t* mask_out,
+                            void* ws, size_t ws_bytes, sig_stream_t stream);
+
+/*
  * l2 norm of every row of a row-major fp16 matrix, accumulated in float64 and
  * rounded once to float32.  For WdT it yields the ||W^down_i|| of RaNA Eqn. 12.
  *   WT [rows x cols] fp16 (16-byte aligned, cols % 8 == 0).  norms [rows] float32 out.

@@ -24,7 +24,7 @@ __all__ = [
     "nm_act_gemm", "take_device_error", "status_string", "gated_mlp_sparse_noalloc",
     "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
     "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch", "OP_SPARSE_GEMV_Q8",
-    "sparse_gemv_q8", "sparsify_nm_ex", "nm_act_gemm_ex", "col_sums",
+    "sparse_gemv_q8", "sparsify_nm_ex", "nm_act_gemm_ex", "col_sums", "teal_mlp_sparse",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -61,6 +61,7 @@ _SIGNATURES = {
     "nm_act_gemm_ex": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _sz,
                               _p]),
     "sig_col_sums": (_i32, [_p, _i64, _i64, _p, _p]),
+    "teal_mlp_sparse": (_i32, [_p, _p, _p, _p, _i64, _i64, _f32, _f32, _p, _p, _p, _p, _sz, _p]),
 }
 
 
@@ -342,6 +343,22 @@ def sparse_gemv_batch(WT, X, t: float, Y=None, ws=None, stream=None):
         _ptr(WT), d_in, d_out, _ptr(X), B, float(t), _ptr(Y), _ptr(ws), ws.numel(),
         _stream(stream)))
     return Y
+
+
+def teal_mlp_sparse(x, WgT, WuT, WdT, t_x: float, t_h: float, y=None, h_out=None, mask_out=None,
+                    ws=None, stream=None):
+    """Gated MLP with the magnitude threshold on x (gate and up) and on h (down).  Returns y."""
+    for name, w in (("WgT", WgT), ("WuT", WuT), ("WdT", WdT), ("x", x)):
+        _need(w, torch.float16, name, x.device)
+    d_model, d_ff = WgT.shape
+    if y is None:
+        y = torch.empty(d_model, dtype=torch.float16, device=x.device)
+    if ws is None:
+        ws = workspace(OP_GATED_MLP, d_model, d_ff, device=x.device, stream=stream)
+    _check("teal_mlp_sparse", _lib.teal_mlp_sparse(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(WdT), d_model, d_ff, float(t_x), float(t_h), _ptr(y),
+        _ptr(h_out), _ptr(mask_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
 
 
 def rank_adapter_sparse(x, BT, AT, t: float, y=None, v_out=None, mask_out=None, ws=None,

@@ -244,6 +244,37 @@ int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT
   return cuda_status(launch_gemv(MASK_THRESH_SCALED, EPI_STORE, g.down, dn, (cudaStream_t)stream));
 }
 
+int teal_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                    const uint16_t* WdT, int64_t d_model, int64_t d_ff, float t_x, float t_h,
+                    uint16_t* y, uint16_t* h_out, uint32_t* mask_out, void* ws, size_t ws_bytes,
+                    sig_stream_t stream) {
+  if (x == nullptr || WgT == nullptr || WuT == nullptr || WdT == nullptr || y == nullptr)
+    return SIG_ERR_NULL;
+  int sh = check_gemv_shape(d_model, d_ff);
+  if (sh == SIG_OK) sh = check_gemv_shape(d_ff, d_model);
+  if (sh != SIG_OK) return sh;
+  if (!aligned16(x) || !aligned16(WgT) || !aligned16(WuT) || !aligned16(WdT) || !aligned16(y) ||
+      (h_out != nullptr && !aligned16(h_out)))
+    return SIG_ERR_ALIGN;
+  const GatedPlan g = plan_gated(d_model, d_ff);
+  if (ws == nullptr || ws_bytes < g.total) return SIG_ERR_WORKSPACE;
+  if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  char* base = reinterpret_cast<char*>(ws);
+  uint16_t* h = h_out != nullptr ? h_out : reinterpret_cast<uint16_t*>(base + g.off_h);
+
+  GemvLaunch up{};
+  up.WT[0] = WgT; up.WT2 = WuT; up.y[0] = h; up.d_out[0] = (int)d_ff;
+  up.x = x; up.t = t_x; up.d_in = (int)d_model; up.ws = base;
+  cudaError_t e = launch_gemv(MASK_THRESH, EPI_SILU_MUL, g.up, up, (cudaStream_t)stream);
+  if (e != cudaSuccess) return SIG_ERR_CUDA;
+
+  GemvLaunch dn{};
+  dn.WT[0] = WdT; dn.y[0] = y; dn.d_out[0] = (int)d_model;
+  dn.x = h; dn.t = t_h; dn.d_in = (int)d_ff; dn.mask_out = mask_out;
+  dn.ws = base + g.off_down;
+  return cuda_status(launch_gemv(MASK_THRESH, EPI_STORE, g.down, dn, (cudaStream_t)stream));
+}
+
 int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uint16_t* AT, int64_t d_in,
                         int64_t r, int64_t d_out, float t, uint16_t* y, uint16_t* v_out,
                         uint32_t* mask_out, void* ws, size_t ws_bytes, sig_stream_t stream) {

@@ -410,8 +410,9 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   k.partials = a.ws != nullptr ? reinterpret_cast<float*>(reinterpret_cast<char*>(a.ws) + p.counters)
                                : nullptr;
   if (epi == EPI_SILU_MUL) {
-    if (mode != MASK_DENSE) return cudaErrorInvalidValue;
-    return launch_t<MASK_DENSE, true, EPI_SILU_MUL>(p, k, stream);
+    if (mode == MASK_DENSE) return launch_t<MASK_DENSE, true, EPI_SILU_MUL>(p, k, stream);
+    if (mode == MASK_THRESH) return launch_t<MASK_THRESH, true, EPI_SILU_MUL>(p, k, stream);
+    return cudaErrorInvalidValue;
   }
   if (a.n_mat > 1) {
     if (mode == MASK_THRESH) return launch_t<MASK_THRESH, false, EPI_STORE, true>(p, k, stream);

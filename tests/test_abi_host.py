@@ -173,6 +173,16 @@ def test_batch_validation(lib):
     assert lib.sig_workspace_bytes(6, 60, 64, 2) == 0
 
 
+def test_teal_mlp_validation(lib):
+    f = lib.teal_mlp_sparse
+    big = 1 << 30
+    assert f(None, FAKE, FAKE, FAKE, 64, 128, 0.0, 0.0, FAKE, None, None, FAKE, big, None) == NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 120 + 4, 0.0, 0.0, FAKE, None, None, FAKE, big, None) == SHAPE
+    assert f(FAKE, FAKE_ODD, FAKE, FAKE, 64, 128, 0.0, 0.0, FAKE, None, None, FAKE, big, None) == ALIGN
+    need = lib.sig_workspace_bytes(3, 64, 128, 0)
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 128, 0.0, 0.0, FAKE, None, None, FAKE, need - 1, None) == WORKSPACE
+
+
 def test_rank_adapter_validation(lib):
     f = lib.rank_adapter_sparse
     big = 1 << 30
