@@ -61,7 +61,7 @@ def mask_words(t):
 
 
 def assert_within(y16, y64, bound, what=""):
-    """The benchmark spec tolerance per output: |y - y64| <= 2e-3 * sum|W x| (plus one
+    """The parity tolerance per output: |y - y64| <= 2e-3 * sum|W x| (plus one
     fp16 subnormal step, the finest spacing an fp16 result can have)."""
     import numpy as np
     y = np.asarray(y16, dtype=np.float16).astype(np.float64).ravel()
