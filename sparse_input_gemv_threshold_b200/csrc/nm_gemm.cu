@@ -12,6 +12,10 @@
 //     and frees each stage with tcgen05.commit;
 //   - all four warps then read their 32 accumulator lanes with tcgen05.ld,
 //     round to fp16 and store.
+// Launched with programmatic stream serialization: the launch, the mbarrier
+// setup and the tensor-memory allocation overlap the end of the kernel before
+// it; every thread then waits for that kernel (griddepcontrol.wait) before it
+// reads global memory or starts a timed wait.
 // Every mbarrier wait gives up after ~2 s of clock cycles: the kernel then
 // records SIG_ERR_TIMEOUT in a device error word, lets the copies it issued
 // land (again with a limit), frees its tensor memory and returns.
@@ -132,6 +136,7 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
   const int kblocks = K / kBK;
   volatile int* abort_flag = &sm.abort_flag;
+  pdl_trigger();
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -154,6 +159,9 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = sm.tmem_base;
+  // Nothing is read from global memory before the kernel before this one in
+  // the stream has finished, and every timed wait starts after it.
+  pdl_wait();
 
   constexpr uint32_t kStageBytes = (kBM * kBK + kBK * BN) * 2;
 
@@ -306,8 +314,9 @@ cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, uint16_t* Y,
   auto fn = gemm_f16_kernel<BN>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(N / BN, M / kBM);
-  fn<<<grid, kThreads, smem, stream>>>(ma, mb, Y, M, N, K, shift, colsum);
+  const dim3 grid(N / BN, M / kBM);
+  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, Y, M, N, K, shift, colsum);
+  if (e != cudaSuccess) return e;
   return cudaPeekAtLastError();
 }
 
