@@ -448,7 +448,7 @@ nm_mask_kernel(const uint16_t* __restrict__ X, int64_t rows, int d, int n, uint1
 // i%32 of word i/32, little-endian), and the row's last vector also clears
 // the padding bytes of its last word.  Each thread takes kVecPerThread
 // vectors a grid-stride apart, all loads issued first.
-constexpr int kVecPerThread = 2;
+constexpr int kVecPerThread = 1;
 
 template <int M>
 __global__ void __launch_bounds__(256)
