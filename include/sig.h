@@ -33,6 +33,10 @@
  *     index first; +v/-v and +0/-0 tie; a NaN ranks below every number.
  *   - All work is enqueued asynchronously on `stream` (NULL = legacy default
  *     stream).  Calls that share a workspace must not overlap on the device.
+ *   - Alignment: besides the 16-byte rules each entry point states, every
+ *     uint32, int32 and float32 buffer (masks, index lists, counts, norms,
+ *     shifts, sums, scales) must be 4-byte aligned and every fp16 buffer
+ *     2-byte aligned; otherwise the call returns SIG_ERR_ALIGN.
  *   - Errors: arguments are checked on the host before anything is enqueued,
  *     and a non-zero sig_status comes back with nothing launched.  A launch
  *     failure returns SIG_ERR_CUDA.  Nothing throws across the ABI.

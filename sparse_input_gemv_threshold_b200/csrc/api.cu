@@ -17,6 +17,9 @@ namespace {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+// Natural alignment of a 32-bit buffer (uint32 masks, int32 indices and
+// counts, float32 vectors); NULL passes.
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SIG_OK : SIG_ERR_CUDA; }
 
 int check_gemv_shape(int64_t d_in, int64_t d_out) {
@@ -94,7 +97,7 @@ int sparsify_threshold(const uint16_t* x, int64_t d, float t, uint32_t* mask_bit
                        int32_t* nnz, sig_stream_t stream) {
   if (x == nullptr || mask_bits == nullptr) return SIG_ERR_NULL;
   if (d < 1 || d > kMaxDIn) return SIG_ERR_SHAPE;
-  if (!aligned16(x)) return SIG_ERR_ALIGN;
+  if (!aligned16(x) || !aligned4(mask_bits) || !aligned4(idx) || !aligned4(nnz)) return SIG_ERR_ALIGN;
   return cuda_status(launch_threshold_compact(x, (int)d, t, mask_bits, idx, nnz,
                                               (cudaStream_t)stream));
 }
@@ -107,7 +110,7 @@ int sparsify_topk(const uint16_t* x, int64_t d, int64_t k, uint32_t* mask_bits, 
     return SIG_ERR_NULL;
   if (d < 1 || d > kMaxTopkD) return SIG_ERR_SHAPE;
   if (k < 0 || k > d) return SIG_ERR_ARG;
-  if (!aligned16(x)) return SIG_ERR_ALIGN;
+  if (!aligned16(x) || !aligned4(mask_bits) || !aligned4(idx) || !aligned4(nnz)) return SIG_ERR_ALIGN;
   return cuda_status(launch_topk(x, (int)d, (int)k, mask_bits, idx, nnz, (cudaStream_t)stream));
 }
 
@@ -117,7 +120,8 @@ int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m, uint16
   if (rows < 0 || d < 1 || d % m != 0 || d > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
   if (rows == 0) return SIG_OK;  // an empty batch: nothing to read or write
   if (X == nullptr || (X_masked == nullptr && mask_bits == nullptr)) return SIG_ERR_NULL;
-  if (d % 8 != 0 || !aligned16(X) || (X_masked != nullptr && !aligned16(X_masked)))
+  if (d % 8 != 0 || !aligned16(X) || (X_masked != nullptr && !aligned16(X_masked)) ||
+      !aligned4(mask_bits))
     return SIG_ERR_ALIGN;
   return cuda_status(launch_nm_mask(X, rows, (int)d, n, m, X_masked, mask_bits,
                                     (cudaStream_t)stream));
@@ -130,7 +134,8 @@ int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t*
   if (idx != nullptr && nnz == nullptr) return SIG_ERR_NULL;
   const int sh = check_gemv_shape(d_in, d_out);
   if (sh != SIG_OK) return sh;
-  if (!aligned16(WT) || !aligned16(x) || !aligned16(y)) return SIG_ERR_ALIGN;
+  if (!aligned16(WT) || !aligned16(x) || !aligned16(y) || !aligned4(idx) || !aligned4(nnz))
+    return SIG_ERR_ALIGN;
   const GemvPlan p = plan_gemv(d_in, d_out, false);
   if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
   if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
@@ -196,7 +201,7 @@ int sparse_gemv_multi(int n_mat, const uint16_t* const* WT, const int64_t* d_out
     total += d_out[i];
   }
   if (total > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
-  if (!aligned16(x)) return SIG_ERR_ALIGN;
+  if (!aligned16(x) || !aligned4(idx) || !aligned4(nnz)) return SIG_ERR_ALIGN;
   const GemvPlan p = plan_gemv_multi(d_in, d_out, n_mat, false);
   if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
   if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
@@ -223,7 +228,7 @@ int gated_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT
   if (sh == SIG_OK) sh = check_gemv_shape(d_ff, d_model);
   if (sh != SIG_OK) return sh;
   if (!aligned16(x) || !aligned16(WgT) || !aligned16(WuT) || !aligned16(WdT) || !aligned16(y) ||
-      (h_out != nullptr && !aligned16(h_out)))
+      (h_out != nullptr && !aligned16(h_out)) || !aligned4(down_norms) || !aligned4(mask_out))
     return SIG_ERR_ALIGN;
   const GatedPlan g = plan_gated(d_model, d_ff);
   if (ws == nullptr || ws_bytes < g.total) return SIG_ERR_WORKSPACE;
@@ -254,7 +259,7 @@ int teal_mlp_sparse(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
   if (sh == SIG_OK) sh = check_gemv_shape(d_ff, d_model);
   if (sh != SIG_OK) return sh;
   if (!aligned16(x) || !aligned16(WgT) || !aligned16(WuT) || !aligned16(WdT) || !aligned16(y) ||
-      (h_out != nullptr && !aligned16(h_out)))
+      (h_out != nullptr && !aligned16(h_out)) || !aligned4(mask_out))
     return SIG_ERR_ALIGN;
   const GatedPlan g = plan_gated(d_model, d_ff);
   if (ws == nullptr || ws_bytes < g.total) return SIG_ERR_WORKSPACE;
@@ -283,7 +288,7 @@ int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uint16_t* A
   if (sh == SIG_OK) sh = check_gemv_shape(r, d_out);
   if (sh != SIG_OK) return sh;
   if (!aligned16(x) || !aligned16(BT) || !aligned16(AT) || !aligned16(y) ||
-      (v_out != nullptr && !aligned16(v_out)))
+      (v_out != nullptr && !aligned16(v_out)) || !aligned4(mask_out))
     return SIG_ERR_ALIGN;
   const RankPlan g = plan_rank(d_in, r, d_out);
   if (ws == nullptr || ws_bytes < g.total) return SIG_ERR_WORKSPACE;
@@ -311,7 +316,8 @@ int sparsify_nm_ex(const uint16_t* X, int64_t rows, int64_t d, int n, int m, con
   if (rows < 0 || d < 1 || d % m != 0 || d > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
   if (rows == 0) return SIG_OK;
   if (X == nullptr || X_masked == nullptr) return SIG_ERR_NULL;
-  if (d % 8 != 0 || !aligned16(X) || !aligned16(X_masked) || (norms != nullptr && !aligned16(norms)))
+  if (d % 8 != 0 || !aligned16(X) || !aligned16(X_masked) || (norms != nullptr && !aligned16(norms)) ||
+      !aligned4(shift) || !aligned4(mask_bits) || !aligned4(gamma_out))
     return SIG_ERR_ALIGN;
   return cuda_status(launch_nm_ex(X, rows, (int)d, n, m, shift, norms, var != 0, X_masked,
                                   mask_bits, gamma_out, (cudaStream_t)stream));
@@ -327,7 +333,8 @@ int nm_act_gemm_ex(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* W
   if (rows < 128 || rows % 128 != 0 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0 ||
       K % m != 0 || rows > (1 << 24) || K > (1 << 20) || N > (1 << 20))
     return SIG_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(WT) || !aligned16(Y) || (norms != nullptr && !aligned16(norms)))
+  if (!aligned16(X) || !aligned16(WT) || !aligned16(Y) || (norms != nullptr && !aligned16(norms)) ||
+      !aligned4(shift) || !aligned4(col_sums))
     return SIG_ERR_ALIGN;
   const size_t need = sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows);
   if (ws == nullptr || ws_bytes < need) return SIG_ERR_WORKSPACE;
@@ -344,6 +351,7 @@ int sig_col_sums(const uint16_t* WT, int64_t rows, int64_t cols, float* sums,
                  sig_stream_t stream) {
   if (WT == nullptr || sums == nullptr) return SIG_ERR_NULL;
   if (rows < 1 || cols < 1 || cols > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(WT) & 1u) != 0 || !aligned4(sums)) return SIG_ERR_ALIGN;
   return cuda_status(launch_col_sums(WT, rows, (int)cols, sums, (cudaStream_t)stream));
 }
 
@@ -351,7 +359,7 @@ int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float* norms,
                   sig_stream_t stream) {
   if (WT == nullptr || norms == nullptr) return SIG_ERR_NULL;
   if (rows < 0 || cols < 8 || cols % 8 != 0 || cols > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
-  if (!aligned16(WT)) return SIG_ERR_ALIGN;
+  if (!aligned16(WT) || !aligned4(norms)) return SIG_ERR_ALIGN;
   return cuda_status(launch_row_norms(WT, rows, (int)cols, norms, (cudaStream_t)stream));
 }
 

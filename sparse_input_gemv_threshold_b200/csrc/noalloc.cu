@@ -54,6 +54,7 @@ cudaError_t scratch_address(void** out) {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 }  // namespace
 
@@ -70,7 +71,7 @@ extern "C" int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT,
       d_ff > kMaxDIn)
     return SIG_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(WgT) || !aligned16(WuT) || !aligned16(WdT) || !aligned16(y) ||
-      (h_out != nullptr && !aligned16(h_out)))
+      (h_out != nullptr && !aligned16(h_out)) || !aligned4(down_norms) || !aligned4(mask_out))
     return SIG_ERR_ALIGN;
   const GatedPlan g = plan_gated(d_model, d_ff);
   if (g.total > (size_t)SIG_NOALLOC_SCRATCH_BYTES) return SIG_ERR_SHAPE;

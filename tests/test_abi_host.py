@@ -244,3 +244,81 @@ def test_product_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "oracle/" not in text, f
+
+
+def test_nm_variant_and_helper_validation(lib):
+    e = lib.sparsify_nm_ex
+    assert e(FAKE, 4, 64, 3, 2, None, None, 0, FAKE, None, None, None) == ARG       # n > m
+    assert e(FAKE, 4, 36, 2, 8, None, None, 0, FAKE, None, None, None) == SHAPE     # m does not divide d
+    assert e(FAKE, 4, 64, 2, 4, None, None, 0, None, None, None, None) == NULL      # X_masked required
+    assert e(None, 4, 64, 2, 4, None, None, 0, FAKE, None, None, None) == NULL
+    assert e(None, 0, 64, 2, 4, None, None, 1, None, None, None, None) == OK        # empty batch
+    assert e(FAKE, 4, 64, 2, 4, None, FAKE + 4, 0, FAKE, None, None, None) == ALIGN   # norms: 16 B
+    assert e(FAKE, 4, 64, 2, 4, FAKE + 2, None, 0, FAKE, None, None, None) == ALIGN   # shift: 4 B
+    assert e(FAKE, 4, 64, 2, 4, None, None, 1, FAKE, None, FAKE + 2, None) == ALIGN   # gamma: 4 B
+    assert e(FAKE, 4, 64, 2, 4, None, None, 0, FAKE, FAKE + 1, None, None) == ALIGN   # mask: 4 B
+    g = lib.nm_act_gemm_ex
+    big = 1 << 30
+    args = dict(shift=None, norms=None, var=0, cs=None, ws=FAKE, nbytes=big)
+
+    def call(rows=256, K=1024, N=1024, n=2, m=4, **kw):
+        a = {**args, **kw}
+        return g(FAKE, rows, K, FAKE, N, n, m, a["shift"], a["norms"], a["var"], a["cs"], FAKE,
+                 a["ws"], a["nbytes"], None)
+    assert call(shift=FAKE) == NULL                      # a shift needs the weight's column sums
+    assert call(rows=100) == SHAPE
+    assert call(K=1000) == SHAPE
+    assert call(n=5) == ARG
+    assert call(shift=FAKE + 2, cs=FAKE) == ALIGN
+    assert call(shift=FAKE, cs=FAKE + 2) == ALIGN
+    assert call(norms=FAKE + 4) == ALIGN
+    assert call(nbytes=16) == WORKSPACE
+    assert call(ws=None) == WORKSPACE
+    c = lib.sig_col_sums
+    assert c(None, 4, 16, FAKE, None) == NULL
+    assert c(FAKE, 4, 16, None, None) == NULL
+    assert c(FAKE, 0, 16, FAKE, None) == SHAPE
+    assert c(FAKE + 1, 4, 16, FAKE, None) == ALIGN       # fp16: 2 B
+    assert c(FAKE, 4, 16, FAKE + 2, None) == ALIGN       # float32: 4 B
+    assert lib.sig_row_norms(FAKE, 4, 16, FAKE + 2, None) == ALIGN
+
+
+def test_noalloc_validation(lib):
+    f = lib.gated_mlp_sparse_noalloc
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 64, 128, 0.1, FAKE, None, None, None) == NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 60, 128, 0.1, FAKE, None, None, None) == SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 131072 + 8, 0.1, FAKE, None, None, None) == SHAPE
+    assert f(FAKE, FAKE_ODD, FAKE, FAKE, FAKE, 64, 128, 0.1, FAKE, None, None, None) == ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 64, 128, 0.1, FAKE, None, None, None) == ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 0.1, FAKE, None, FAKE + 1, None) == ALIGN
+
+
+def test_32bit_buffers_must_be_4_byte_aligned(lib):
+    """Masks, index lists, counts and float vectors are checked on the host,
+    like the 16-byte rules, before anything is enqueued."""
+    big = 1 << 30
+    odd = FAKE + 2
+    st = lib.sparsify_threshold
+    assert st(FAKE, 64, 0.0, odd, None, None, None) == ALIGN
+    assert st(FAKE, 64, 0.0, FAKE, odd, None, None) == ALIGN
+    assert st(FAKE, 64, 0.0, FAKE, FAKE, odd, None) == ALIGN
+    tk = lib.sparsify_topk
+    assert tk(FAKE, 64, 3, odd, FAKE, FAKE, None, 0, None) == ALIGN
+    assert tk(FAKE, 64, 3, FAKE, odd, FAKE, None, 0, None) == ALIGN
+    assert tk(FAKE, 64, 3, FAKE, FAKE, odd, None, 0, None) == ALIGN
+    assert lib.sparsify_nm(FAKE, 4, 64, 2, 4, None, odd, None) == ALIGN
+    sg = lib.sparse_gemv
+    assert sg(FAKE, 64, 64, FAKE, 0.0, odd, FAKE, FAKE, FAKE, big, None) == ALIGN
+    assert sg(FAKE, 64, 64, FAKE, 0.0, FAKE, odd, FAKE, FAKE, big, None) == ALIGN
+    P = ctypes.c_void_p * 2
+    I = ctypes.c_int64 * 2
+    mm = lib.sparse_gemv_multi
+    assert mm(2, P(FAKE, FAKE), I(64, 64), 64, FAKE, 0.0, odd, FAKE, P(FAKE, FAKE), FAKE, big,
+              None) == ALIGN
+    ga = lib.gated_mlp_sparse
+    assert ga(FAKE, FAKE, FAKE, FAKE, odd, 64, 128, 0.1, FAKE, None, None, FAKE, big, None) == ALIGN
+    assert ga(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 0.1, FAKE, None, odd, FAKE, big, None) == ALIGN
+    te = lib.teal_mlp_sparse
+    assert te(FAKE, FAKE, FAKE, FAKE, 64, 128, 0.0, 0.0, FAKE, None, odd, FAKE, big, None) == ALIGN
+    ra = lib.rank_adapter_sparse
+    assert ra(FAKE, FAKE, FAKE, 64, 32, 16, 0.0, FAKE, None, odd, FAKE, big, None) == ALIGN
