@@ -170,9 +170,10 @@ SIG_API int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m
  *   x    [d_in] fp16, 16-byte aligned.       y [d_out] fp16 out, 16-byte aligned.
  *   ws   sig_workspace_bytes(SIG_OP_SPARSE_GEMV, d_in, d_out, 0) bytes, 256-byte
  *        aligned, zeroed once by sig_workspace_init (or allocated zeroed); it
- *        holds the partial sums of the cluster groups of a column tile and
- *        their arrival counters.  When the size is 0 (one group per tile, as
- *        for d_out >= 37888) ws may be NULL.
+ *        holds the float32 partial sums of the split-K slices and one arrival
+ *        counter per 256-column tile.  When the size is 0 (one slice per tile,
+ *        which the planner chooses above 296 tiles, i.e. d_out > 75776) ws may
+ *        be NULL.
  * The result is bit-identical from run to run (fixed-order split-K reduction;
  * no floating-point atomics).  An empty mask writes y = 0.
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d_in < 1, d_in > SIG_MAX_D_IN, d_out < 8,

@@ -73,6 +73,8 @@ def test_workspace_sizes(lib):
     assert ws(1, 4096, 4096, 0) > 0           # split-K partials and per-tile counters
     assert ws(1, 4096, 4096, 0) % 256 == 0
     assert ws(1, 64, 131072, 0) == 0          # > 296 column tiles: one slice, no partials
+    assert ws(1, 4096, 296 * 256, 0) > 0      # 296 tiles of 256 columns still split K
+    assert ws(1, 4096, 296 * 256 + 8, 0) == 0
     assert ws(1, 0, 4096, 0) == 0            # invalid shape
     assert ws(1, 4096, 12, 0) == 0           # d_out % 8
     assert ws(2, 8192, 0, 0) == 0            # top-k needs none
