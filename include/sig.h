@@ -65,7 +65,7 @@ typedef enum {
   SIG_OK = 0,
   SIG_ERR_NULL = 1,       /* a required pointer is NULL                        */
   SIG_ERR_SHAPE = 2,      /* a size is out of range or inconsistent            */
-  SIG_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned where required   */
+  SIG_ERR_ALIGN = 3,      /* a pointer is not aligned as required              */
   SIG_ERR_WORKSPACE = 4,  /* workspace NULL or smaller than sig_workspace_bytes */
   SIG_ERR_CUDA = 5,       /* the CUDA runtime reported an error                */
   SIG_ERR_TIMEOUT = 6,    /* a bounded device-side wait gave up                */
@@ -120,7 +120,8 @@ SIG_API int sig_workspace_init(void* ws, size_t ws_bytes, sig_stream_t stream);
  *   idx        [d] int32 out, nullable: ascending kept indices (first *nnz valid).
  *   nnz        [1] int32 out, nullable: number of kept entries.
  * Errors: SIG_ERR_NULL (x or mask_bits), SIG_ERR_SHAPE (d < 1 or d > SIG_MAX_D_IN),
- *         SIG_ERR_ALIGN (x).
+ *         SIG_ERR_ALIGN (x not 16-byte aligned, or mask_bits, idx or nnz not
+ *         4-byte aligned).
  */
 SIG_API int sparsify_threshold(const uint16_t* x, int64_t d, float t,
                        uint32_t* mask_bits, int32_t* idx, int32_t* nnz,
@@ -146,9 +147,11 @@ SIG_API int sparsify_topk(const uint16_t* x, int64_t d, int64_t k,
  * N:M activation mask (N:M summary, Methodology; Block Q-Sparse in the
  * Q-Sparse rebuttal, A2): for every row of X and every block of m consecutive
  * entries, keep the n of largest |x| (ties by lower index).
- *   X          [rows x d] fp16 row-major, 16-byte aligned.
- *   n, m       1 <= n <= m <= 32, d % m == 0.
- *   X_masked   [rows x d] fp16 out, nullable: X with dropped entries set to +0.
+ *   X          [rows x d] fp16 row-major, 16-byte aligned; d % 8 == 0 so that
+ *              every row starts 16-byte aligned (else SIG_ERR_ALIGN).
+ *   n, m       m in {1, 2, 4, 8, 16, 32}, 1 <= n <= m, d % m == 0.
+ *   X_masked   [rows x d] fp16 out, 16-byte aligned, nullable: X with dropped
+ *              entries set to +0.
  *   mask_bits  [rows x ceil(d/32)] uint32 out, nullable.
  * At least one of X_masked and mask_bits must be non-NULL.  rows == 0 is an
  * empty batch: the call returns SIG_OK and touches no pointer.
@@ -198,8 +201,10 @@ SIG_API int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out,
  *   x, t, idx, nnz   as sparse_gemv (one mask for all the weights).
  *   ws       sig_workspace_bytes_multi(n_mat, d_out, d_in) bytes, 256-byte
  *            aligned, zeroed once (it may be NULL when that size is 0).
- * Results are bit-identical to n_mat separate sparse_gemv calls only up to
- * the split-K order (the grid is planned for all the weights together).
+ * Each y[p] meets the tolerance of sparse_gemv and is bit-identical from run
+ * to run.  It can differ in the last bits from a separate sparse_gemv call on
+ * W_p, because the grid, and so the split-K order, is planned for all the
+ * weights together; with n_mat == 1 it is that call.
  * Errors: SIG_ERR_NULL, SIG_ERR_ARG (n_mat), SIG_ERR_SHAPE, SIG_ERR_ALIGN,
  *         SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
  */
@@ -285,8 +290,8 @@ SIG_API int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, i
  *   y [d_out] fp16 out.  v_out [r] fp16 out, nullable.
  *   mask_out [ceil(r/32)] uint32 out, nullable.
  *   ws sig_workspace_bytes(SIG_OP_RANK_ADAPTER, d_in, d_out, r) bytes.
- * d_in, r, d_out: multiples of 8 (r and d_out as output widths), each
- * <= SIG_MAX_D_IN.  Two launches on `stream`; the caller owns every buffer.
+ * r % 8 == 0 and d_out % 8 == 0 (they are output widths); d_in and r each
+ * in [1, SIG_MAX_D_IN].  Two launches on `stream`; the caller owns every buffer.
  * Errors: as sparse_gemv.
  */
 SIG_API int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uint16_t* AT,
@@ -308,8 +313,9 @@ SIG_API int rank_adapter_sparse(const uint16_t* x, const uint16_t* BT, const uin
  *   X_masked = fp16(gamma_r * m . x')           (VAR: gamma_r = sqrt(sum x'^2 /
  *                                                sum (m x')^2), float32, 1 when
  *                                                either sum is 0; var = 0: gamma 1)
- *   X [rows x d] fp16, row-major.  shift [rows] float32, nullable.
- *   norms [d] float32, 16-byte aligned, nullable.  X_masked [rows x d] fp16 out (required).
+ *   X [rows x d] fp16, row-major, 16-byte aligned.  shift [rows] float32, nullable.
+ *   norms [d] float32, 16-byte aligned, nullable.
+ *   X_masked [rows x d] fp16 out, 16-byte aligned (required).
  *   mask_bits [rows x ceil(d/32)] uint32 out, nullable.  gamma_out [rows] float32 out, nullable.
  * 1 <= n <= m, m in {1, 2, 4, 8, 16, 32}, d % m == 0, d % 8 == 0.
  * Errors: SIG_ERR_ARG (n, m), SIG_ERR_SHAPE, SIG_ERR_NULL, SIG_ERR_ALIGN, SIG_ERR_CUDA.
@@ -336,8 +342,8 @@ SIG_API int nm_act_gemm_ex(const uint16_t* X, int64_t rows, int64_t K, const uin
  * Column sums of a row-major fp16 matrix, accumulated in float64 and rounded
  * once to float32: for WT, r_j = sum_i W[j, i], the vector a per-token shift
  * mu brings back as mu * r (x W = (x - mu) W + mu r).
- *   WT [rows x cols] fp16.  sums [cols] float32 out.
- * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE.
+ *   WT [rows x cols] fp16, rows >= 1, 1 <= cols <= 2^30.  sums [cols] float32 out.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ALIGN.
  */
 SIG_API int sig_col_sums(const uint16_t* WT, int64_t rows, int64_t cols, float* sums,
                          sig_stream_t stream);
@@ -378,7 +384,9 @@ SIG_API int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float*
  *   accumulation on the tensor cores, Y rounded once to fp16.  When n == m
  *   the GEMM runs on X directly.
  *   X  [rows x K] fp16 row-major.   WT [K x N] fp16 row-major.   Y [rows x N] fp16 out.
- *   rows % 128 == 0, K % 64 == 0, N % 128 == 0; m in {1,2,4,8,16,32}, 1 <= n <= m.
+ *   All three 16-byte aligned (WT and X are read by TMA).
+ *   rows % 128 == 0, K % 64 == 0, N % 128 == 0, rows <= 2^24, K and N <= 2^20;
+ *   m in {1,2,4,8,16,32}, 1 <= n <= m, K % m == 0.
  *   ws sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows) bytes (the masked X;
  *      not touched when n == m, so it may be NULL then).
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ARG, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE,
