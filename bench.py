@@ -2,6 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+(W below 3 is raised to 3; the JSON line reports the warm-up steps run.)
+
 Workload (one step): one Llama-2-7B decoder layer's seven projections at
 batch 1 (q, k, v, o 4096x4096; gate, up 4096->11008; down 11008->4096), fp16
 weights ~ N(0, 0.02^2), Laplace activations, TEAL-style magnitude threshold
@@ -62,7 +64,10 @@ def parse():
                          "'gate|up' at 50%%, 'topk70b', 'batchB' (B tokens, 4096->11008), "
                          "'q8up70b', 'nm2:4' or 'nmex2:4')")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
-    return ap.parse_args()
+    args = ap.parse_args()
+    # at least three untimed warm-up steps; the JSON line reports the number run
+    args.warmup = max(3, args.warmup)
+    return args
 
 
 # ---------------------------------------------------------------------------
