@@ -80,3 +80,10 @@ def test_max_over_ranks_two_gloo_ranks():
     for rank, slow, value in got:
         assert slow == 1.75                        # every rank sees the slowest time
         assert value == pytest.approx(20.0 / 1.75)  # all ranks' units over it
+
+
+def test_warmup_is_at_least_three_steps(monkeypatch):
+    for given, run in (("0", 3), ("1", 3), ("3", 3), ("7", 7)):
+        monkeypatch.setattr("sys.argv", ["bench.py", "--steps", "5", "--warmup", given])
+        args = bench.parse()
+        assert args.warmup == run and args.steps == 5
