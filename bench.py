@@ -187,42 +187,72 @@ def capture(fn, stream):
 class StepGraphs:
     """CUDA graphs over a rotation of step callables.
 
-    `big` holds `per_graph` consecutive steps (step i uses fns[i % R]), so the
-    host pays one graph launch per `per_graph` steps; `singles` cover a
-    remainder, so that exactly the requested number of steps runs.
+    ``run(n)`` replays exactly ``n`` steps (step i uses fns[i % R]) as ONE
+    graph of n steps when n <= ``cap``, so that no graph boundary falls inside
+    the timed region and every launch can overlap its predecessor
+    (programmatic dependent launch works inside a graph, not across two graph
+    launches).  Longer runs replay a ``cap``-step graph (a multiple of R) and
+    one graph of the remainder.  Graphs are captured on first use and cached
+    by step count.
     """
 
-    def __init__(self, fns, stream, per_graph):
+    def __init__(self, fns, stream):
         import torch
-        self.fns, self.R = fns, len(fns)
-        self.per = max(self.R, (per_graph // self.R) * self.R)
+        self.fns, self.R, self.stream = fns, len(fns), stream
+        self.cap = max(self.R, (cap // self.R) * self.R)
+        self.graphs = {}
         with torch.cuda.stream(stream):
             for f in fns:                      # one eager pass (kernel attributes)
                 f()
         torch.cuda.synchronize()
 
-        def many():
-            for i in range(self.per):
-                fns[i % self.R]()
-        self.big = capture(many, stream)
-        self.singles = [capture(f, stream) for f in fns]
+    def _graph(self, n):
+        g = self.graphs.get(n)
+        if g is None:
+            fns, R = self.fns, self.R
+
+            def many():
+                for i in range(n):
+                    fns[i % R]()
+            g = self.graphs[n] = capture(many, self.stream)
+        return g
+
+    def prepare(self, n):
+        """Capture the graphs ``run(n)`` replays (outside any timed region)."""
+        q, r = divmod(n, self.cap) if n > self.cap else (0, n)
+        if q:
+            self._graph(self.cap)
+        if r:
+            self._graph(r)
 
     def run(self, n):
-        q, r = divmod(n, self.per)
+        q, r = divmod(n, self.cap) if n > self.cap else (0, n)
         for _ in range(q):
-            self.big.replay()
-        for i in range(r):
-            self.singles[i % self.R].replay()
+            self._graph(self.cap).replay()
+        if r:
+            self._graph(r).replay()
+
+
+def _queue_delay(stream, us=200.0):
+    """Keep the device busy for ~``us`` microseconds before the start event, so
+    that the host has queued the timed graph launches by the time the device
+    reaches them (the wait for the host is then not inside the timed region)."""
+    import torch
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(us * 2000))    # cycles at ~2 GHz
 
 
 def time_steps(sg, steps, warmup, stream, world=1):
     """Warm up, then time exactly `steps` steps with CUDA events on `stream`."""
     import torch
+    sg.prepare(warmup)
+    sg.prepare(steps)
     with torch.cuda.stream(stream):
         sg.run(warmup)
     barrier(world)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _queue_delay(stream)
     with torch.cuda.stream(stream):
         start.record(stream)
         sg.run(steps)
@@ -347,7 +377,7 @@ def run_ours(args, rank, world, local):
         return f
 
     def graphs_for(s):
-        return StepGraphs([step_fn(c, s) for c in range(N_COPIES)], stream, per_graph=12)
+        return StepGraphs([step_fn(c, s) for c in range(N_COPIES)], stream)
 
     # ---- headline ----
     g50 = graphs_for(HEADLINE_SPARSITY)
@@ -390,7 +420,7 @@ def run_ours(args, rank, world, local):
     }
 
     # ---- e2e through the public API with host buffers ----
-    result["e2e"] = e2e(args, groups, copies, gys, gws, stream, sig, world, bytes_step)
+    result["e2e"] = e2e(args, groups, copies, gws, stream, sig, world, bytes_step)
 
     if not args.no_extras and rank == 0:
         extras = {}
@@ -437,7 +467,7 @@ def per_launch(groups, copies, gx, gys, gws, stream, sig, steps):
                 launch_group(sig, copies[c][gi], gx[gi], grp[0].thresholds[HEADLINE_SPARSITY],
                              gys[gi], gws[gi], stream)
             return g
-        sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=48)
+        sg = StepGraphs([f(c) for c in range(N_COPIES)], stream)
         sec = time_steps(sg, steps, 24, stream)
         us = sec / steps * 1e6
         b = group_bytes(grp, kept_count(grp[0], HEADLINE_SPARSITY))
@@ -461,7 +491,7 @@ def seven_launches(groups, copies, gx, stream, sig, steps, bytes_step):
                 sig.sparse_gemv(copies[c][gi][j], gx[gi], t=p.thresholds[HEADLINE_SPARSITY],
                                 y=ys[k], ws=wss[k], stream=stream)
         return g
-    sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=12)
+    sg = StepGraphs([f(c) for c in range(N_COPIES)], stream)
     sec = time_steps(sg, steps, 24, stream)
     us = sec / steps * 1e6
     return {"us_per_step": round(us, 2), "GBps_same_bytes": round(bytes_step / (us * 1e-6) / 1e9, 1)}
@@ -478,7 +508,7 @@ def cublas_dense(groups, copies, gx, stream, steps):
             for k, (gi, j, p) in enumerate(flat):
                 torch.matmul(gx[gi].view(1, -1), copies[c][gi][j], out=outs[k])
         return g
-    sg = StepGraphs([f(c) for c in range(N_COPIES)], stream, per_graph=12)
+    sg = StepGraphs([f(c) for c in range(N_COPIES)], stream)
     sec = time_steps(sg, steps, 24, stream)
     us = sec / steps * 1e6
     dense_bytes = sum(sum(p.d_in * p.d_out * 2 + 2 * p.d_out for p in g) + 2 * g[0].d_in
@@ -508,7 +538,7 @@ def bench_topk(args, stream, sig, hbm_peak):
                 sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
                 sig.sparse_gemv(ws_w[j], X[j], idx=idx, nnz=nnz, y=ys[j], ws=ws[j], stream=stream)
         return g
-    sg = StepGraphs([f(W), f(Wc)], stream, per_graph=8)
+    sg = StepGraphs([f(W), f(Wc)], stream)
     steps = 200
     sec = time_steps(sg, steps, 8, stream)
     us = sec / steps * 1e6
@@ -518,7 +548,7 @@ def bench_topk(args, stream, sig, hbm_peak):
         for j, p in enumerate(projs):
             mb, idx, nnz = bufs[j]
             sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
-    st = StepGraphs([h], stream, per_graph=8)
+    st = StepGraphs([h], stream)
     sec_t = time_steps(st, steps, 8, stream)
     res = {"shapes": "8192->28672 and 28672->8192", "keep": k_frac,
            "us_per_pair": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
@@ -552,7 +582,7 @@ def bench_rana(args, stream, sig, hbm_peak):
             sig.gated_mlp_sparse(x, *W, norms, t, y=y, h_out=h, mask_out=mask, ws=ws, stream=stream)
         return g
     nnz = int((s >= t).sum())
-    sg = StepGraphs([f(W) for W in Ws], stream, per_graph=8)
+    sg = StepGraphs([f(W) for W in Ws], stream)
     steps = 300
     sec = time_steps(sg, steps, 8, stream)
     us = sec / steps * 1e6
@@ -593,7 +623,7 @@ def bench_teal_mlp(args, stream, sig, hbm_peak):
         def g():
             sig.teal_mlp_sparse(x, *W, t_x, t_h, y=y, h_out=h, ws=ws, stream=stream)
         return g
-    sg = StepGraphs([f(W) for W in Ws], stream, per_graph=12)
+    sg = StepGraphs([f(W) for W in Ws], stream)
     steps = 300
     us = time_steps(sg, steps, 12, stream) / steps * 1e6
     b = nnz_x * 2 * d_ff * 2 + nnz_h * 2 * d_model + 2 * d_model * 2 + 2 * d_ff * 2
@@ -633,7 +663,7 @@ def bench_rank_adapter(args, stream, sig, hbm_peak):
         def g():
             sig.rank_adapter_sparse(x, Bs[c], As[c], t, y=y, v_out=v, ws=ws, stream=stream)
         return g
-    sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies)
+    sg = StepGraphs([f(c) for c in range(copies)], stream)
     steps = 320
     sec = time_steps(sg, steps, copies, stream)
     us = sec / steps * 1e6
@@ -647,7 +677,7 @@ def bench_rank_adapter(args, stream, sig, hbm_peak):
         def g():
             torch.matmul(x.view(1, -1), W[c], out=yd)
         return g
-    sd = StepGraphs([dn(c) for c in range(copies)], stream, per_graph=copies)
+    sd = StepGraphs([dn(c) for c in range(copies)], stream)
     us_dense = time_steps(sd, steps, copies, stream) / steps * 1e6
     res = {"shapes": f"B {r}x{d_in} dense, A {d_out}x{r} masked", "sparsity": round(1 - nnz / r, 4),
            "us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
@@ -681,7 +711,7 @@ def bench_batch(args, stream, sig, hbm_peak):
             def g():
                 sig.sparse_gemv_batch(Ws[c], Xd, t, Y=Y, ws=ws, stream=stream)
             return g
-        sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies * 2)
+        sg = StepGraphs([f(c) for c in range(copies)], stream)
         steps = 240
         us = time_steps(sg, steps, copies, stream) / steps * 1e6
         d_in, d_out = WT.shape
@@ -695,7 +725,7 @@ def bench_batch(args, stream, sig, hbm_peak):
                 for j in range(B):
                     sig.sparse_gemv(Ws[c], Xd[j], t=t, y=ys[j], ws=wss[j], stream=stream)
             return g
-        sh = StepGraphs([h(c) for c in range(copies)], stream, per_graph=copies * 2)
+        sh = StepGraphs([h(c) for c in range(copies)], stream)
         us_sep = time_steps(sh, steps, copies, stream) / steps * 1e6
         out[f"B={B}"] = {"union_density": round(union / d_in, 4), "us": round(us, 2),
                          "GBps": round(b / (us * 1e-6) / 1e9, 1),
@@ -729,7 +759,7 @@ def bench_q8(args, stream, sig, hbm_peak):
             def g():
                 sig.sparse_gemv_q8(Qs[c], sd, xd, t, y=y, ws=ws, stream=stream)
             return g
-        sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies * 4)
+        sg = StepGraphs([f(c) for c in range(copies)], stream)
         steps = 400
         us = time_steps(sg, steps, copies, stream) / steps * 1e6
         nnz = int((np.abs(x.astype(np.float32)) >= t).sum())
@@ -744,7 +774,7 @@ def bench_q8(args, stream, sig, hbm_peak):
             def g():
                 sig.sparse_gemv(Ws[c], xd, t=t, y=y, ws=ws16, stream=stream)
             return g
-        sh = StepGraphs([h(c) for c in range(len(Ws))], stream, per_graph=len(Ws) * 4)
+        sh = StepGraphs([h(c) for c in range(len(Ws))], stream)
         us16 = time_steps(sh, steps, len(Ws), stream) / steps * 1e6
         out[f"{name} {d_in}->{d_out}"] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
                                           "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
@@ -774,7 +804,7 @@ def bench_nm(args, stream, sig, bf16_peak):
             def g():
                 sig.nm_act_gemm(Xs[c], Ws[c], n, m, Y=Y, ws=ws, stream=stream)
             return g
-        sg = StepGraphs([f(c) for c in range(copies)], stream, per_graph=copies)
+        sg = StepGraphs([f(c) for c in range(copies)], stream)
         sec = time_steps(sg, steps, copies, stream)
         us = sec / steps * 1e6
         Xm = torch.empty_like(Xs[0])
@@ -783,7 +813,7 @@ def bench_nm(args, stream, sig, bf16_peak):
             def g():
                 sig.sparsify_nm(Xs[c], n, m, X_masked=Xm, want_bits=False, stream=stream)
             return g
-        sm = StepGraphs([mk(c) for c in range(copies)], stream, per_graph=copies)
+        sm = StepGraphs([mk(c) for c in range(copies)], stream)
         us_mask = time_steps(sm, steps, copies, stream) / steps * 1e6
         out[f"{n}:{m}"] = {"us": round(us, 2),
                            "TFLOPs_executed": round(flops_dense / (us * 1e-6) / 1e12, 1),
@@ -796,7 +826,7 @@ def bench_nm(args, stream, sig, bf16_peak):
         def g():
             torch.matmul(Xs[c], Ws[c], out=Yd)
         return g
-    sg = StepGraphs([d(c) for c in range(copies)], stream, per_graph=copies)
+    sg = StepGraphs([d(c) for c in range(copies)], stream)
     sec = time_steps(sg, steps, copies, stream)
     us = sec / steps * 1e6
     out["cublas_dense"] = {"us": round(us, 2), "TFLOPs": round(flops_dense / (us * 1e-6) / 1e12, 1)}
@@ -814,79 +844,127 @@ def bench_nm(args, stream, sig, bf16_peak):
                 sig.nm_act_gemm_ex(Xs[c], Ws[c], 2, 4, shift=shifts[c % 2] if use_shift else None,
                                    col_sums=csum if use_shift else None, Y=Y, ws=ws, stream=stream, **kw)
             return g
-        sv = StepGraphs([fv(c) for c in range(copies)], stream, per_graph=copies)
+        sv = StepGraphs([fv(c) for c in range(copies)], stream)
         usv = time_steps(sv, steps, copies, stream) / steps * 1e6
         out[label] = {"us": round(usv, 2), "TFLOPs_executed": round(flops_dense / (usv * 1e-6) / 1e12, 1)}
     out["tensor_peak_tflops"] = bf16_peak
     return out
 
 
-def e2e(args, groups, copies, gys, gws, stream, sig, world, bytes_step):
-    """Public binding calls with host buffers: every step copies the layer's
+def e2e(args, groups, copies, gws, stream, sig, world, bytes_step):
+    """Public binding calls with host buffers.  Every step copies the layer's
     inputs in from pinned host memory (the four x vectors, one buffer, one
-    copy), runs the four launches through the binding, and copies the seven
-    y vectors (views of one device buffer) out to pinned host memory in one
-    copy.  Timed two ways: the step captured once per weight copy into a CUDA
-    graph and replayed (how a decoding loop runs it), and the same calls issued
-    eagerly from Python."""
+    copy), runs the four launches through the binding, and copies the seven y
+    vectors (views of one device buffer) out to pinned host memory in one
+    copy.  The copies run on their own streams with two buffers each way, so
+    that step i+1's input copy and step i-1's output copy overlap step i's
+    launches, as a serving loop would run them.  Timed two ways: the steps
+    captured into CUDA graphs and replayed (how a decoding loop runs them),
+    and the same calls issued eagerly from Python."""
     import torch
     d_ins = [g[0].d_in for g in groups]
     d_outs = [[p.d_out for p in g] for g in groups]
     xh = torch.from_numpy(np.concatenate([g[0].x for g in groups])).pin_memory()
-    xd_all = torch.empty(sum(d_ins), dtype=torch.float16, device="cuda")
-    yd_all = torch.empty(sum(sum(d) for d in d_outs), dtype=torch.float16, device="cuda")
-    yh = torch.empty_like(yd_all, device="cpu").pin_memory()
-    xd, ys, o = [], [], 0
-    for gi, di in enumerate(d_ins):
-        xd.append(xd_all[o:o + di])
-        o += di
-    o = 0
-    for gi, ds in enumerate(d_outs):
-        ys.append([])
-        for dj in ds:
-            ys[gi].append(yd_all[o:o + dj])
-            o += dj
+    nx, ny = sum(d_ins), sum(sum(d) for d in d_outs)
+    xd_all = [torch.empty(nx, dtype=torch.float16, device="cuda") for _ in range(2)]
+    yd_all = [torch.empty(ny, dtype=torch.float16, device="cuda") for _ in range(2)]
+    yh = [torch.empty(ny, dtype=torch.float16).pin_memory() for _ in range(2)]
+    xd, ys = [], []
+    for b in range(2):
+        xs, o = [], 0
+        for di in d_ins:
+            xs.append(xd_all[b][o:o + di])
+            o += di
+        yb, o = [], 0
+        for ds in d_outs:
+            yb.append([])
+            for dj in ds:
+                yb[-1].append(yd_all[b][o:o + dj])
+                o += dj
+        xd.append(xs)
+        ys.append(yb)
+    cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def step(c):
-        xd_all.copy_(xh, non_blocking=True)
-        for gi, g in enumerate(groups):
-            launch_group(sig, copies[c][gi], xd[gi], g[0].thresholds[HEADLINE_SPARSITY], ys[gi],
-                         gws[gi], stream)
-        yh.copy_(yd_all, non_blocking=True)
+    def steps(n, c0):
+        """Enqueue n pipelined steps; returns after `stream` has joined both copy streams."""
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        cs_in.wait_event(fork)
+        cs_out.wait_event(fork)
+        comp, out = [None, None], [None, None]
+        for i in range(n):
+            b, c = i % 2, (c0 + i) % len(copies)
+            with torch.cuda.stream(cs_in):
+                if comp[b] is not None:        # step i-2 has finished reading x[b]
+                    cs_in.wait_event(comp[b])
+                xd_all[b].copy_(xh, non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(cs_in)
+            stream.wait_event(ev_in)
+            if out[b] is not None:             # step i-2's y[b] has been copied out
+                stream.wait_event(out[b])
+            for gi, g in enumerate(groups):
+                launch_group(sig, copies[c][gi], xd[b][gi], g[0].thresholds[HEADLINE_SPARSITY],
+                             ys[b][gi], gws[gi], stream)
+            comp[b] = torch.cuda.Event()
+            comp[b].record(stream)
+            with torch.cuda.stream(cs_out):
+                cs_out.wait_event(comp[b])
+                yh[b].copy_(yd_all[b], non_blocking=True)
+                out[b] = torch.cuda.Event()
+                out[b].record(cs_out)
+        join = torch.cuda.Event()
+        join.record(cs_in)
+        stream.wait_event(join)
+        for e in out:
+            if e is not None:
+                stream.wait_event(e)
 
-    def timed(n, run):
+    n_steps = max(200, min(args.steps, 1200))
+    per = 600 if n_steps > 600 else n_steps
+    chunks = [per] * (n_steps // per) + ([n_steps % per] if n_steps % per else [])
+    with torch.cuda.stream(stream):
+        steps(2 * len(copies), 0)             # eager warm-up
+    torch.cuda.synchronize()
+    graphs = {n: capture(lambda n=n: steps(n, 0), stream) for n in set(chunks)}
+
+    def timed(run):
         torch.cuda.synchronize()
         barrier(world)
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _queue_delay(stream)
         with torch.cuda.stream(stream):
             s.record(stream)
-            for i in range(n):
-                run(i)
+            run()
             e.record(stream)
         torch.cuda.synchronize()
         return max_over_ranks(s.elapsed_time(e) / 1e3, world)
 
-    with torch.cuda.stream(stream):
-        for i in range(2 * len(copies)):
-            step(i % len(copies))
-    graphs = [capture(lambda c=c: step(c), stream) for c in range(len(copies))]
-    steps = max(10, min(args.steps // 4, 5000))
-    timed(24, lambda i: graphs[i % len(graphs)].replay())          # warm-up
-    sec = timed(steps, lambda i: graphs[i % len(graphs)].replay())
-    steps_e = max(10, min(args.steps // 20, 1000))
-    sec_e = timed(steps_e, lambda i: step(i % len(copies)))
+    def replay_all():
+        for n in chunks:
+            graphs[n].replay()
+
+    timed(replay_all)                                                 # warm-up
+    sec = timed(replay_all)
+    n_eager = max(50, min(args.steps, 400))
+
+    def eager():
+        steps(n_eager, 0)
+    timed(eager)                                                      # warm-up
+    sec_e = timed(eager)
     del graphs
-    return {"value": round(bytes_step * steps * world / sec / 1e9, 1), "unit": UNIT,
-            "steps": steps, "us_per_step": round(sec / steps * 1e6, 2),
-            "h2d_bytes_per_step": 2 * sum(d_ins),
-            "d2h_bytes_per_step": 2 * sum(sum(d) for d in d_outs),
-            "eager_value": round(bytes_step * steps_e * world / sec_e / 1e9, 1),
-            "eager_us_per_step": round(sec_e / steps_e * 1e6, 2),
+    return {"value": round(bytes_step * n_steps * world / sec / 1e9, 1), "unit": UNIT,
+            "steps": n_steps, "us_per_step": round(sec / n_steps * 1e6, 2),
+            "h2d_bytes_per_step": 2 * nx, "d2h_bytes_per_step": 2 * ny,
+            "eager_value": round(bytes_step * n_eager * world / sec_e / 1e9, 1),
+            "eager_steps": n_eager, "eager_us_per_step": round(sec_e / n_eager * 1e6, 2),
             "note": "weights resident (model parameters, the same rotating copies as the device "
                     "timing); every step copies the layer's four x vectors in from pinned host "
                     "memory (one copy) and its seven y vectors out to pinned host memory (one "
-                    "copy); value: the step's binding calls captured in a CUDA graph and replayed; "
-                    "eager_value: the same calls issued from Python"}
+                    "copy), on two copy streams with double buffers so the copies of steps i+1 "
+                    "and i-1 overlap step i's launches; value: the steps' binding calls captured "
+                    "in CUDA graphs and replayed; eager_value: the same calls issued from Python "
+                    "every step (host-bound: the binding's per-call cost is paid each step)"}
 
 
 # ---------------------------------------------------------------------------
@@ -900,6 +978,23 @@ def _blas_threads():
         return int(max(n)) if n else os.cpu_count()
     except Exception:
         return os.cpu_count()
+
+
+def cpu_model():
+    """The host CPU's model name and logical core count (as nproc reports)."""
+    name = None
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.lower().startswith("model name"):
+                name = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except AttributeError:
+        nproc = os.cpu_count()
+    return name or "unknown", nproc
 
 
 def oracle_sample(groups, cols_per_proj, rng):
@@ -917,8 +1012,7 @@ def oracle_sample(groups, cols_per_proj, rng):
     return b, time.perf_counter() - t0
 
 
-def cpu_baseline(groups, budget_s=12.0):
-    rng = np.random.default_rng(0)
+def _timed_oracle(groups, budget_s, rng):
     _, t1 = oracle_sample(groups, 256, rng)                      # warm-up and calibration
     reps = max(1, int(budget_s / max(t1, 1e-3)))
     tot_b, tot_t = 0, 0.0
@@ -926,10 +1020,26 @@ def cpu_baseline(groups, budget_s=12.0):
         b, t = oracle_sample(groups, 256, rng)
         tot_b += b
         tot_t += t
-    return {"value": round(tot_b / tot_t / 1e9, 3), "unit": UNIT, "cores": _blas_threads(),
-            "kind": "oracle",
+    return tot_b / tot_t / 1e9, reps, tot_t
+
+
+def cpu_baseline(groups, budget_s=8.0):
+    """The oracle as it stands on the host cores: once with the BLAS thread
+    pool at its default (all cores) and once limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    rng = np.random.default_rng(0)
+    name, nproc = cpu_model()
+    threads = _blas_threads()
+    v_all, reps, tot = _timed_oracle(groups, budget_s, rng)
+    with threadpool_limits(limits=1, user_api="blas"):
+        v_one, reps1, tot1 = _timed_oracle(groups, budget_s, rng)
+    return {"value": round(v_all, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "cpu_model": name, "nproc": nproc,
+            "single_thread": {"value": round(v_one, 4), "cores": 1,
+                              "sample": f"{reps1} passes ({tot1:.1f} s)"},
             "sample": f"{reps} passes over the 7 projections, 256 random output columns each, "
-                      f"one 50% threshold mask per shared input, numpy float64 ({tot_t:.1f} s)"}
+                      f"one 50% threshold mask per shared input, numpy float64 ({tot:.1f} s, "
+                      f"BLAS on {threads} threads); single_thread: the same with one BLAS thread"}
 
 
 def run_reference(args, rank, world):
@@ -959,7 +1069,8 @@ def run_reference(args, rank, world):
             "config": {"workload": "llama2_7b_decode_layer_b1", "batch": 1,
                        "sparsity": HEADLINE_SPARSITY, "seed": args.seed, "parallelism": "cpu"},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": _blas_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample, "cpu_model": cpu_model()[0],
+                             "nproc": cpu_model()[1]},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "gpu_launches": 0}

@@ -418,7 +418,11 @@ SIG_API int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16
  *     GPU (other streams, other host threads) race; serialise them.
  *   - The first call on each device, with that device current, looks up the
  *     array's device address (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  The cached address belongs to
+ *     the device's primary context as it was then: cudaDeviceReset (or
+ *     anything else that destroys that context) leaves it stale, so do not
+ *     call this entry point on a device after resetting it in the same
+ *     process.
  * Errors: as gated_mlp_sparse, except SIG_ERR_WORKSPACE (none is taken).
  */
 #define SIG_NOALLOC_SCRATCH_BYTES (2u << 20)

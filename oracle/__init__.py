@@ -43,7 +43,8 @@ Sources, cited by page title and section:
 Readings where the pages are silent or disagree (each one is a choice):
 
 * Threshold comparison is ``|x_i| >= t`` ([RaNA] Eqn. 12 writes ``>= t``; TEAL
-  gives no operator).  A NaN is never kept by a threshold.
+  gives no operator), with t a float32 value.  A NaN is never kept by a
+  threshold.
 * Ranking by magnitude (top-k, N:M): larger |x| first, equal |x| by lower index
   first; +v and -v tie, +0 and -0 tie; a NaN ranks below every number.
 * N:M keeps the N largest of each M consecutive elements ([NM] Methodology;
@@ -121,8 +122,11 @@ def magnitude_order(x) -> np.ndarray:
 
 
 def threshold_mask(x, t: float) -> np.ndarray:
-    """[TEAL] Abstract: keep x_i when |x_i| >= t (a NaN is never kept)."""
-    return np.abs(np.asarray(x, dtype=np.float64)) >= np.float64(t)
+    """[TEAL] Abstract: keep x_i when |x_i| >= t (a NaN is never kept).
+
+    The threshold is a float32 value (the layer takes it as one), so ``t`` is
+    rounded to float32 first; |x_i| of an fp16 input is exact in float64."""
+    return np.abs(np.asarray(x, dtype=np.float64)) >= np.float64(np.float32(t))
 
 
 def topk_mask(x, k: int) -> np.ndarray:

@@ -20,7 +20,10 @@
 // In host code the array's name is a host-side stand-in, not a device
 // address.  The first call on each device (with that device current) asks the
 // runtime for the array's device address and caches it; make that first call
-// before any stream capture.
+// before any stream capture.  The cache is keyed by device ordinal only: after
+// cudaDeviceReset the primary context (and the array's address in it) is new,
+// and the cached address is stale, so the header tells callers not to use
+// this entry point on a device after resetting it.
 #include "../../include/sig.h"
 #include "internal.h"
 

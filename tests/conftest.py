@@ -75,3 +75,30 @@ def assert_within(y16, y64, bound, what=""):
         raise AssertionError(f"{what}: {bad.size}/{y.size} outputs out of tolerance; "
                              f"worst j={j} y={y[j]} ref={y64[j]} bound={bound[j]}")
     assert np.isfinite(y).all()
+
+
+def fp32_sum_bound(n_terms, abs_sum):
+    """Worst-case error of a float32 sum of ``n_terms`` exactly representable
+    products, in any order: gamma_n * sum|terms| with gamma_n = n u / (1 - n u),
+    u = 2^-24 (every fp16 x fp16 product is exact in float32; only the n - 1
+    additions round)."""
+    import numpy as np
+    u = 2.0 ** -24
+    n = np.asarray(n_terms, dtype=np.float64)
+    return n * u / (1.0 - n * u) * np.asarray(abs_sum, dtype=np.float64)
+
+
+def silu_mul_tolerance(g, u, eg, eu, h_ref):
+    """How far the GPU's h = fp16(SiLU(g) u), computed in float32 from g and u
+    that carry errors of at most eg and eu, may sit from the oracle's h (float64
+    g, u, one fp16 rounding): the errors carried through h = SiLU(g) u by its
+    derivatives (dSiLU/dg = sigma(g) (1 + g (1 - sigma(g)))), eight float32
+    roundings of the SiLU and product evaluation, and one fp16 ulp for the
+    final rounding."""
+    import numpy as np
+    with np.errstate(over="ignore"):
+        sg = 1.0 / (1.0 + np.exp(-g))
+    dsilu = sg * (1.0 + g * (1.0 - sg))
+    h64 = g * sg * u
+    return (np.spacing(np.abs(h_ref)).astype(np.float64) + np.abs(dsilu * u) * eg
+            + np.abs(g * sg) * eu + 8 * 2.0 ** -24 * np.abs(h64))

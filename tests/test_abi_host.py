@@ -295,6 +295,29 @@ def test_noalloc_validation(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 0.1, FAKE, None, FAKE + 1, None) == ALIGN
 
 
+def test_noalloc_scratch_covers_every_accepted_shape(lib):
+    """Every (d_model, d_ff) that gated_mlp_sparse accepts (multiples of 8 up
+    to SIG_MAX_D_IN) fits the allocation-free entry point's 2 MiB scratch.
+
+    The gated MLP's workspace is the sum of a term that depends only on d_ff
+    (the gate/up product's counters and partials, and the hidden vector) and
+    one that depends only on d_model (the down product's): the maximum of the
+    sum is the sum of the two one-dimensional maxima.  The decomposition is
+    checked on a spread of pairs first, so that a change that couples the two
+    terms fails here instead of hiding an oversize shape."""
+    ws = lib.sig_workspace_bytes
+    OP_GATED_MLP, LIMIT, MAX_D = 3, 2 << 20, 131072
+    sizes = range(8, MAX_D + 1, 8)
+    base = ws(OP_GATED_MLP, 8, 8, 0)
+    f = {d: ws(OP_GATED_MLP, 8, d, 0) - base for d in sizes}      # d_ff term
+    g = {d: ws(OP_GATED_MLP, d, 8, 0) - base for d in sizes}      # d_model term
+    for dm in (8, 1024, 4096, 8192, 11008, 28672, 75776, MAX_D):
+        for dff in (8, 4096, 11008, 28672, 75776, 75784, MAX_D):
+            assert ws(OP_GATED_MLP, dm, dff, 0) == base + f[dff] + g[dm], (dm, dff)
+    worst = base + max(f.values()) + max(g.values())
+    assert worst <= LIMIT, worst
+
+
 def test_32bit_buffers_must_be_4_byte_aligned(lib):
     """Masks, index lists, counts and float vectors are checked on the host,
     like the 16-byte rules, before anything is enqueued."""

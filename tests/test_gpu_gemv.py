@@ -42,6 +42,18 @@ def test_ragged_shapes(sig, d_in, d_out):
         _check_threshold(sig, p.WT, p.x, t, f"{d_in}x{d_out} s={s}")
 
 
+def test_threshold_between_fp16_values_and_not_a_float32(sig):
+    """t reaches the library as a float32: 0.5 + 1e-12 arrives as 0.5 (|x| =
+    0.5 kept), 0.5002 as a float32 between two fp16 values (0.5 dropped,
+    0.50048828125 kept).  The oracle rounds t to float32 the same way."""
+    rng = np.random.default_rng(21)
+    WT = workloads.draw_weight(rng, 1000, 264, 0.02)
+    x = rng.choice([0.5, -0.5, 0.49975586, 0.50048828125, -0.50048828125, 1.0, 0.0],
+                   size=1000).astype(np.float16)
+    for t in (0.5 + 1e-12, 0.5002, 0.50048828125 - 1e-9):
+        _check_threshold(sig, WT, x, t, f"t={t!r}")
+
+
 def test_empty_and_full_masks(sig):
     p = workloads.projection("e", 300, 136, sigma=0.02, dist="laplace", seed=5)
     y, ref = _check_threshold(sig, p.WT, p.x, float("inf"), "empty mask")

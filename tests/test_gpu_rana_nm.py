@@ -4,7 +4,8 @@ import pytest
 
 import oracle
 import workloads
-from tests.conftest import assert_within, mask_words, to_dev, to_host
+from tests.conftest import (assert_within, fp32_sum_bound, mask_words, silu_mul_tolerance,
+                            to_dev, to_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -41,20 +42,17 @@ def _rana_case(sig, mlp, t, what):
     ref = oracle.sparse_linear(mlp.WdT, h, m_strict)
     assert_within(y, ref["y64"], ref["bound"], what + " strict")
 
-    # end to end against the oracle's own h.  g and u are float32 sums on the
-    # GPU: give each the product tolerance 2e-3 * sum|W x| and carry it through
-    # h = SiLU(g) u (dSiLU/dg = sigma(g) (1 + g (1 - sigma(g)))), plus one fp16
-    # ulp for the final rounding.
+    # end to end against the oracle's own h.  g and u are float32 sums of
+    # d_model exact products on the GPU: each carries at most the float32
+    # summation bound gamma_d * sum|W x|, which h = SiLU(g) u carries on
+    # (conftest.silu_mul_tolerance).
     full = oracle.gated_mlp(mlp.x, mlp.WgT, mlp.WuT, mlp.WdT, norms, t)
     h_ref, g, u = full["h16"], full["g"], full["u"]
     x64 = np.abs(mlp.x.astype(np.float64))
-    Bg = x64 @ np.abs(mlp.WgT.astype(np.float64))
-    Bu = x64 @ np.abs(mlp.WuT.astype(np.float64))
-    with np.errstate(over="ignore"):
-        sg = 1.0 / (1.0 + np.exp(-g))
-    dsilu = sg * (1.0 + g * (1.0 - sg))
-    tol_h = (np.spacing(np.abs(h_ref)).astype(np.float64)
-             + np.abs(dsilu * u) * 2e-3 * Bg + np.abs(g * sg) * 2e-3 * Bu)
+    n_terms = int(np.count_nonzero(mlp.x))
+    eg = fp32_sum_bound(n_terms, x64 @ np.abs(mlp.WgT.astype(np.float64)))
+    eu = fp32_sum_bound(n_terms, x64 @ np.abs(mlp.WuT.astype(np.float64)))
+    tol_h = silu_mul_tolerance(g, u, eg, eu, h_ref)
     dh = np.abs(h.astype(np.float64) - h_ref.astype(np.float64))
     assert (dh <= tol_h).all(), (what + " h", int((dh > tol_h).sum()))
     assert (dh <= np.spacing(np.abs(h_ref))).mean() > 0.999, what + " h mostly within 1 ulp"

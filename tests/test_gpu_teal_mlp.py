@@ -4,14 +4,15 @@ launch with the SiLU(g) u epilogue), |h_i| >= t_h for down.
 
 Checked like the RaNA masker: strictly (the h mask follows bit for bit from
 the GPU's own h, and y is within tolerance of the product on that mask) and
-end to end against the oracle's own h (g and u carry the product tolerance
-through h = SiLU(g) u; masks may differ only where |h| is that close to t_h)."""
+end to end against the oracle's own h (g and u carry the float32 summation
+bound through h = SiLU(g) u; masks may differ only where |h| is that close to t_h)."""
 import numpy as np
 import pytest
 
 import oracle
 import workloads
-from tests.conftest import assert_within, mask_words, to_dev, to_host
+from tests.conftest import (assert_within, fp32_sum_bound, mask_words, silu_mul_tolerance,
+                            to_dev, to_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -32,14 +33,12 @@ def _case(sig, mlp, x, t_x, t_h, what):
 
     full = oracle.teal_mlp(x, mlp.WgT, mlp.WuT, mlp.WdT, t_x, t_h)
     h_ref, g, u = full["h16"], full["g"], full["u"]
+    # g and u: float32 sums of the kept products (conftest.fp32_sum_bound)
     xm = np.where(full["mask_x"], np.abs(x.astype(np.float64)), 0.0)
-    Bg = xm @ np.abs(mlp.WgT.astype(np.float64))
-    Bu = xm @ np.abs(mlp.WuT.astype(np.float64))
-    with np.errstate(over="ignore"):
-        sg = 1.0 / (1.0 + np.exp(-g))
-    dsilu = sg * (1.0 + g * (1.0 - sg))
-    tol_h = (np.spacing(np.abs(h_ref)).astype(np.float64)
-             + np.abs(dsilu * u) * 2e-3 * Bg + np.abs(g * sg) * 2e-3 * Bu)
+    n_terms = int(np.count_nonzero(xm))
+    eg = fp32_sum_bound(n_terms, xm @ np.abs(mlp.WgT.astype(np.float64)))
+    eu = fp32_sum_bound(n_terms, xm @ np.abs(mlp.WuT.astype(np.float64)))
+    tol_h = silu_mul_tolerance(g, u, eg, eu, h_ref)
     dh = np.abs(h.astype(np.float64) - h_ref.astype(np.float64))
     assert (dh <= tol_h).all(), (what + " h", int((dh > tol_h).sum()))
     diff = np.flatnonzero(m_gpu != full["mask"])

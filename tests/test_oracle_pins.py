@@ -119,6 +119,16 @@ def test_threshold_matches_brute_force_loop_and_sorted_count():
         assert int(m.sum()) >= x.size - math.floor(s * x.size)
 
 
+def test_threshold_is_a_float32_value():
+    """The threshold is compared as the float32 value the layer receives: a t
+    within half a float32 ulp above 0.5 is 0.5 (so |x| = 0.5 is kept), while
+    0.5002 stays above 0.5 and below the next fp16 value 0.50048828125."""
+    x = np.array([0.5, -0.5, 0.49975586, 0.50048828125], dtype=np.float16)
+    assert list(oracle.threshold_mask(x, 0.5 + 1e-12)) == [True, True, False, True]
+    assert list(oracle.threshold_mask(x, 0.5002)) == [False, False, False, True]
+    assert np.float32(0.5 + 1e-12) == np.float32(0.5) and 0.5 + 1e-12 > 0.5
+
+
 def test_threshold_never_keeps_nan_and_keeps_inf():
     x = np.array([np.nan, np.inf, -np.inf, 1.0], dtype=np.float16)
     assert oracle.threshold_mask(x, 0.0).tolist() == [False, True, True, True]

@@ -6,9 +6,11 @@ memory budget fixed at start-up, C code without an allocator).  This file is
 named so that pytest collects it last.
 
 The test calls it through the C ABI twice in a row and checks each output
-against the existing gated_mlp_sparse on the same inputs, with the tolerance
-the other parity tests use.  Both calls run on the same stream, so the second
-call finds the first call's contents in the shared scratch array.
+against the existing gated_mlp_sparse on the same inputs.  The two entry
+points run the same kernels with the same launch plan and split-K order, so y
+must be bit-identical (which implies the tolerance the other parity tests
+use).  Both calls run on the same stream, so the second call finds the first
+call's contents in the shared scratch array.
 """
 import numpy as np
 import pytest
@@ -51,10 +53,12 @@ def test_noalloc_matches_gated_mlp_twice_in_a_row(sig):
         y = to_host(sig.gated_mlp_sparse_noalloc(dx, dg, du, dd, norms, t, h_out=h, mask_out=m))
         assert np.array_equal(to_host(h).view(np.uint16), h_host.view(np.uint16)), call
         assert np.array_equal(mask_words(m), mw), call
+        assert np.array_equal(y.view(np.uint16), y_ref.view(np.uint16)), call
         assert_within(y, y_ref.astype(np.float64), bound, f"no-alloc call {call}")
 
     # without h_out / mask_out the hidden vector stays in the library's array
     y3 = to_host(sig.gated_mlp_sparse_noalloc(dx, dg, du, dd, norms, t))
+    assert np.array_equal(y3.view(np.uint16), y_ref.view(np.uint16))
     assert_within(y3, y_ref.astype(np.float64), bound, "no-alloc without h_out")
     torch.cuda.synchronize()
 
