@@ -62,7 +62,8 @@ def parse():
                     help="for ncu: run only this kernel case eagerly and exit "
                          "(a Llama-2-7B projection name or launch group such as 'q|k|v' or "
                          "'gate|up' at 50%%, 'topk70b', 'batchB' (B tokens, 4096->11008), "
-                         "'q8up70b', 'nm2:4' or 'nmex2:4')")
+                         "'q8up70b', 'nm2:4', 'nmsp2:4' (packed 2:4 operand, sparse GEMM) or "
+                         "'nmex2:4')")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     args = ap.parse_args()
     # at least three untimed warm-up steps; the JSON line reports the number run
@@ -196,7 +197,7 @@ class StepGraphs:
     by step count.
     """
 
-    def __init__(self, fns, stream):
+    def __init__(self, fns, stream, cap=600):
         import torch
         self.fns, self.R, self.stream = fns, len(fns), stream
         self.cap = max(self.R, (cap // self.R) * self.R)
@@ -815,11 +816,41 @@ def bench_nm(args, stream, sig, bf16_peak):
             return g
         sm = StepGraphs([mk(c) for c in range(copies)], stream)
         us_mask = time_steps(sm, steps, copies, stream) / steps * 1e6
-        out[f"{n}:{m}"] = {"us": round(us, 2),
-                           "TFLOPs_executed": round(flops_dense / (us * 1e-6) / 1e12, 1),
-                           "TFLOPs_algorithmic": round(flops_dense * n / m / (us * 1e-6) / 1e12, 1),
-                           "mask_only_us": round(us_mask, 2),
-                           "mask_GBps": round(2 * X.nbytes / (us_mask * 1e-6) / 1e9, 1)}
+        row = {"us": round(us, 2),
+               "TFLOPs_executed": round(flops_dense / (us * 1e-6) / 1e12, 1),
+               "TFLOPs_algorithmic": round(flops_dense * n / m / (us * 1e-6) / 1e12, 1),
+               "mask_only_us": round(us_mask, 2),
+               "mask_GBps": round(2 * X.nbytes / (us_mask * 1e-6) / 1e9, 1)}
+        if m == 4 and n <= 2:
+            # the sparse tensor-core path: pack, then the 2:4 GEMM on the packed operand
+            row["path"] = "packed 2:4 operand, tcgen05.mma.sp"
+            row["TFLOPs_executed"] = round(flops_dense / 2 / (us * 1e-6) / 1e12, 1)
+            row["TFLOPs_dense_equivalent"] = round(flops_dense / (us * 1e-6) / 1e12, 1)
+            pk = [sig.sparsify_nm_packed(Xs[c], n) for c in range(2)]
+
+            def fp(c, n=n):
+                def g():
+                    sig.sparsify_nm_packed(Xs[c], n, out=pk[c % 2], stream=stream)
+                return g
+
+            def fg(c):
+                def g():
+                    sig.nm_act_gemm_packed(pk[c % 2], rows, K, Ws[c], Y=Y, stream=stream)
+                return g
+            sp = StepGraphs([fp(c) for c in range(copies)], stream)
+            us_pack = time_steps(sp, steps, copies, stream) / steps * 1e6
+            sgm = StepGraphs([fg(c) for c in range(copies)], stream)
+            us_gemm = time_steps(sgm, steps, copies, stream) / steps * 1e6
+            pbytes = X.nbytes + sig.nm_packed_bytes(rows, K)
+            row.update({"pack_only_us": round(us_pack, 2),
+                        "pack_GBps": round(pbytes / (us_pack * 1e-6) / 1e9, 1),
+                        "sparse_gemm_only_us": round(us_gemm, 2),
+                        "sparse_gemm_TFLOPs_dense_equivalent":
+                            round(flops_dense / (us_gemm * 1e-6) / 1e12, 1)})
+            del pk, sp, sgm
+        else:
+            row["path"] = "masked X, dense tcgen05.mma"
+        out[f"{n}:{m}"] = row
     Yd = torch.empty_like(Y)
 
     def d(c):
@@ -949,7 +980,14 @@ def e2e(args, groups, copies, gws, stream, sig, world, bytes_step):
     n_eager = max(50, min(args.steps, 400))
 
     def eager():
-        steps(n_eager, 0)
+        # one stream, in order: copy in, the four binding calls, copy out
+        for i in range(n_eager):
+            b, c = i % 2, i % len(copies)
+            xd_all[b].copy_(xh, non_blocking=True)
+            for gi, g in enumerate(groups):
+                launch_group(sig, copies[c][gi], xd[b][gi], g[0].thresholds[HEADLINE_SPARSITY],
+                             ys[b][gi], gws[gi], stream)
+            yh[b].copy_(yd_all[b], non_blocking=True)
     timed(eager)                                                      # warm-up
     sec_e = timed(eager)
     del graphs
@@ -963,8 +1001,9 @@ def e2e(args, groups, copies, gws, stream, sig, world, bytes_step):
                     "memory (one copy) and its seven y vectors out to pinned host memory (one "
                     "copy), on two copy streams with double buffers so the copies of steps i+1 "
                     "and i-1 overlap step i's launches; value: the steps' binding calls captured "
-                    "in CUDA graphs and replayed; eager_value: the same calls issued from Python "
-                    "every step (host-bound: the binding's per-call cost is paid each step)"}
+                    "in CUDA graphs and replayed; eager_value: the same calls and copies issued "
+                    "from Python every step on one stream, in order (the binding's per-call host "
+                    "cost is paid each step)"}
 
 
 # ---------------------------------------------------------------------------
@@ -1128,6 +1167,17 @@ def profile_case(args):
         norms = sig.row_norms(Wd)
         for _ in range(args.launches):
             sig.sparsify_nm_ex(Xd, 2, 4, shift=shift, norms=norms, var=True, want_bits=False)
+        info = {"case": case, "launches": args.launches}
+    elif case in ("nmsp2:4", "nmsp1:4"):
+        WT, X = workloads.nm_tokens(args.seed)
+        n = int(case[4])
+        copies = 8
+        Xs = [torch.from_numpy(X).cuda() for _ in range(copies)]
+        Wd = torch.from_numpy(WT).cuda()
+        pk = [sig.sparsify_nm_packed(x, n) for x in Xs]
+        for i in range(args.launches):
+            sig.sparsify_nm_packed(Xs[i % copies], n, out=pk[i % copies])
+            sig.nm_act_gemm_packed(pk[i % copies], X.shape[0], X.shape[1], Wd)
         info = {"case": case, "launches": args.launches}
     elif case == "nm2:4":
         WT, X = workloads.nm_tokens(args.seed)

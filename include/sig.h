@@ -153,13 +153,37 @@ SIG_API int sparsify_topk(const uint16_t* x, int64_t d, int64_t k,
  *   X_masked   [rows x d] fp16 out, 16-byte aligned, nullable: X with dropped
  *              entries set to +0.
  *   mask_bits  [rows x ceil(d/32)] uint32 out, nullable.
- * At least one of X_masked and mask_bits must be non-NULL.  rows == 0 is an
- * empty batch: the call returns SIG_OK and touches no pointer.
+ *   packed     sig_nm_packed_bytes(rows, d) bytes out, 16-byte aligned,
+ *              nullable: the 2:4 operand of the sparse tensor cores, for
+ *              nm_act_gemm_packed.  Only for 2:4 and 1:4 (n:m = 2:4 or 1:4,
+ *              else SIG_ERR_ARG), rows % 128 == 0 and d % 128 == 0 (else
+ *              SIG_ERR_SHAPE).  1:4 is padded to 2:4: the block's second slot
+ *              holds +0 at the smallest position that is not kept.  Layout:
+ *                values  [rows x d/2] fp16 at byte 0: for row r and block b
+ *                        (entries 4b .. 4b+3), the two slots in ascending
+ *                        position order at [r, 2b] and [r, 2b+1];
+ *                meta    rows*d/8 bytes at byte rows*d: one 2048-byte tile per
+ *                        128 x 128 block (row block R, column block C; tile
+ *                        R * (d/128) + C).  Byte 16 L + 4 j + 2 s + i of a tile
+ *                        (lane L < 128, group j < 4, s and i < 2) holds the
+ *                        blocks of row r = 128 R + L % 8 + 8 s + 16 (L / 16),
+ *                        entries 128 C + 32 j + 16 ((L / 8) % 2) + 8 i + 4 k
+ *                        for k = 0 (low nibble) and k = 1 (high nibble); a
+ *                        block's nibble is p0 | p1 << 2, p0 < p1 the positions
+ *                        of its two slots.  This is the order in which a
+ *                        128x128b tensor-memory copy hands a 128 x 128 block of
+ *                        metadata to the sparse MMA.
+ * At least one of X_masked, mask_bits and packed must be non-NULL.  rows == 0
+ * is an empty batch: the call returns SIG_OK and touches no pointer.
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (rows < 0, d < 1, d % m), SIG_ERR_ARG (n, m),
  *         SIG_ERR_ALIGN.
  */
 SIG_API int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m,
-                uint16_t* X_masked, uint32_t* mask_bits, sig_stream_t stream);
+                uint16_t* X_masked, uint32_t* mask_bits, void* packed, sig_stream_t stream);
+
+/* Bytes of sparsify_nm's packed output (rows*d*9/8), or 0 when rows or d is
+ * not a positive multiple of 128. */
+SIG_API size_t sig_nm_packed_bytes(int64_t rows, int64_t d);
 
 /*
  * Sparse-input GEMV y = W (m . x) (RaNA rebuttal, Q5.1; Q-Sparse A3):
@@ -382,19 +406,36 @@ SIG_API int sig_row_norms(const uint16_t* WT, int64_t rows, int64_t cols, float*
  * Batched N:M activation GEMM (Block Q-Sparse, Q-Sparse rebuttal A2):
  *   Y = (M . X) WT, M the per-row n:m mask of X (as sparsify_nm), float32
  *   accumulation on the tensor cores, Y rounded once to fp16.  When n == m
- *   the GEMM runs on X directly.
+ *   the GEMM runs on X directly.  For 2:4 and 1:4 with K % 128 == 0, X is
+ *   packed (as sparsify_nm's packed output) and the product runs on the
+ *   sparse tensor cores (as nm_act_gemm_packed); other patterns run the dense
+ *   tensor cores on the masked X.
  *   X  [rows x K] fp16 row-major.   WT [K x N] fp16 row-major.   Y [rows x N] fp16 out.
  *   All three 16-byte aligned (WT and X are read by TMA).
  *   rows % 128 == 0, K % 64 == 0, N % 128 == 0, rows <= 2^24, K and N <= 2^20;
  *   m in {1,2,4,8,16,32}, 1 <= n <= m, K % m == 0.
- *   ws sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows) bytes (the masked X;
- *      not touched when n == m, so it may be NULL then).
+ *   ws sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows) bytes (the masked or
+ *      packed X; not touched when n == m, so it may be NULL then).
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ARG, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE,
  *         SIG_ERR_CUDA.
  */
 SIG_API int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT,
                 int64_t N, int n, int m, uint16_t* Y, void* ws, size_t ws_bytes,
                 sig_stream_t stream);
+
+/*
+ * The product of nm_act_gemm on an operand that sparsify_nm has already
+ * packed (2:4, or 1:4 padded to 2:4): Y = A WT, A the rows x K activation
+ * block the packed values and metadata describe, on the sparse tensor cores
+ * (tcgen05.mma.sp, kind::f16: half the A bytes, each MMA covers 32 logical K).
+ * Float32 accumulation, Y rounded once to fp16.
+ *   packed  sig_nm_packed_bytes(rows, K) bytes, 16-byte aligned (the layout
+ *           of sparsify_nm).   WT [K x N] fp16.   Y [rows x N] fp16 out.
+ *   rows % 128 == 0, K % 128 == 0, N % 128 == 0, rows <= 2^24, K and N <= 2^20.
+ * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ALIGN, SIG_ERR_CUDA.
+ */
+SIG_API int nm_act_gemm_packed(const void* packed, int64_t rows, int64_t K, const uint16_t* WT,
+                               int64_t N, uint16_t* Y, sig_stream_t stream);
 
 /*
  * gated_mlp_sparse without a workspace argument, for callers that cannot

@@ -87,6 +87,7 @@ __all__ = [
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
     "union_mask", "batched_sparse_linear", "q8_sparse_linear", "teal_mlp",
     "pts_shift", "wt_scores", "nm_mask_by_score", "var_gamma", "nm_variant", "nm_variant_gemm",
+    "nm_pack_2of4",
 ]
 
 
@@ -196,6 +197,33 @@ def flops(d_out: int, nnz: int) -> int:
     """[QS] A3: a d_out x d_in by d_in x 1 product costs 2 d_out d_in; with
     only nnz inputs kept it costs 2 d_out nnz (mask cost left out)."""
     return 2 * int(d_out) * int(nnz)
+
+
+def nm_pack_2of4(X, n: int) -> dict:
+    """The 2:4 operand of an N:M mask with M = 4 ([NM] Hardware implications:
+    2:4 is the pattern the hardware supports; [NM] Methodology / [QS] A2 for
+    the mask).  Per row and block of four entries: the kept entries of
+    :func:`nm_mask` (n = 2), or the kept entry plus a padding slot at the
+    block's smallest position that is not kept, holding +0 (n = 1, 1:4
+    padded to 2:4), both slots in ascending position order.  Returns fp16
+    ``values`` and uint8 ``positions`` (0..3 within the block), each of shape
+    (rows, d/2), and the ``mask``."""
+    X = np.asarray(X, dtype=np.float16)
+    X2 = X.reshape(1, -1) if X.ndim == 1 else X
+    if n not in (1, 2):
+        raise ValueError("the 2:4 operand packs 2:4 or 1:4")
+    rows, d = X2.shape
+    mask = nm_mask(X2, n, 4)
+    values = np.zeros((rows, d // 2), dtype=np.float16)
+    positions = np.zeros((rows, d // 2), dtype=np.uint8)
+    for r in range(rows):
+        for b in range(d // 4):
+            kept = [j for j in range(4) if mask[r, 4 * b + j]]
+            slots = kept if n == 2 else sorted(kept + [min(j for j in range(4) if j not in kept)])
+            for s, j in enumerate(slots):
+                positions[r, 2 * b + s] = j
+                values[r, 2 * b + s] = X2[r, 4 * b + j] if j in kept else np.float16(0.0)
+    return {"values": values, "positions": positions, "mask": mask}
 
 
 # ---------------------------------------------------------------------------

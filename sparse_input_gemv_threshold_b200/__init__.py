@@ -25,6 +25,7 @@ __all__ = [
     "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
     "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch", "OP_SPARSE_GEMV_Q8",
     "sparse_gemv_q8", "sparsify_nm_ex", "nm_act_gemm_ex", "col_sums", "teal_mlp_sparse",
+    "nm_packed_bytes", "sparsify_nm_packed", "nm_act_gemm_packed",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -45,7 +46,9 @@ _SIGNATURES = {
     "sig_workspace_init": (_i32, [_p, _sz, _p]),
     "sparsify_threshold": (_i32, [_p, _i64, _f32, _p, _p, _p, _p]),
     "sparsify_topk": (_i32, [_p, _i64, _i64, _p, _p, _p, _p, _sz, _p]),
-    "sparsify_nm": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _p]),
+    "sparsify_nm": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _p, _p]),
+    "sig_nm_packed_bytes": (_sz, [_i64, _i64]),
+    "nm_act_gemm_packed": (_i32, [_p, _i64, _i64, _p, _i64, _p, _p]),
     "sparse_gemv": (_i32, [_p, _i64, _i64, _p, _f32, _p, _p, _p, _p, _sz, _p]),
     "gated_mlp_sparse": (_i32, [_p, _p, _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
     "sig_row_norms": (_i32, [_p, _i64, _i64, _p, _p]),
@@ -180,8 +183,40 @@ def sparsify_nm(X, n: int, m: int, X_masked=None, mask_bits=None, want_masked=Tr
     if want_bits and mask_bits is None:
         mask_bits = torch.empty((rows, (d + 31) // 32), dtype=torch.int32, device=X.device)
     _check("sparsify_nm", _lib.sparsify_nm(
-        _ptr(X), rows, d, int(n), int(m), _ptr(X_masked), _ptr(mask_bits), _stream(stream)))
+        _ptr(X), rows, d, int(n), int(m), _ptr(X_masked), _ptr(mask_bits), None, _stream(stream)))
     return X_masked, mask_bits
+
+
+def nm_packed_bytes(rows: int, d: int) -> int:
+    return int(_lib.sig_nm_packed_bytes(rows, d))
+
+
+def sparsify_nm_packed(X, n: int = 2, out=None, stream=None):
+    """The packed 2:4 operand of ``X`` (n = 2: 2:4; n = 1: 1:4 padded to 2:4),
+    as a uint8 tensor of sig_nm_packed_bytes(rows, d) bytes (values, then the
+    tensor-core metadata; layout in include/sig.h)."""
+    _need(X, torch.float16, "X")
+    rows, d = X.shape
+    nbytes = nm_packed_bytes(rows, d)
+    if nbytes == 0:
+        raise SigError("sparsify_nm", 2)
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
+    _check("sparsify_nm", _lib.sparsify_nm(
+        _ptr(X), rows, d, int(n), 4, None, None, _ptr(out), _stream(stream)))
+    return out
+
+
+def nm_act_gemm_packed(packed, rows: int, K: int, WT, Y=None, stream=None):
+    """Y = A WT with A (rows x K) given as sparsify_nm's packed 2:4 operand."""
+    _need(packed, torch.uint8, "packed")
+    _need(WT, torch.float16, "WT", packed.device)
+    N = WT.shape[1]
+    if Y is None:
+        Y = torch.empty((rows, N), dtype=torch.float16, device=packed.device)
+    _check("nm_act_gemm_packed", _lib.nm_act_gemm_packed(
+        _ptr(packed), rows, K, _ptr(WT), N, _ptr(Y), _stream(stream)))
+    return Y
 
 
 def sparse_gemv(WT, x, t: float = 0.0, idx=None, nnz=None, y=None, ws=None, stream=None):

@@ -54,7 +54,7 @@ const char* sig_status_string(int status) {
   return "unknown status";
 }
 
-int sig_abi_version(void) { return 1; }
+int sig_abi_version(void) { return 2; }
 
 size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
   switch (op) {
@@ -114,17 +114,36 @@ int sparsify_topk(const uint16_t* x, int64_t d, int64_t k, uint32_t* mask_bits, 
   return cuda_status(launch_topk(x, (int)d, (int)k, mask_bits, idx, nnz, (cudaStream_t)stream));
 }
 
+size_t sig_nm_packed_bytes(int64_t rows, int64_t d) {
+  if (rows < 128 || rows % 128 != 0 || d < 128 || d % 128 != 0 || rows > (1 << 24) ||
+      d > (1 << 20))
+    return 0;
+  return (size_t)rows * (size_t)d / 8 * 9;   // d/2 fp16 values + d/8 metadata bytes per row
+}
+
 int sparsify_nm(const uint16_t* X, int64_t rows, int64_t d, int n, int m, uint16_t* X_masked,
-                uint32_t* mask_bits, sig_stream_t stream) {
+                uint32_t* mask_bits, void* packed, sig_stream_t stream) {
   if (!nm_pattern_ok(n, m)) return SIG_ERR_ARG;
+  if (packed != nullptr && !(m == 4 && (n == 2 || n == 1))) return SIG_ERR_ARG;
   if (rows < 0 || d < 1 || d % m != 0 || d > ((int64_t)1 << 30)) return SIG_ERR_SHAPE;
   if (rows == 0) return SIG_OK;  // an empty batch: nothing to read or write
-  if (X == nullptr || (X_masked == nullptr && mask_bits == nullptr)) return SIG_ERR_NULL;
+  if (X == nullptr || (X_masked == nullptr && mask_bits == nullptr && packed == nullptr))
+    return SIG_ERR_NULL;
+  if (packed != nullptr && sig_nm_packed_bytes(rows, d) == 0) return SIG_ERR_SHAPE;
   if (d % 8 != 0 || !aligned16(X) || (X_masked != nullptr && !aligned16(X_masked)) ||
-      !aligned4(mask_bits))
+      !aligned4(mask_bits) || !aligned16(packed))
     return SIG_ERR_ALIGN;
-  return cuda_status(launch_nm_mask(X, rows, (int)d, n, m, X_masked, mask_bits,
-                                    (cudaStream_t)stream));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (X_masked != nullptr || mask_bits != nullptr) {
+    const cudaError_t e = launch_nm_mask(X, rows, (int)d, n, m, X_masked, mask_bits, st);
+    if (e != cudaSuccess) return SIG_ERR_CUDA;
+  }
+  if (packed != nullptr) {
+    uint16_t* vals = static_cast<uint16_t*>(packed);
+    uint8_t* meta = static_cast<uint8_t*>(packed) + (size_t)rows * (size_t)d;
+    return cuda_status(launch_nm_pack(X, rows, (int)d, n, vals, meta, st));
+  }
+  return SIG_OK;
 }
 
 int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out, const uint16_t* x, float t,
@@ -371,15 +390,35 @@ int nm_act_gemm(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* WT, 
       K % m != 0 || rows > (1 << 24) || K > (1 << 20) || N > (1 << 20))
     return SIG_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(WT) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  cudaStream_t st = (cudaStream_t)stream;
   if (n == m)   // every entry kept: the plain tensor-core GEMM on X
-    return cuda_status(launch_gemm_f16(X, WT, Y, (int)rows, (int)N, (int)K, (cudaStream_t)stream));
+    return cuda_status(launch_gemm_f16(X, WT, Y, (int)rows, (int)N, (int)K, st));
   const size_t need = sig_workspace_bytes(SIG_OP_NM_GEMM, K, N, rows);
   if (ws == nullptr || ws_bytes < need) return SIG_ERR_WORKSPACE;
   if (!aligned256(ws)) return SIG_ERR_ALIGN;
+  if (m == 4 && n <= 2 && K % 128 == 0) {
+    // 2:4 (and 1:4 padded to 2:4): packed operand, sparse tensor cores
+    uint16_t* vals = reinterpret_cast<uint16_t*>(ws);
+    uint8_t* meta = reinterpret_cast<uint8_t*>(ws) + (size_t)rows * (size_t)K;
+    if (launch_nm_pack(X, rows, (int)K, n, vals, meta, st) != cudaSuccess) return SIG_ERR_CUDA;
+    return cuda_status(launch_gemm_sp(vals, meta, WT, Y, (int)rows, (int)N, (int)K, st));
+  }
   uint16_t* Xm = reinterpret_cast<uint16_t*>(ws);
-  cudaError_t e = launch_nm_mask(X, rows, (int)K, n, m, Xm, nullptr, (cudaStream_t)stream);
+  cudaError_t e = launch_nm_mask(X, rows, (int)K, n, m, Xm, nullptr, st);
   if (e != cudaSuccess) return SIG_ERR_CUDA;
-  return cuda_status(launch_gemm_f16(Xm, WT, Y, (int)rows, (int)N, (int)K, (cudaStream_t)stream));
+  return cuda_status(launch_gemm_f16(Xm, WT, Y, (int)rows, (int)N, (int)K, st));
+}
+
+int nm_act_gemm_packed(const void* packed, int64_t rows, int64_t K, const uint16_t* WT, int64_t N,
+                       uint16_t* Y, sig_stream_t stream) {
+  if (packed == nullptr || WT == nullptr || Y == nullptr) return SIG_ERR_NULL;
+  if (sig_nm_packed_bytes(rows, K) == 0 || N < 128 || N % 128 != 0 || N > (1 << 20))
+    return SIG_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(WT) || !aligned16(Y)) return SIG_ERR_ALIGN;
+  const uint16_t* vals = static_cast<const uint16_t*>(packed);
+  const uint8_t* meta = static_cast<const uint8_t*>(packed) + (size_t)rows * (size_t)K;
+  return cuda_status(launch_gemm_sp(vals, meta, WT, Y, (int)rows, (int)N, (int)K,
+                                    (cudaStream_t)stream));
 }
 
 int sig_take_device_error(unsigned* code, sig_stream_t stream) {

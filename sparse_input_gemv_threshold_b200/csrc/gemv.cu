@@ -110,6 +110,37 @@ __device__ __forceinline__ void build_local_words(const KArgs& a, int s, int K, 
   }
 }
 
+// Mask bits of one 8-input group starting at input e0 (inputs past d_in are
+// not kept).
+template <int MODE>
+__device__ __forceinline__ uint32_t group_bits(const KArgs& a, int e0, __half2 th2) {
+  const int d_in = a.d_in;
+  const float t = a.t;
+  if (e0 + 8 <= d_in) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + e0));
+    if (MODE == MASK_THRESH) return thresh_bits8(v, th2);
+    uint32_t b = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float m = fabsf(h2f(lane_half(v, j)));
+      const bool keep = MODE == MASK_THRESH_SCALED ? __fmul_rn(m, __ldg(a.scale + e0 + j)) >= t
+                        : MODE == MASK_SQUARE      ? __fmul_rn(m, m) >= t
+                                                   : m >= t;
+      b |= (keep ? 1u : 0u) << j;
+    }
+    return b;
+  }
+  uint32_t b = 0;
+  for (int j = 0; j < 8 && e0 + j < d_in; ++j) {
+    const float m = fabsf(h2f(a.x[e0 + j]));
+    const bool keep = MODE == MASK_THRESH_SCALED ? __fmul_rn(m, __ldg(a.scale + e0 + j)) >= t
+                      : MODE == MASK_SQUARE      ? __fmul_rn(m, m) >= t
+                                                 : m >= t;
+    b |= (keep ? 1u : 0u) << j;
+  }
+  return b;
+}
+
 template <int MODE, bool DUAL, int EPI, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 4)
 sgemv_kernel(const __grid_constant__ KArgs a) {
@@ -133,47 +164,83 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   // ascending order; index and dense modes: the s-th of S equal slices of the
   // index list / of all rows
   int lo = 0, hi = 0, nwords = 0, K = 0;
+  bool placed = false;   // the kept-row list is already in sidx (one chunk)
   if (MODE == MASK_THRESH || MODE == MASK_THRESH_SCALED || MODE == MASK_SQUARE) {
     const int ngroups = (d_in + 7) >> 3;
     K = s < ngroups ? (ngroups - 1 - s) / S + 1 : 0;
-    nwords = (K + 3) >> 2;
-    build_local_words<MODE>(a, s, K, nwords, words);
-    __syncthreads();
-    // exclusive prefix of the words' popcounts, thread-contiguous word ranges
-    const int per = (nwords + kThreads - 1) / kThreads;
-    const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(words[w]);
-    int incl = cnt;
+    if (K <= kThreads) {
+      // one group per thread: its 8 mask bits from one 16-byte load, one
+      // block-wide exclusive scan of the popcounts (ascending group order is
+      // ascending input order), then the thread places its own kept rows
+      const int e0 = (s + tid * S) * 8;
+      const uint32_t b = tid < K ? group_bits<MODE>(a, e0, thresh_half2(a.t)) : 0u;
+      const int cnt = __popc(b);
+      int incl = cnt;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int before = 0, total = 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (lane == 31) warp_tot[warp] = incl;
+      __syncthreads();
+      int before = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const int v = warp_tot[w];
-      before += w < warp ? v : 0;
-      total += v;
+      for (int w = 0; w < kWarps; ++w) {
+        const int v = warp_tot[w];
+        before += w < warp ? v : 0;
+        total += v;
+      }
+      int r = before + incl - cnt;
+      for (uint32_t m = b; m != 0u; m &= m - 1u) sidx[r++] = e0 + (__ffs(m) - 1);
+      if (a.mask_out != nullptr && cg == 0) {
+        uint8_t* mb = reinterpret_cast<uint8_t*>(a.mask_out);
+        if (tid < K) mb[s + tid * S] = (uint8_t)b;
+        if (s == 0 && tid < 4 * ((d_in + 31) >> 5) - ngroups) mb[ngroups + tid] = 0;
+      }
+      lo = 0;
+      hi = total;
+      placed = true;
+      __syncthreads();
+    } else {
+      nwords = (K + 3) >> 2;
+      build_local_words<MODE>(a, s, K, nwords, words);
+      __syncthreads();
+      // exclusive prefix of the words' popcounts, thread-contiguous word ranges
+      const int per = (nwords + kThreads - 1) / kThreads;
+      const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
+      int cnt = 0;
+      for (int w = w0; w < w1; ++w) cnt += __popc(words[w]);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (lane == 31) warp_tot[warp] = incl;
+      __syncthreads();
+      int before = 0, total = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const int v = warp_tot[w];
+        before += w < warp ? v : 0;
+        total += v;
+      }
+      int r = before + incl - cnt;
+      for (int w = w0; w < w1; ++w) {            // first rank held by each word
+        wpre[w] = r;
+        r += __popc(words[w]);
+      }
+      lo = 0;
+      hi = total;
+      if (a.mask_out != nullptr && cg == 0) {
+        // byte g of the mask words holds group g's bits; the slice writes its
+        // own groups, slice 0 also the padding bytes of the last word
+        uint8_t* mb = reinterpret_cast<uint8_t*>(a.mask_out);
+        for (int k = tid; k < K; k += kThreads) mb[s + k * S] = (uint8_t)(words[k >> 2] >> (8 * (k & 3)));
+        if (s == 0 && tid < 4 * ((d_in + 31) >> 5) - ngroups) mb[ngroups + tid] = 0;
+      }
+      __syncthreads();
     }
-    int r = before + incl - cnt;
-    for (int w = w0; w < w1; ++w) {            // first rank held by each word
-      wpre[w] = r;
-      r += __popc(words[w]);
-    }
-    lo = 0;
-    hi = total;
-    if (a.mask_out != nullptr && cg == 0) {
-      // byte g of the mask words holds group g's bits; the slice writes its
-      // own groups, slice 0 also the padding bytes of the last word
-      uint8_t* mb = reinterpret_cast<uint8_t*>(a.mask_out);
-      for (int k = tid; k < K; k += kThreads) mb[s + k * S] = (uint8_t)(words[k >> 2] >> (8 * (k & 3)));
-      if (s == 0 && tid < 4 * ((d_in + 31) >> 5) - ngroups) mb[ngroups + tid] = 0;
-    }
-    __syncthreads();
   } else if (MODE == MASK_IDX) {
     const int total = min(max(__ldg(a.nnz), 0), d_in);
     lo = (int)(((long long)s * total) / S);
@@ -206,7 +273,7 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
 
   for (int cb = 0; cb < n_rows; cb += a.chunk) {
     const int c_lo = lo + cb, c_hi = min(hi, c_lo + a.chunk), cn = c_hi - c_lo;
-    if (MODE != MASK_DENSE) {
+    if (MODE != MASK_DENSE && !placed) {
       if (cb > 0) __syncthreads();   // the previous chunk's rows are no longer read
       if (MODE == MASK_IDX) {
         for (int j = tid; j < cn; j += kThreads) {

@@ -142,4 +142,17 @@ cudaError_t read_device_error(unsigned* out, cudaStream_t stream);
 cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
                             int K, cudaStream_t stream);
 
+// 2:4 sparse-operand GEMM (nm_gemm.cu): Y = A WT with A given packed (vals
+// [M x K/2] fp16, the two kept values of every block of four; meta the
+// tensor-core metadata, 2048 bytes per 128 x 128 block, see sparsify_nm).
+// M % 128 == 0, K % 128 == 0, N % 128 == 0.
+cudaError_t launch_gemm_sp(const uint16_t* vals, const uint8_t* meta, const uint16_t* WT,
+                           uint16_t* Y, int M, int N, int K, cudaStream_t stream);
+
+// Packed 2:4 operand of X (mask.cu): n = 2 keeps the two largest |x| of every
+// block of four, n = 1 the largest plus a zero at the block's smallest other
+// position.  rows % 128 == 0, d % 128 == 0.
+cudaError_t launch_nm_pack(const uint16_t* X, int64_t rows, int d, int n, uint16_t* vals,
+                           uint8_t* meta, cudaStream_t stream);
+
 }  // namespace sig

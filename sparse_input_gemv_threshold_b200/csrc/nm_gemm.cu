@@ -111,6 +111,45 @@ __host__ __device__ constexpr uint32_t instr_desc_f16(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);
 }
 
+// Epilogue of one 128 x BN accumulator tile: warp w reads tensor-memory lanes
+// 32w .. 32w+31 (one output row per thread), 32 columns at a time, adds
+// mu * colsum[c] when colsum is given, rounds to fp16 and stores the row.
+template <int BN>
+__device__ __forceinline__ void store_tile(uint32_t tmem, int warp, uint16_t* yrow, float mu,
+                                           const float* colsum) {
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t r[32];
+    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    uint32_t p[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      float v0 = __uint_as_float(r[2 * q]), v1 = __uint_as_float(r[2 * q + 1]);
+      if (colsum != nullptr) {
+        v0 = fmaf(mu, __ldg(colsum + c + 2 * q), v0);
+        v1 = fmaf(mu, __ldg(colsum + c + 2 * q + 1), v1);
+      }
+      const __half2 h = __floats2half2_rn(v0, v1);
+      p[q] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+  }
+}
+
 template <int BN>
 struct __align__(1024) GemmSmem {
   uint16_t A[kStages][kBM * kBK];   // 16 KB per stage, K-major, swizzled rows of 128 B
@@ -235,44 +274,194 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (have_acc) {
     const int row = m0 + warp * 32 + lane;
-    uint16_t* yrow = Y + (size_t)row * N + n0;
-    const float mu = shift != nullptr ? __ldg(shift + row) : 0.f;   // the per-token shift added back
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c;
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-          "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-            "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-            "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-            "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-            "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-            "=r"(r[31])
-          : "r"(taddr));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      uint32_t p[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        float v0 = __uint_as_float(r[2 * q]), v1 = __uint_as_float(r[2 * q + 1]);
-        if (shift != nullptr) {
-          v0 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q), v0);
-          v1 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q + 1), v1);
-        }
-        const __half2 h = __floats2half2_rn(v0, v1);
-        p[q] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-      uint4* dst = reinterpret_cast<uint4*>(yrow + c);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
-    }
+    store_tile<BN>(tmem, warp, Y + (size_t)row * N + n0,
+                   shift != nullptr ? __ldg(shift + row) : 0.f,   // the per-token shift added back
+                   shift != nullptr ? colsum + n0 : nullptr);
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2:4 sparse-operand GEMM (tcgen05.mma.sp, kind::f16).
+//
+// A is the packed activation: per row, the two kept values of every block of
+// four entries (K/2 fp16, K contiguous), and their positions as 2-bit
+// metadata.  For M = 128 and K = 32 logical entries one sparse MMA reads 32
+// bits of metadata per tensor-memory lane; a 128 x 128 block of the logical
+// A carries 2048 bytes of metadata = 128 lanes x 16 bytes, which one
+// tcgen05.cp (128x128b) moves from shared to tensor memory.  The packed
+// buffer keeps the metadata in exactly that lane order (see sparsify_nm in
+// the header), so a stage brings it in with one 2048-byte bulk copy.
+//
+// Stage = 128 logical K: A 128 rows x 64 packed fp16 (16 KB, one 128-byte
+// swizzled row each), B 128 k-rows x BN (BN/64 blocks of 16 KB), metadata
+// 2 KB.  The issuer copies the stage's metadata into tensor memory, then
+// issues four sparse MMAs (K = 32 each: A advances 32 bytes in its row, B
+// 32 k-rows = 4096 bytes, the metadata one tensor-memory column; an odd
+// column is addressed as the even one below it with selector id2 = 1).
+// ---------------------------------------------------------------------------
+constexpr int kSpBK = 128;        // logical K per stage
+constexpr int kSpStages = 2;
+constexpr uint32_t kSpMetaBytes = 2048;
+
+template <int BN>
+struct __align__(1024) SpSmem {
+  uint16_t A[kSpStages][kBM * 64];      // 16 KB per stage
+  uint16_t B[kSpStages][kSpBK * BN];    // BN/64 blocks of 128 k-rows x 128 B
+  uint8_t E[kSpStages][kSpMetaBytes];   // metadata, lane-major (lane L at 16 L)
+  unsigned long long full[kSpStages];
+  unsigned long long empty[kSpStages];
+  unsigned long long accum;
+  uint32_t tmem_base;
+  int abort_flag;
+  int consumed;
+};
+
+// Instruction descriptor of the sparse MMA: the dense one with the sparse
+// flag (bit 2) and the metadata selector id2 (bits 0-1).
+__host__ __device__ constexpr uint32_t instr_desc_f16_sp(int M, int N, uint32_t id2) {
+  return instr_desc_f16(M, N) | (1u << 2) | (id2 & 3u);
+}
+
+// Shared-memory descriptor of the metadata tile for tcgen05.cp 128x128b: no
+// swizzle, K-major, 8-row core matrices of 16-byte rows stored contiguously
+// (128 bytes apart); one 16-byte column, so the leading offset is unused.
+__device__ __forceinline__ uint64_t smem_desc_meta(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fffu);
+  d |= (uint64_t)((kSpMetaBytes >> 4) & 0x3fffu) << 16;   // leading offset (unused)
+  d |= (uint64_t)((128u >> 4) & 0x3fffu) << 32;           // 8-row groups 128 B apart
+  d |= (uint64_t)1 << 46;                                  // descriptor version for sm_100
+  return d;                                                // layout type 0: no swizzle
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+               const uint8_t* __restrict__ meta, uint16_t* __restrict__ Y, int M, int N, int K) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  SpSmem<BN>& sm = *reinterpret_cast<SpSmem<BN>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+  const int kblocks = K / kSpBK;
+  volatile int* abort_flag = &sm.abort_flag;
+  constexpr uint32_t kTmemCols = BN == 256 ? 512u : 256u;   // BN accumulator + 4 metadata columns
+  pdl_trigger();
+
+  if (tid == 0) {
+    for (int s = 0; s < kSpStages; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 1);
+      mbar_init(smem_u32(&sm.empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm.accum), 1);
+    sm.abort_flag = 0;
+    sm.consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t tmem_e = tmem + (uint32_t)BN;   // metadata columns, 4-aligned
+  pdl_wait();
+
+  constexpr uint32_t kStageBytes = kBM * 64 * 2 + kSpBK * BN * 2 + kSpMetaBytes;
+  const uint8_t* meta_rb = meta + (size_t)blockIdx.y * (size_t)kblocks * kSpMetaBytes;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer ----
+      int issued = 0;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % kSpStages;
+        const uint32_t ph = (uint32_t)(kb / kSpStages) & 1u;
+        if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag)) break;
+        const uint32_t fb = smem_u32(&sm.full[s]);
+        mbar_expect_tx(fb, kStageBytes);
+        tma_load_2d(smem_u32(sm.A[s]), &mapA, kb * 64, m0, fb);
+#pragma unroll
+        for (int j = 0; j < BN / 64; ++j)
+          tma_load_2d(smem_u32(sm.B[s]) + j * (kSpBK * 128), &mapB, n0 + j * 64, kb * kSpBK, fb);
+        bulk_load(smem_u32(sm.E[s]), meta_rb + (size_t)kb * kSpMetaBytes, kSpMetaBytes, fb);
+        ++issued;
+      }
+      if (*abort_flag) {
+        for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb) {
+          const long long t0 = clock64();
+          while (!mbar_try(smem_u32(&sm.full[kb % kSpStages]), (uint32_t)(kb / kSpStages) & 1u) &&
+                 clock64() - t0 < kTimeoutCycles) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer ----
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % kSpStages;
+        const uint32_t ph = (uint32_t)(kb / kSpStages) & 1u;
+        if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag)) break;
+        *(volatile int*)&sm.consumed = kb + 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
+        asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(tmem_e),
+                     "l"(smem_desc_meta(smem_u32(sm.E[s])))
+                     : "memory");
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t da = smem_desc(a0 + j * 32, 16, 1024);
+          const uint64_t db = smem_desc(b0 + j * 4096, kSpBK * 128, 1024);
+          const uint32_t e_col = tmem_e + (uint32_t)j;
+          const uint32_t idesc = instr_desc_f16_sp(kBM, BN, e_col & 1u);
+          const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "setp.ne.b32 p, %5, 0;\n\t"
+              "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(tmem),
+              "l"(da), "l"(db), "r"(e_col & ~1u), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+        asm volatile(
+            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                smem_u32(&sm.empty[s]))
+            : "memory");
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(&sm.accum))
+          : "memory");
+    }
+    __syncwarp();
+  }
+
+  const bool have_acc = mbar_wait(smem_u32(&sm.accum), 0u, abort_flag) && !*abort_flag;
+  __syncwarp();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (have_acc) store_tile<BN>(tmem, warp, Y + (size_t)(m0 + warp * 32 + lane) * N + n0, 0.f, nullptr);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
 }
@@ -320,6 +509,19 @@ cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, uint16_t* Y,
   return cudaPeekAtLastError();
 }
 
+template <int BN>
+cudaError_t launch_sp_bn(const CUtensorMap& ma, const CUtensorMap& mb, const uint8_t* meta,
+                         uint16_t* Y, int M, int N, int K, cudaStream_t stream) {
+  const size_t smem = sizeof(SpSmem<BN>) + 1024;
+  auto fn = gemm_sp_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(N / BN, M / kBM);
+  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, meta, Y, M, N, K);
+  if (e != cudaSuccess) return e;
+  return cudaPeekAtLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
@@ -337,6 +539,17 @@ cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_
 cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
                             int K, cudaStream_t stream) {
   return launch_gemm_f16_shift(A, WT, Y, M, N, K, nullptr, nullptr, stream);
+}
+
+cudaError_t launch_gemm_sp(const uint16_t* vals, const uint8_t* meta, const uint16_t* WT,
+                           uint16_t* Y, int M, int N, int K, cudaStream_t stream) {
+  if (M % kBM != 0 || K % kSpBK != 0 || N % 128 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, vals, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, kBM))
+    return cudaErrorInvalidValue;
+  if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kSpBK)) return cudaErrorInvalidValue;
+  if (N % 256 == 0) return launch_sp_bn<256>(ma, mb, meta, Y, M, N, K, stream);
+  return launch_sp_bn<128>(ma, mb, meta, Y, M, N, K, stream);
 }
 
 cudaError_t read_device_error(unsigned* out, cudaStream_t stream) {

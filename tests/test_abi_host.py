@@ -62,7 +62,7 @@ def test_binding_covers_every_declared_symbol():
 
 
 def test_status_strings_and_version(lib):
-    assert lib.sig_abi_version() == 1
+    assert lib.sig_abi_version() == 2
     for s in range(8):
         assert lib.sig_status_string(s)
     assert lib.sig_status_string(99) == b"unknown status"
@@ -114,13 +114,30 @@ def test_mask_validation(lib):
     assert t(FAKE, 0, 0, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
     assert t(FAKE, 131073, 5, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
     n = lib.sparsify_nm
-    assert n(FAKE, 4, 64, 3, 2, FAKE, FAKE, None) == ARG      # n > m
-    assert n(FAKE, 4, 64, 0, 4, FAKE, FAKE, None) == ARG      # n < 1
-    assert n(FAKE, 4, 60, 2, 3, FAKE, FAKE, None) == ARG      # m not a power of two
-    assert n(FAKE, 4, 36, 2, 8, FAKE, FAKE, None) == SHAPE    # m does not divide d
-    assert n(FAKE, 4, 64, 2, 4, None, None, None) == NULL     # no output requested
-    assert n(FAKE, -1, 64, 2, 4, FAKE, FAKE, None) == SHAPE
-    assert n(None, 0, 64, 2, 4, None, None, None) == OK          # empty batch
+    assert n(FAKE, 4, 64, 3, 2, FAKE, FAKE, None, None) == ARG      # n > m
+    assert n(FAKE, 4, 64, 0, 4, FAKE, FAKE, None, None) == ARG      # n < 1
+    assert n(FAKE, 4, 60, 2, 3, FAKE, FAKE, None, None) == ARG      # m not a power of two
+    assert n(FAKE, 4, 36, 2, 8, FAKE, FAKE, None, None) == SHAPE    # m does not divide d
+    assert n(FAKE, 4, 64, 2, 4, None, None, None, None) == NULL     # no output requested
+    assert n(FAKE, -1, 64, 2, 4, FAKE, FAKE, None, None) == SHAPE
+    assert n(None, 0, 64, 2, 4, None, None, None, None) == OK          # empty batch
+    # the packed 2:4 operand: 2:4 and 1:4 only, rows and d multiples of 128
+    assert n(FAKE, 128, 128, 4, 8, None, None, FAKE, None) == ARG
+    assert n(FAKE, 128, 128, 2, 2, None, None, FAKE, None) == ARG
+    assert n(FAKE, 128, 128, 3, 4, None, None, FAKE, None) == ARG
+    assert n(FAKE, 100, 128, 2, 4, None, None, FAKE, None) == SHAPE
+    assert n(FAKE, 128, 192, 2, 4, None, None, FAKE, None) == SHAPE
+    assert n(FAKE, 128, 128, 1, 4, None, None, FAKE + 8, None) == ALIGN
+    pb = lib.sig_nm_packed_bytes
+    assert pb(128, 128) == 128 * 128 * 9 // 8
+    assert pb(4096, 1024) == 4096 * 1024 * 9 // 8
+    assert pb(100, 128) == 0 and pb(128, 64) == 0 and pb(0, 128) == 0
+    g = lib.nm_act_gemm_packed
+    assert g(None, 128, 128, FAKE, 128, FAKE, None) == NULL
+    assert g(FAKE, 128, 128, FAKE, 96, FAKE, None) == SHAPE
+    assert g(FAKE, 128, 64, FAKE, 128, FAKE, None) == SHAPE
+    assert g(FAKE, 96, 128, FAKE, 128, FAKE, None) == SHAPE
+    assert g(FAKE + 8, 128, 128, FAKE, 128, FAKE, None) == ALIGN
 
 
 def test_multi_validation(lib):
@@ -331,7 +348,7 @@ def test_32bit_buffers_must_be_4_byte_aligned(lib):
     assert tk(FAKE, 64, 3, odd, FAKE, FAKE, None, 0, None) == ALIGN
     assert tk(FAKE, 64, 3, FAKE, odd, FAKE, None, 0, None) == ALIGN
     assert tk(FAKE, 64, 3, FAKE, FAKE, odd, None, 0, None) == ALIGN
-    assert lib.sparsify_nm(FAKE, 4, 64, 2, 4, None, odd, None) == ALIGN
+    assert lib.sparsify_nm(FAKE, 4, 64, 2, 4, None, odd, None, None) == ALIGN
     sg = lib.sparse_gemv
     assert sg(FAKE, 64, 64, FAKE, 0.0, odd, FAKE, FAKE, FAKE, big, None) == ALIGN
     assert sg(FAKE, 64, 64, FAKE, 0.0, FAKE, odd, FAKE, FAKE, big, None) == ALIGN

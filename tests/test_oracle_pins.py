@@ -205,6 +205,50 @@ def test_nm_golden():
     assert checked == 8
 
 
+def test_nm_pack_golden():
+    lines = _read_lines("nm_packed_small.txt")
+    row, checked = None, 0
+    for ln in lines:
+        if ln.startswith("row:"):
+            row = np.array(_floats(ln[4:]), dtype=np.float16)
+            continue
+        head, vals, pos = ln.split("|")
+        p = oracle.nm_pack_2of4(row, int(head))
+        want_v = np.array(_floats(vals), dtype=np.float16)
+        assert np.array_equal(p["values"][0].view(np.uint16), want_v.view(np.uint16)), ln
+        assert p["positions"][0].tolist() == [int(v) for v in pos.split()], ln
+        checked += 1
+    assert checked == 4
+
+
+@pytest.mark.parametrize("n", [2, 1])
+def test_nm_pack_decodes_to_the_masked_block(n):
+    """Scattering the slots back to their positions gives the masked X (bit
+    for bit, +0 where dropped); positions ascend inside every block; a 1:4
+    block pads at its smallest unkept position, with +0."""
+    rng = np.random.default_rng(40 + n)
+    X = rng.choice([0.0, -0.0, 0.5, -0.5, 1.0, 2.0, -2.0], size=(6, 64)).astype(np.float16)
+    X[0, :5] = np.nan
+    X = np.concatenate([X, rng.laplace(0, 1, (4, 64)).astype(np.float16)])
+    p = oracle.nm_pack_2of4(X, n)
+    rows, d = X.shape
+    back = np.zeros_like(X)
+    pos = p["positions"].reshape(rows, d // 4, 2).astype(int)
+    vals = p["values"].reshape(rows, d // 4, 2)
+    assert (pos[..., 0] < pos[..., 1]).all()
+    for r in range(rows):
+        for b in range(d // 4):
+            for s in range(2):
+                back[r, 4 * b + pos[r, b, s]] = vals[r, b, s]
+    want = np.where(oracle.nm_mask(X, n, 4), X, np.float16(0))
+    assert np.array_equal(back.view(np.uint16), want.view(np.uint16))
+    if n == 1:
+        kept = oracle.nm_mask(X, 1, 4).reshape(rows, d // 4, 4)
+        first_free = np.argmax(~kept, axis=-1)
+        pad_slot = np.where(np.take_along_axis(kept, pos, axis=-1), -1, pos).max(axis=-1)
+        assert np.array_equal(pad_slot, first_free)
+
+
 @pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (3, 4), (4, 8), (8, 16)])
 def test_nm_brute_force_blocks(n, m):
     rng = np.random.default_rng(5 + n + m)
