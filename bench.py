@@ -454,7 +454,8 @@ def run_ours(args, rank, world, local):
         extras["teal_mlp"] = bench_teal_mlp(args, stream, sig, hbm_peak)
         extras["rana_rank_adapter"] = bench_rank_adapter(args, stream, sig, hbm_peak)
         extras["batched_per_token_masks"] = bench_batch(args, stream, sig, hbm_peak)
-        extras["int8_weights"] = bench_q8(args, stream, sig, hbm_peak)
+        extras["int8_weights"] = bench_q8(args, stream, sig, hbm_peak, "int8")
+        extras["fp8_weights"] = bench_q8(args, stream, sig, hbm_peak, "fp8")
         result["extras"] = extras
         result["cpu_baseline"] = cpu_baseline(groups)
     return result
@@ -737,15 +738,18 @@ def bench_batch(args, stream, sig, hbm_peak):
     return out
 
 
-def bench_q8(args, stream, sig, hbm_peak):
-    """int8 weights (one scale per column) at the Llama-2-7B shapes and a Llama-70B
-    MLP shape, 50 % threshold, against the fp16 sparse GEMV on the same shapes."""
+def bench_q8(args, stream, sig, hbm_peak, fmt="int8"):
+    """8-bit weights (int8 or fp8 e4m3, one scale per column) at the Llama-2-7B
+    shapes and a Llama-70B MLP shape, 50 % threshold, against the fp16 sparse
+    GEMV on the same shapes."""
     import torch
-    out = {"note": "int8 kept rows cost d_out bytes; fp16 rows 2 d_out"}
+    out = {"note": f"{fmt} kept rows cost d_out bytes; fp16 rows 2 d_out"}
+    gen = workloads.q8_projection if fmt == "int8" else workloads.f8_projection
+    call = sig.sparse_gemv_q8 if fmt == "int8" else sig.sparse_gemv_f8
+    op = sig.OP_SPARSE_GEMV_Q8 if fmt == "int8" else sig.OP_SPARSE_GEMV_F8
     for name, d_in, d_out in (("q", 4096, 4096), ("gate", 4096, 11008), ("down", 11008, 4096),
                               ("70B up", 8192, 28672)):
-        QT, scale, x, ts = workloads.q8_projection(seed=args.seed + d_in + d_out, d_in=d_in,
-                                                   d_out=d_out)
+        QT, scale, x, ts = gen(seed=args.seed + d_in + d_out, d_in=d_in, d_out=d_out)
         t = ts[0.5]
         copies = max(2, math.ceil(4 * 126e6 / (d_in * d_out)))
         Qs = [torch.from_numpy(QT).cuda()]
@@ -753,12 +757,12 @@ def bench_q8(args, stream, sig, hbm_peak):
         sd = torch.from_numpy(scale).cuda()
         xd = torch.from_numpy(x).cuda()
         y = torch.empty(d_out, dtype=torch.float16, device="cuda")
-        ws = torch.zeros(max(256, sig.workspace_bytes(sig.OP_SPARSE_GEMV_Q8, d_in, d_out)),
-                         dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(max(256, sig.workspace_bytes(op, d_in, d_out)), dtype=torch.uint8,
+                         device="cuda")
 
         def f(c):
             def g():
-                sig.sparse_gemv_q8(Qs[c], sd, xd, t, y=y, ws=ws, stream=stream)
+                call(Qs[c], sd, xd, t, y=y, ws=ws, stream=stream)
             return g
         sg = StepGraphs([f(c) for c in range(copies)], stream)
         steps = 400
@@ -779,7 +783,8 @@ def bench_q8(args, stream, sig, hbm_peak):
         us16 = time_steps(sh, steps, len(Ws), stream) / steps * 1e6
         out[f"{name} {d_in}->{d_out}"] = {"us": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
                                           "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
-                                          "fp16_sparse_us": round(us16, 2)}
+                                          "fp16_sparse_us": round(us16, 2),
+                                          "speedup_vs_fp16": round(us16 / us, 3)}
         del Qs, Ws, sg, sh
         torch.cuda.empty_cache()
     return out

@@ -80,7 +80,8 @@ typedef enum {
   SIG_OP_NM_GEMM = 4,      /* nm_act_gemm(K = d_in, N = d_out, rows)   */
   SIG_OP_RANK_ADAPTER = 5, /* rank_adapter_sparse(d_in, d_out, rows = r) */
   SIG_OP_SPARSE_GEMV_BATCH = 6, /* sparse_gemv_batch(d_in, d_out, rows = tokens) */
-  SIG_OP_SPARSE_GEMV_Q8 = 7     /* sparse_gemv_q8(d_in, d_out)              */
+  SIG_OP_SPARSE_GEMV_Q8 = 7,    /* sparse_gemv_q8(d_in, d_out)              */
+  SIG_OP_SPARSE_GEMV_F8 = 8     /* sparse_gemv_f8(d_in, d_out)              */
 } sig_op;
 
 /* Largest activation length the fused mask prologue accepts. */
@@ -104,10 +105,13 @@ SIG_API int sig_abi_version(void);
 SIG_API size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows);
 
 /*
- * Zero a workspace once before its first use (asynchronously on `stream`).
- * Every operation leaves its counters at zero again when it completes, so a
- * workspace needs this only once after allocation.  ws must be 256-byte
- * aligned.
+ * Zero a workspace before its first use (asynchronously on `stream`).  A
+ * workspace then serves any number of calls of ONE operation at ONE shape
+ * (the same sizes and, for sparse_gemv_multi, the same d_out list): the fp16
+ * GEMVs tag their split-K partial sums with a per-tile epoch that advances
+ * with every call, and the other operations leave their counters at zero.
+ * Zero it again before using it for another operation or another shape.
+ * ws must be 256-byte aligned.
  */
 SIG_API int sig_workspace_init(void* ws, size_t ws_bytes, sig_stream_t stream);
 
@@ -196,11 +200,16 @@ SIG_API size_t sig_nm_packed_bytes(int64_t rows, int64_t d);
  *   WT   [d_in x d_out] fp16 row-major, 16-byte aligned, d_out % 8 == 0.
  *   x    [d_in] fp16, 16-byte aligned.       y [d_out] fp16 out, 16-byte aligned.
  *   ws   sig_workspace_bytes(SIG_OP_SPARSE_GEMV, d_in, d_out, 0) bytes, 256-byte
- *        aligned, zeroed once by sig_workspace_init (or allocated zeroed); it
- *        holds the float32 partial sums of the split-K slices and one arrival
- *        counter per 256-column tile.  When the size is 0 (one slice per tile,
- *        which the planner chooses above 296 tiles, i.e. d_out > 75776) ws may
- *        be NULL.
+ *        aligned, zeroed by sig_workspace_init (or allocated zeroed) before
+ *        its first use and serving this shape only (see sig_workspace_init);
+ *        it holds one epoch word per 256-column tile and the split-K slices'
+ *        partial sums as 64-bit {float32 value, epoch tag} words.  When the
+ *        size is 0 (one slice per tile, which the planner chooses above 296
+ *        tiles, i.e. d_out > 75776) ws may be NULL.
+ * The split-K finish: every slice stores its partial sums and exits; the
+ * tile's last slice waits (bounded, ~2 s; on expiry it sets bit 1 of the
+ * device error word, see sig_take_device_error) until every slice's word
+ * carries this call's tag, then adds them in slice order.
  * The result is bit-identical from run to run (fixed-order split-K reduction;
  * no floating-point atomics).  An empty mask writes y = 0.
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d_in < 1, d_in > SIG_MAX_D_IN, d_out < 8,
@@ -224,7 +233,8 @@ SIG_API int sparse_gemv(const uint16_t* WT, int64_t d_in, int64_t d_out,
  *   d_out    HOST array of n_mat sizes, each a multiple of 8.
  *   x, t, idx, nnz   as sparse_gemv (one mask for all the weights).
  *   ws       sig_workspace_bytes_multi(n_mat, d_out, d_in) bytes, 256-byte
- *            aligned, zeroed once (it may be NULL when that size is 0).
+ *            aligned, zeroed before its first use and serving these shapes only
+ *            (see sig_workspace_init); it may be NULL when that size is 0.
  * Each y[p] meets the tolerance of sparse_gemv and is bit-identical from run
  * to run.  It can differ in the last bits from a separate sparse_gemv call on
  * W_p, because the grid, and so the split-K order, is planned for all the
@@ -298,6 +308,20 @@ SIG_API int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out,
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
  */
 SIG_API int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+                           const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                           sig_stream_t stream);
+
+/*
+ * The same product with fp8 weights: QT holds OCP E4M3 codes (sign bit 7,
+ * exponent bits 6..3 with bias 7, mantissa bits 2..0; no infinities,
+ * S.1111.111 is NaN), W[j, i] = s_j e4m3(QT[i, j]):
+ *   y_j = fp16( s_j * sum_{i: m_i} e4m3(QT[i, j]) x_i )   (float32 accumulation)
+ * Every e4m3 value is exact in fp16, so the hardware converts two codes to an
+ * fp16 pair in one instruction.  Arguments, workspace
+ * (sig_workspace_bytes(SIG_OP_SPARSE_GEMV_F8, d_in, d_out, 0)), shape rules
+ * and errors as sparse_gemv_q8.
+ */
+SIG_API int sparse_gemv_f8(const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
                            const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                            sig_stream_t stream);
 
@@ -444,18 +468,19 @@ SIG_API int nm_act_gemm_packed(const void* packed, int64_t rows, int64_t K, cons
  * budget is fixed at start-up, or plain C code with no allocator.  The pages
  * have no counterpart to this entry point; it computes exactly what
  * gated_mlp_sparse computes, with the same arguments minus ws / ws_bytes.
- * Its scratch (split-K partial sums and arrival counters of the two
- * products, and the fp16 hidden vector h when h_out is NULL) lives in one
- * device array of SIG_NOALLOC_SCRATCH_BYTES (2 MiB) inside the library,
+ * Its scratch (the split-K partial sums of the two products with their
+ * epoch words, and the fp16 hidden vector h when h_out is NULL) lives in one
+ * device array of SIG_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library,
  * which every GPU that loads the library holds until the process exits.  It
  * allocates nothing and calls no allocating routine.
  *   - A call whose scratch (sig_workspace_bytes(SIG_OP_GATED_MLP, d_model,
  *     d_ff, 0)) would exceed SIG_NOALLOC_SCRATCH_BYTES returns SIG_ERR_SHAPE
  *     with nothing enqueued.  Every shape gated_mlp_sparse accepts
- *     (d_model, d_ff <= SIG_MAX_D_IN) needs at most 1927 KiB, so it fits;
+ *     (d_model, d_ff <= SIG_MAX_D_IN) needs at most 3703 KiB, so it fits;
  *     larger sizes are rejected with SIG_ERR_SHAPE like everywhere else.
  *   - Every call shares the array and finds the previous call's contents in
- *     it; the call clears what must start at zero.  Calls that overlap on the
+ *     it; the call clears what must start at zero (a memset of the partial-sum
+ *     area, about 3.3 MB at Llama-2-7B MLP shapes).  Calls that overlap on the
  *     GPU (other streams, other host threads) race; serialise them.
  *   - The first call on each device, with that device current, looks up the
  *     array's device address (cudaGetSymbolAddress) and caches it; make that
@@ -466,7 +491,7 @@ SIG_API int nm_act_gemm_packed(const void* packed, int64_t rows, int64_t K, cons
  *     process.
  * Errors: as gated_mlp_sparse, except SIG_ERR_WORKSPACE (none is taken).
  */
-#define SIG_NOALLOC_SCRATCH_BYTES (2u << 20)
+#define SIG_NOALLOC_SCRATCH_BYTES (4u << 20)
 SIG_API int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                      const uint16_t* WdT, const float* down_norms,
                                      int64_t d_model, int64_t d_ff, float t,
@@ -474,13 +499,28 @@ SIG_API int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT, con
                                      sig_stream_t stream);
 
 /*
- * Read and clear the library's device error word (no counterpart on the
- * pages; it reports the bounded waits of the tensor-core GEMM).  Synchronises
- * `stream`.  *code receives 0 when no kernel gave up on a wait, else a
- * non-zero bit set; the call then returns SIG_ERR_TIMEOUT.
+ * Read and clear the library's device error words (no counterpart on the
+ * pages; they report the bounded waits: bit 0, a tensor-core GEMM pipeline
+ * wait; bit 1, the split-K finish of an fp16 GEMV).  Synchronises `stream`.
+ * *code receives 0 when no kernel gave up on a wait, else the bits set; the
+ * call then returns SIG_ERR_TIMEOUT.
  * Errors: SIG_ERR_NULL (code), SIG_ERR_CUDA.
  */
 SIG_API int sig_take_device_error(unsigned* code, sig_stream_t stream);
+
+/*
+ * Set the limit, in SM clock cycles, after which a pipeline wait of the
+ * tensor-core GEMMs (nm_act_gemm, nm_act_gemm_ex, nm_act_gemm_packed) gives
+ * up, on the current device; cycles <= 0 restores the default (4e9, about 2 s
+ * at 1.9 GHz).  No counterpart on the pages: it lets a caller (or a test)
+ * shorten the failure-detection window.  A kernel that gives up records a bit
+ * in the device error word (sig_take_device_error), lets the copies it has
+ * issued land (waiting up to the default limit for each), frees its tensor
+ * memory and returns; its output is not valid.  Synchronous with respect to
+ * the host (cudaMemcpyToSymbol); do not call it during stream capture.
+ * Errors: SIG_ERR_CUDA.
+ */
+SIG_API int sig_set_wait_limit(long long cycles);
 
 #ifdef __cplusplus
 }

@@ -60,7 +60,8 @@ Readings where the pages are silent or disagree (each one is a choice):
   ``float32(v_i) * float32(v_i)`` as one float32 multiply; ``score >= t``.
 * Weight-quantised product (the pages fix no format): int8 weights q with one
   float32 scale per output column, ``W_ij = s_j * q_ij``; the activation and
-  its mask stay fp16, and ``y_j = s_j * sum_i q_ij (m_i x_i)``.
+  its mask stay fp16, and ``y_j = s_j * sum_i q_ij (m_i x_i)``.  The same with
+  fp8 e4m3 weights (OCP E4M3, decoded exactly) in place of int8.
 * N:M mitigation variants ([NM] Methodology: selection criteria ACT and WT,
   error mitigation D-/S-/L-PTS and VAR): a per-token shift mu gives
   ``x' = fp16(float32(x) - mu)`` (the product adds back ``mu * r_j`` with
@@ -87,7 +88,7 @@ __all__ = [
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
     "union_mask", "batched_sparse_linear", "q8_sparse_linear", "teal_mlp",
     "pts_shift", "wt_scores", "nm_mask_by_score", "var_gamma", "nm_variant", "nm_variant_gemm",
-    "nm_pack_2of4",
+    "nm_pack_2of4", "e4m3_value", "f8_sparse_linear",
 ]
 
 
@@ -457,6 +458,37 @@ def q8_sparse_linear(QT, scale, x, mask, cols=None) -> dict:
         QT, s64 = QT[:, np.asarray(cols)], s64[np.asarray(cols)]
     xm = np.where(np.asarray(mask, dtype=bool), np.asarray(x, dtype=np.float64), 0.0)
     Q64 = QT.astype(np.float64)
+    y64 = (xm @ Q64) * s64
+    bound = (np.abs(xm) @ np.abs(Q64)) * np.abs(s64)
+    idx = compact(mask)
+    return {"mask": np.asarray(mask, dtype=bool), "idx": idx, "nnz": int(idx.size),
+            "y64": y64, "y16": fp16(y64), "bound": bound}
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """The value of each fp8 e4m3 code (the OCP 8-bit floating-point format
+    E4M3: sign bit 7, four exponent bits 6..3 with bias 7, three mantissa bits
+    2..0; exponent 0 is subnormal, 2^-6 * m/8; S.1111.111 is NaN; no
+    infinities), exactly, in float64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def f8_sparse_linear(QT, scale, x, mask, cols=None) -> dict:
+    """y_j = s_j * sum_i e4m3(QT[i, j]) * (m_i ? x_i : 0) in float64: the
+    weight-quantised product of :func:`q8_sparse_linear` with fp8 e4m3 weights
+    (one float32 scale per output column) in place of int8 ones."""
+    QT = np.asarray(QT, dtype=np.uint8)
+    s64 = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    if cols is not None:
+        QT, s64 = QT[:, np.asarray(cols)], s64[np.asarray(cols)]
+    Q64 = e4m3_value(QT)
+    xm = np.where(np.asarray(mask, dtype=bool), np.asarray(x, dtype=np.float64), 0.0)
     y64 = (xm @ Q64) * s64
     bound = (np.abs(xm) @ np.abs(Q64)) * np.abs(s64)
     idx = compact(mask)

@@ -25,7 +25,8 @@ __all__ = [
     "sparse_gemv_multi", "workspace_bytes_multi", "OP_RANK_ADAPTER", "rank_adapter_sparse",
     "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch", "OP_SPARSE_GEMV_Q8",
     "sparse_gemv_q8", "sparsify_nm_ex", "nm_act_gemm_ex", "col_sums", "teal_mlp_sparse",
-    "nm_packed_bytes", "sparsify_nm_packed", "nm_act_gemm_packed",
+    "nm_packed_bytes", "sparsify_nm_packed", "nm_act_gemm_packed", "sparse_gemv_f8",
+    "OP_SPARSE_GEMV_F8", "set_wait_limit",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -33,6 +34,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
 OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM, OP_RANK_ADAPTER = 1, 2, 3, 4, 5
 OP_SPARSE_GEMV_BATCH = 6
 OP_SPARSE_GEMV_Q8 = 7
+OP_SPARSE_GEMV_F8 = 8
 MAX_BATCH = 16
 MAX_D_IN = 131072
 
@@ -54,12 +56,14 @@ _SIGNATURES = {
     "sig_row_norms": (_i32, [_p, _i64, _i64, _p, _p]),
     "nm_act_gemm": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _sz, _p]),
     "sig_take_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _p]),
+    "sig_set_wait_limit": (_i32, [ctypes.c_longlong]),
     "gated_mlp_sparse_noalloc": (_i32, [_p, _p, _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p]),
     "sparse_gemv_multi": (_i32, [_i32, _p, _p, _i64, _p, _f32, _p, _p, _p, _p, _sz, _p]),
     "sig_workspace_bytes_multi": (_sz, [_i32, _p, _i64]),
     "rank_adapter_sparse": (_i32, [_p, _p, _p, _i64, _i64, _i64, _f32, _p, _p, _p, _p, _sz, _p]),
     "sparse_gemv_batch": (_i32, [_p, _i64, _i64, _p, _i64, _f32, _p, _p, _sz, _p]),
     "sparse_gemv_q8": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
+    "sparse_gemv_f8": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
     "sparsify_nm_ex": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _p]),
     "nm_act_gemm_ex": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _sz,
                               _p]),
@@ -362,6 +366,25 @@ def sparse_gemv_q8(QT, scale, x, t: float, y=None, ws=None, stream=None):
     return y
 
 
+def sparse_gemv_f8(QT, scale, x, t: float, y=None, ws=None, stream=None):
+    """y = W (m . x) with fp8 e4m3 weight codes QT (uint8, d_in x d_out) and
+    float32 column scales."""
+    _need(QT, torch.uint8, "QT")
+    _need(scale, torch.float32, "scale", QT.device)
+    _need(x, torch.float16, "x", QT.device)
+    d_in, d_out = QT.shape
+    if x.numel() != d_in or scale.numel() != d_out:
+        raise ValueError("shapes: QT (d_in, d_out), scale (d_out), x (d_in)")
+    if y is None:
+        y = torch.empty(d_out, dtype=torch.float16, device=QT.device)
+    if ws is None:
+        ws = workspace(OP_SPARSE_GEMV_F8, d_in, d_out, device=QT.device, stream=stream)
+    _check("sparse_gemv_f8", _lib.sparse_gemv_f8(
+        _ptr(QT), _ptr(scale), d_in, d_out, _ptr(x), float(t), _ptr(y), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return y
+
+
 def sparse_gemv_batch(WT, X, t: float, Y=None, ws=None, stream=None):
     """Y[b] = W (m_b . X[b]), m_b = |X[b]| >= t, for B <= MAX_BATCH tokens in one launch."""
     _need(WT, torch.float16, "WT")
@@ -468,3 +491,8 @@ def take_device_error(stream=None) -> int:
     if st not in (0, 6):
         raise SigError("sig_take_device_error", st)
     return int(code.value)
+
+
+def set_wait_limit(cycles: int) -> None:
+    """Cycles after which a tensor-core GEMM wait gives up (<= 0: the default)."""
+    _check("sig_set_wait_limit", _lib.sig_set_wait_limit(int(cycles)))

@@ -77,6 +77,7 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
         return 0;
       return plan_gemv_batch(d_in, d_out, (int)rows).ws_bytes();
     case SIG_OP_SPARSE_GEMV_Q8:
+    case SIG_OP_SPARSE_GEMV_F8:
       if (check_gemv_shape(d_in, d_out) != SIG_OK || d_out % 16 != 0) return 0;
       return plan_gemv_q8(d_in, d_out).ws_bytes();
     case SIG_OP_NM_GEMM:
@@ -181,21 +182,36 @@ int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out, const uin
                                        (cudaStream_t)stream));
 }
 
-int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+namespace {
+
+int quantised_gemv(int fmt, const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
                    const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                    sig_stream_t stream) {
   if (QT == nullptr || scale == nullptr || x == nullptr || y == nullptr) return SIG_ERR_NULL;
   const int sh = check_gemv_shape(d_in, d_out);
   if (sh != SIG_OK) return sh;
   if (d_out % 16 != 0) return SIG_ERR_SHAPE;
-  if (!aligned16(QT) || !aligned16(x) || !aligned16(y) ||
-      (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
-    return SIG_ERR_ALIGN;
+  if (!aligned16(QT) || !aligned16(x) || !aligned16(y) || !aligned4(scale)) return SIG_ERR_ALIGN;
   const GemvPlan p = plan_gemv_q8(d_in, d_out);
   if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
   if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
-  return cuda_status(launch_gemv_q8(p, QT, scale, x, t, y, (int)d_in, (int)d_out, ws,
+  return cuda_status(launch_gemv_q8(p, fmt, QT, scale, x, t, y, (int)d_in, (int)d_out, ws,
                                     (cudaStream_t)stream));
+}
+
+}  // namespace
+
+int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+                   const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                   sig_stream_t stream) {
+  return quantised_gemv(kFmtInt8, reinterpret_cast<const uint8_t*>(QT), scale, d_in, d_out, x, t, y,
+                        ws, ws_bytes, stream);
+}
+
+int sparse_gemv_f8(const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+                   const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                   sig_stream_t stream) {
+  return quantised_gemv(kFmtE4M3, QT, scale, d_in, d_out, x, t, y, ws, ws_bytes, stream);
 }
 
 size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in) {
@@ -421,9 +437,16 @@ int nm_act_gemm_packed(const void* packed, int64_t rows, int64_t K, const uint16
                                     (cudaStream_t)stream));
 }
 
+int sig_set_wait_limit(long long cycles) {
+  return cuda_status(set_wait_limit(cycles));
+}
+
 int sig_take_device_error(unsigned* code, sig_stream_t stream) {
   if (code == nullptr) return SIG_ERR_NULL;
-  if (read_device_error(code, (cudaStream_t)stream) != cudaSuccess) return SIG_ERR_CUDA;
+  unsigned gemm = 0, gemv = 0;
+  if (read_device_error(&gemm, (cudaStream_t)stream) != cudaSuccess) return SIG_ERR_CUDA;
+  if (read_gemv_error(&gemv, (cudaStream_t)stream) != cudaSuccess) return SIG_ERR_CUDA;
+  *code = gemm | gemv;
   return *code == 0u ? SIG_OK : SIG_ERR_TIMEOUT;
 }
 

@@ -22,12 +22,18 @@
 //   2. 8 warps stream the slice's rows of the tile, 8 rows in flight per warp:
 //      16-byte non-allocating loads with an L2 evict-first policy, the
 //      activation value riding along as a broadcast load, fp32 FMA;
-//   3. the warps' sums meet in shared memory (fixed order), the CTA writes one
-//      partial per column, and the CTA that arrives last for the tile (one
-//      acquire-release atomic per CTA) loads the S partials in one batch, adds
-//      them in slice order and stores fp16.
-// No floating-point atomics and no spin-waits; y is bit-identical from run to
-// run.
+//   3. the warps' sums meet in shared memory (fixed order) and the CTA
+//      stores one partial per column as a 64-bit word {value, tag} (tag = the
+//      tile's epoch + 1, read from the workspace at the start) with a relaxed
+//      store, and exits.  The tile's last slice, the CTA dispatched last,
+//      instead polls the tile's partial words in batches until every tag is
+//      current, adds them in slice order (its own last) and stores fp16; it
+//      then advances the tile's epoch.  The value and its tag travel in one
+//      single-copy-atomic 64-bit word, so no fence and no atomic stand
+//      between the last partial store and the sum.  The wait is bounded
+//      (~2 s of clock cycles; on expiry the kernel sets a bit in the device
+//      error word and stores what it has).
+// No floating-point atomics; y is bit-identical from run to run.
 #include "common.cuh"
 #include "internal.h"
 
@@ -35,9 +41,14 @@
 
 namespace sig {
 
+// Device error word of the split-K finish (bit 1: a tile's last slice gave up
+// waiting for the other slices' partial sums); read with the GEMM's word.
+__device__ unsigned g_gemv_error = 0u;
+
 namespace {
 
 constexpr int kThreads = kGemvThreads;        // 256
+constexpr long long kFinishSpinCycles = 4000000000ll;   // ~2 s at 1.9 GHz
 constexpr int kWarps = kThreads / 32;         // 8
 constexpr int kTile = kGemvTile;              // 256 outputs per CTA
 constexpr int kMaxS = kGemvMaxSplits;         // 64
@@ -62,8 +73,8 @@ struct KArgs {
   uint32_t words_bytes;   // shared bytes of the mask words (and again of their prefixes)
   uint32_t union_bytes;   // shared bytes of words + prefixes / the warp-sum buffer
   uint32_t* mask_out;
-  unsigned* counters;     // [C]
-  float* partials;        // [S][d_out_total] (then the same again for the second product)
+  unsigned* epochs;       // [C]: calls completed on each tile
+  unsigned long long* slots;   // [S][d_out_total] {value, tag} (then again for the second product)
 };
 
 // Mask bits of the 8-input groups this slice owns.  Group g covers inputs
@@ -146,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 sgemv_kernel(const __grid_constant__ KArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_tot[kWarps];
-  __shared__ int s_last;
+  __shared__ unsigned s_tag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cg = blockIdx.x, s = blockIdx.y;   // global column tile, slice
@@ -158,6 +169,13 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
 
   pdl_trigger();
   pdl_wait();
+  // tag of this call's partial sums: the tile's epoch + 1 (the tile's finishing
+  // slices advance the epoch only after every slice of the tile has read it
+  // and stored its partials).  The word was written by an earlier grid that
+  // has completed, so a plain load suffices; it is issued now and published
+  // to shared memory only after the prologue, so that it does not delay
+  // thread 0's own activation load.
+  const unsigned epoch0 = (tid == 0 && S > 1) ? __ldcg(a.epochs + cg) : 0u;
 
   // ---- 1. this CTA's rows [lo, hi) of its kept-row list -----------------
   // threshold modes: the kept inputs of the slice's own 8-input groups, in
@@ -250,6 +268,7 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     hi = (int)(((long long)(s + 1) * d_in) / S);
   }
   const int n_rows = hi - lo;
+  if (tid == 0) s_tag = epoch0 + 1u;   // read after the barriers that follow
 
   // ---- 2. stream the slice's rows of this column tile ------------------
   // the weight this tile belongs to (static indices only: the arguments stay
@@ -369,41 +388,105 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     if (colr_ok) finish(p, p2);
     return;
   }
-  const size_t pcol = (size_t)e_col0 + colr;       // column in the partial-sum space
-  if (colr_ok) {
-    a.partials[(size_t)s * dtot + pcol] = p;
-    if (DUAL) a.partials[(size_t)S * dtot + (size_t)s * dtot + pcol] = p2;
+  // ---- split-K finish: slices S-1 and S-2 finish the tile's two 128-column
+  // halves (slice S-1 the first, S-2 the second); every other partial sum is
+  // stored as a tagged 64-bit word and the CTA exits
+  const unsigned tag = s_tag;
+  const int kdes = S - 1 - s;                 // 0 or 1 for the finishing slices
+  const bool des = kdes == 0 || kdes == 1;
+  const size_t pbase = (size_t)e_col0 + (size_t)(cg - e_first) * kTile;   // tile column 0
+  unsigned long long* const slots = a.slots;
+  unsigned long long* const slots2 = a.slots + (size_t)S * dtot;
+  if (colr_ok && !(des && (tid >> 7) == kdes)) {
+    st_relaxed_u64(slots + (size_t)s * dtot + pbase + tid,
+                   ((unsigned long long)tag << 32) | __float_as_uint(p));
+    if (DUAL)
+      st_relaxed_u64(slots2 + (size_t)s * dtot + pbase + tid,
+                     ((unsigned long long)tag << 32) | __float_as_uint(p2));
   }
-  // one release-acquire arrival per CTA: the barrier orders every thread's
-  // partial store before thread 0's release, and thread 0's acquire before
-  // the last arriver's loads
+  if (!des) return;
+  // this CTA's own partials of every column, then two threads per column of
+  // the half it finishes: thread h sums slices [0, mid) (h = 0) or
+  // [mid, S) (h = 1) in order, polling each word until it carries the tag
+  __syncthreads();                            // the warp sums have been read
+  float* own = red;                           // [256] (and [256] for the second product)
+  float* half_sum = red + 2 * kTile;          // [128] (and [128])
+  own[tid] = p;
+  if (DUAL) own[kTile + tid] = p2;
   __syncthreads();
-  if (tid == 0) s_last = atomic_add_acq_rel_gpu(a.counters + cg, 1u) == (unsigned)(S - 1);
-  __syncthreads();
-  if (!s_last) return;
-  if (colr_ok) {
-    // the partials of the column in flight together (32 per batch for the
-    // single product, 8 for the dual one), then added in slice order
-    constexpr int B = DUAL ? 8 : 32;
-    const float* pp = a.partials + pcol;
-    float g = 0.f, u = 0.f;
-    for (int q0 = 0; q0 < S; q0 += B) {
-      float pg[B], pu[B];
+  const int c = kdes * (kTile / 2) + (tid & (kTile / 2 - 1));   // tile column finished here
+  const int h = tid >> 7;
+  const int mid = S >> 1;
+  const int q_lo = h ? mid : 0, q_hi = h ? S : mid;
+  const int colc = (cg - e_first) * kTile + c;
+  const bool colc_ok = colc < e_dout;
+  bool gave_up = false;
+  float g = 0.f, u = 0.f;
+  if (colc_ok) {
+    constexpr int B = DUAL ? 4 : 16;          // words of the column in flight together
+    unsigned long long* sl = slots + pbase + c;
+    unsigned long long* sl2 = slots2 + pbase + c;
+    const long long t0 = clock64();
+    for (int q0 = q_lo; q0 < q_hi; q0 += B) {
+      unsigned long long v[B], v2[B];
+      uint32_t missing = 0u;
 #pragma unroll
       for (int k = 0; k < B; ++k) {
-        const bool ok = q0 + k < S;
-        pg[k] = ok ? __ldcg(pp + (size_t)(q0 + k) * dtot) : 0.f;
-        if (DUAL) pu[k] = ok ? __ldcg(pp + (size_t)(S + q0 + k) * dtot) : 0.f;
+        const int q = q0 + k;
+        if (q < q_hi && q != s) {
+          v[k] = ld_relaxed_u64(sl + (size_t)q * dtot);
+          if (DUAL) v2[k] = ld_relaxed_u64(sl2 + (size_t)q * dtot);
+        } else {   // past the range (adds +0), or this CTA's own slice (from shared memory)
+          v[k] = ((unsigned long long)tag << 32) | (q < q_hi ? __float_as_uint(own[c]) : 0u);
+          v2[k] = ((unsigned long long)tag << 32) |
+                  (DUAL && q < q_hi ? __float_as_uint(own[kTile + c]) : 0u);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < B; ++k)
+        missing |= ((unsigned)(v[k] >> 32) != tag || (DUAL && (unsigned)(v2[k] >> 32) != tag) ? 1u : 0u) << k;
+      while (missing != 0u) {
+        if (clock64() - t0 > kFinishSpinCycles) {
+          gave_up = true;
+          break;
+        }
+        __nanosleep(64);
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+          if ((missing >> k) & 1u) {
+            v[k] = ld_relaxed_u64(sl + (size_t)(q0 + k) * dtot);
+            if (DUAL) v2[k] = ld_relaxed_u64(sl2 + (size_t)(q0 + k) * dtot);
+          }
+        }
+        missing = 0u;
+#pragma unroll
+        for (int k = 0; k < B; ++k)
+          missing |= ((unsigned)(v[k] >> 32) != tag || (DUAL && (unsigned)(v2[k] >> 32) != tag) ? 1u : 0u) << k;
       }
 #pragma unroll
       for (int k = 0; k < B; ++k) {
-        g += pg[k];
-        if (DUAL) u += pu[k];
+        g += __uint_as_float((unsigned)v[k]);
+        if (DUAL) u += __uint_as_float((unsigned)v2[k]);
       }
     }
-    finish(g, u);
   }
-  if (tid == 0) a.counters[cg] = 0u;  // ready for the next call on this workspace
+  if (h == 1) {
+    half_sum[tid & 127] = g;
+    if (DUAL) half_sum[kTile / 2 + (tid & 127)] = u;
+  }
+  __syncthreads();
+  if (h == 0 && colc_ok) {
+    const float gs = g + half_sum[tid];                      // slices [0, mid) then [mid, S)
+    const float us = DUAL ? u + half_sum[kTile / 2 + tid] : 0.f;
+    if (EPI == EPI_STORE) {
+      Y[colc] = f2h_rn(gs);
+    } else {
+      const float sg = gs / (1.0f + expf(-gs));
+      Y[colc] = f2h_rn(sg * us);
+    }
+  }
+  if (gave_up) atomicOr(&g_gemv_error, 2u);
+  if (tid == 0) st_relaxed_u32(a.epochs + cg, tag);   // the next call tags with tag + 1
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -438,8 +521,10 @@ GemvPlan plan_gemv_multi(int64_t d_in, const int64_t* d_out, int n_mat, bool dua
   const size_t words = round_up((size_t)((d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)kWarps * kTile * 4 * (dual ? 2 : 1);
   p.smem = std::max(2 * words, red) + round_up((size_t)p.chunk * 4, 16);
+  // workspace: one epoch word per column tile, then the slices' 64-bit
+  // {partial sum, tag} words
   p.counters = p.S > 1 ? round_up((size_t)p.C * 4, 256) : 0;
-  p.partials = p.S > 1 ? round_up((size_t)p.S * total * 4 * (dual ? 2 : 1), 256) : 0;
+  p.partials = p.S > 1 ? round_up((size_t)p.S * total * 8 * (dual ? 2 : 1), 256) : 0;
   return p;
 }
 
@@ -473,9 +558,10 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   k.words_bytes = (uint32_t)words;
   k.union_bytes = (uint32_t)std::max(2 * words, red);
   k.mask_out = a.mask_out;
-  k.counters = reinterpret_cast<unsigned*>(a.ws);
-  k.partials = a.ws != nullptr ? reinterpret_cast<float*>(reinterpret_cast<char*>(a.ws) + p.counters)
-                               : nullptr;
+  k.epochs = reinterpret_cast<unsigned*>(a.ws);
+  k.slots = a.ws != nullptr
+                ? reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(a.ws) + p.counters)
+                : nullptr;
   if (epi == EPI_SILU_MUL) {
     if (mode == MASK_DENSE) return launch_t<MASK_DENSE, true, EPI_SILU_MUL>(p, k, stream);
     if (mode == MASK_THRESH) return launch_t<MASK_THRESH, true, EPI_SILU_MUL>(p, k, stream);
@@ -494,6 +580,17 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
     case MASK_DENSE: return launch_t<MASK_DENSE, false, EPI_STORE>(p, k, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t read_gemv_error(unsigned* out, cudaStream_t stream) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_gemv_error, sizeof(unsigned), 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  const unsigned zero = 0;
+  return cudaMemcpyToSymbolAsync(g_gemv_error, &zero, sizeof(unsigned), 0, cudaMemcpyHostToDevice,
+                                 stream);
 }
 
 }  // namespace sig

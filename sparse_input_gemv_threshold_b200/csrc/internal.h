@@ -56,8 +56,10 @@ struct GemvPlan {
   int S;              // K-splits (slices of the kept-row list), <= kGemvMaxSplits
   int chunk;          // rows of a slice staged in shared memory at once
   size_t smem;        // dynamic shared memory per CTA
-  size_t counters;    // workspace bytes for per-tile arrival counters
-  size_t partials;    // workspace bytes for the slices' float32 partial sums
+  size_t counters;    // workspace bytes for one word per column tile (arrival
+                      // counter, or epoch of the fp16 GEMV's tagged partials)
+  size_t partials;    // workspace bytes for the slices' partial sums (float32;
+                      // 64-bit {value, tag} words in the fp16 GEMV)
   size_t ws_bytes() const { return counters + partials; }
 };
 
@@ -137,7 +139,9 @@ cudaError_t launch_row_norms(const uint16_t* WT, int64_t rows, int cols, float* 
 
 // Tensor-core GEMM (nm_gemm.cu): Y = A * B, A [M x K] fp16 row-major,
 // B given as WT [K x N] fp16 row-major, Y [M x N] fp16.
-cudaError_t read_device_error(unsigned* out, cudaStream_t stream);
+cudaError_t read_device_error(unsigned* out, cudaStream_t stream);   // GEMM word (gemm .cu)
+cudaError_t read_gemv_error(unsigned* out, cudaStream_t stream);     // split-K finish word
+cudaError_t set_wait_limit(long long cycles);   // <= 0: the default (~2 s)
 
 cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
                             int K, cudaStream_t stream);

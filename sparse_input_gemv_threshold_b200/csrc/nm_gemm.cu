@@ -16,9 +16,11 @@
 // setup and the tensor-memory allocation overlap the end of the kernel before
 // it; every thread then waits for that kernel (griddepcontrol.wait) before it
 // reads global memory or starts a timed wait.
-// Every mbarrier wait gives up after ~2 s of clock cycles: the kernel then
-// records SIG_ERR_TIMEOUT in a device error word, lets the copies it issued
-// land (again with a limit), frees its tensor memory and returns.
+// Every mbarrier wait gives up after ~2 s of clock cycles (a device variable,
+// settable through sig_set_wait_limit): the kernel then records
+// SIG_ERR_TIMEOUT in a device error word, lets the copies it issued land
+// (waiting at most the default ~2 s for each), frees its tensor memory and
+// returns.
 #include "common.cuh"
 #include "internal.h"
 #include "nm_ex.h"
@@ -32,14 +34,17 @@ namespace sig {
 
 __device__ unsigned g_device_error = 0u;
 
+// Cycles after which a pipeline wait gives up (sig_set_wait_limit); the waits
+// that let already issued copies land after a give-up keep the full default.
+constexpr long long kTimeoutCycles = 4000000000ll;  // ~2 s at 1.9 GHz
+__device__ long long g_wait_limit = kTimeoutCycles;
+
 namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;          // one 128-byte swizzle row of fp16
 constexpr int kStages = 4;
 constexpr int kThreads = 128;
-constexpr long long kTimeoutCycles = 4000000000ll;  // ~2 s at 1.9 GHz
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -68,14 +73,25 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // Bounded wait: false after the time limit or once another role aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   const long long t0 = clock64();
+  const long long limit = *(volatile long long*)&g_wait_limit;
   while (!mbar_try(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kTimeoutCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       atomicOr(&g_device_error, 1u);
       return false;
     }
   }
+  return true;
+}
+
+// Wait that is not cut short by a give-up: used to let issued copies and
+// MMAs finish before the CTA frees its tensor memory and exits.  Bounded by
+// the default limit; false if that ran out.
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kTimeoutCycles) return false;
   return true;
 }
 
@@ -203,10 +219,10 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   pdl_wait();
 
   constexpr uint32_t kStageBytes = (kBM * kBK + kBK * BN) * 2;
+  int issued = 0;   // stages whose copies thread 0 has issued
 
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer ----
-      int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % kStages;
         const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
@@ -218,15 +234,6 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         for (int j = 0; j < BN / 64; ++j)
           tma_load_2d(smem_u32(sm.B[s]) + j * (kBK * 128), &mapB, n0 + j * 64, kb * kBK, fb);
         ++issued;
-      }
-      if (*abort_flag) {
-        // let the copies already issued land before the CTA can exit
-        for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb) {
-          const long long t0 = clock64();
-          while (!mbar_try(smem_u32(&sm.full[kb % kStages]), (uint32_t)(kb / kStages) & 1u) &&
-                 clock64() - t0 < kTimeoutCycles) {
-          }
-        }
       }
     }
     __syncwarp();
@@ -269,16 +276,26 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   }
 
   // ---- epilogue: TMEM -> registers -> fp16 -> global ----
-  const bool have_acc = mbar_wait(smem_u32(&sm.accum), 0u, abort_flag) && !*abort_flag;
+  // The MMA thread commits the accumulator barrier also after a give-up, so
+  // it completes once every issued MMA has finished; this wait is not cut
+  // short by the abort flag.
+  const bool acc_done = drain_wait(smem_u32(&sm.accum), 0u);
   __syncwarp();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (have_acc) {
+  if (acc_done && !*abort_flag) {
     const int row = m0 + warp * 32 + lane;
     store_tile<BN>(tmem, warp, Y + (size_t)row * N + n0,
                    shift != nullptr ? __ldg(shift + row) : 0.f,   // the per-token shift added back
                    shift != nullptr ? colsum + n0 : nullptr);
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    // after a give-up: let the copies issued but never consumed land before
+    // the CTA's shared memory goes away
+    for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb)
+      drain_wait(smem_u32(&sm.full[kb % kStages]), (uint32_t)(kb / kStages) & 1u);
+  }
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN)
@@ -388,10 +405,10 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 
   constexpr uint32_t kStageBytes = kBM * 64 * 2 + kSpBK * BN * 2 + kSpMetaBytes;
   const uint8_t* meta_rb = meta + (size_t)blockIdx.y * (size_t)kblocks * kSpMetaBytes;
+  int issued = 0;   // stages whose copies thread 0 has issued
 
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer ----
-      int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % kSpStages;
         const uint32_t ph = (uint32_t)(kb / kSpStages) & 1u;
@@ -404,14 +421,6 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           tma_load_2d(smem_u32(sm.B[s]) + j * (kSpBK * 128), &mapB, n0 + j * 64, kb * kSpBK, fb);
         bulk_load(smem_u32(sm.E[s]), meta_rb + (size_t)kb * kSpMetaBytes, kSpMetaBytes, fb);
         ++issued;
-      }
-      if (*abort_flag) {
-        for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb) {
-          const long long t0 = clock64();
-          while (!mbar_try(smem_u32(&sm.full[kb % kSpStages]), (uint32_t)(kb / kSpStages) & 1u) &&
-                 clock64() - t0 < kTimeoutCycles) {
-          }
-        }
       }
     }
     __syncwarp();
@@ -454,14 +463,272 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     __syncwarp();
   }
 
-  const bool have_acc = mbar_wait(smem_u32(&sm.accum), 0u, abort_flag) && !*abort_flag;
+  // the accumulator barrier completes once every issued MMA has finished,
+  // also after a give-up (see gemm_f16_kernel)
+  const bool acc_done = drain_wait(smem_u32(&sm.accum), 0u);
   __syncwarp();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (have_acc) store_tile<BN>(tmem, warp, Y + (size_t)(m0 + warp * 32 + lane) * N + n0, 0.f, nullptr);
+  if (acc_done && !*abort_flag)
+    store_tile<BN>(tmem, warp, Y + (size_t)(m0 + warp * 32 + lane) * N + n0, 0.f, nullptr);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb)
+      drain_wait(smem_u32(&sm.full[kb % kSpStages]), (uint32_t)(kb / kSpStages) & 1u);
+  }
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair GEMMs (tcgen05 cta_group::2), dense kind::f16 and 2:4 sparse.
+//
+// A cluster of two CTAs computes a 256 x BN output tile: CTA r of the pair
+// owns rows 128 r .. 128 r + 127 of the tile.  Each CTA loads its own 128 rows
+// of A and HALF of the tile's B columns (BN/2, from column n0 + r BN/2) into
+// the same shared-memory offsets; the leader (rank 0) issues one M = 256
+// MMA that reads A and B from both CTAs' shared memory and accumulates each
+// CTA's 128 rows in that CTA's tensor memory.  B (the weight) is therefore
+// read from L2 half as often per SM as in the one-CTA kernels, and a stage is
+// small enough for a four- (sparse) or six-stage (dense) ring.
+//
+// Both CTAs' copies for a stage complete on the LEADER's full barrier (the
+// 2-SM form of the TMA load lets the peer signal it); the leader's thread
+// posts the stage's bytes of both CTAs.  The leader's MMA thread frees a stage
+// in both CTAs with one multicast commit, and commits the accumulator barrier
+// of both CTAs the same way.  No TMA load multicasts: each CTA fetches its own
+// tiles from this GPU's memory.
+//
+// Bounded waits as in the one-CTA kernels.  A give-up sets the CTA's abort
+// flag; the epilogue of either CTA stores nothing if either flag is set
+// (read across the pair through distributed shared memory), the leader lets
+// the stages it posted land, and both CTAs then wait ~20 us before the final
+// cluster barrier so that a peer copy whose stage the leader never posted has
+// landed too.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// TMA load whose completion is signalled on the pair leader's barrier
+// (`bar` is a shared::cluster address, possibly in the peer CTA).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_1d_pair(uint32_t dst, const CUtensorMap* map, int c0,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2}], [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+template <bool SPARSE>
+struct PairCfg {
+  static constexpr int kBN = 256;                        // N of the pair's MMA
+  static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
+  static constexpr int kStages = SPARSE ? 4 : 6;
+  static constexpr uint32_t kABytes = kBM * 64 * 2;      // 128 rows x 128 B
+  static constexpr uint32_t kBBytes = kBK * (kBN / 2) * 2;
+  static constexpr uint32_t kEBytes = SPARSE ? kSpMetaBytes : 0;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kEBytes;   // per CTA
+  static constexpr uint32_t kTmemCols = SPARSE ? 512u : 256u;
+};
+
+template <bool SPARSE>
+struct __align__(1024) PairSmem {
+  using C = PairCfg<SPARSE>;
+  uint16_t A[C::kStages][kBM * 64];
+  uint16_t B[C::kStages][C::kBK * (C::kBN / 2)];          // 2 blocks of 64 columns
+  uint8_t E[SPARSE ? C::kStages : 1][SPARSE ? kSpMetaBytes : 16];
+  unsigned long long full[C::kStages];                    // used in the leader
+  unsigned long long empty[C::kStages];
+  unsigned long long accum;
+  uint32_t tmem_base;
+  int abort_flag;
+  int consumed;
+};
+
+template <bool SPARSE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                 const __grid_constant__ CUtensorMap mapE, uint16_t* __restrict__ Y, int M, int N,
+                 int K, const float* __restrict__ shift, const float* __restrict__ colsum) {
+  using C = PairCfg<SPARSE>;
+  constexpr int BN = C::kBN, BK = C::kBK, S = C::kStages;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  PairSmem<SPARSE>& sm = *reinterpret_cast<PairSmem<SPARSE>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int m0 = blockIdx.x * kBM;                 // this CTA's rows
+  const int n0 = blockIdx.y * BN;                  // the pair's columns
+  const int nb = n0 + (int)rank * (BN / 2);        // this CTA's half of B
+  const int kblocks = K / BK;
+  volatile int* abort_flag = &sm.abort_flag;
+  pdl_trigger();
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 1);
+      mbar_init(smem_u32(&sm.empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm.accum), 1);
+    sm.abort_flag = 0;
+    sm.consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  // both CTAs' barriers exist before any copy or commit of the pair targets them
+  cluster_sync();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = sm.tmem_base;
+  pdl_wait();
+
+  int issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer (both CTAs) ----
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag)) break;
+        const uint32_t fb = map_to_rank(smem_u32(&sm.full[s]), 0);
+        if (leader) mbar_expect_tx(smem_u32(&sm.full[s]), 2 * C::kStageBytes);
+        tma_load_2d_pair(smem_u32(sm.A[s]), &mapA, kb * 64, m0, fb);
+#pragma unroll
+        for (int j = 0; j < BN / 128; ++j)
+          tma_load_2d_pair(smem_u32(sm.B[s]) + j * (BK * 128), &mapB, nb + j * 64, kb * BK, fb);
+        if constexpr (SPARSE)
+          tma_load_1d_pair(smem_u32(sm.E[s]), &mapE,
+                           (int)(((size_t)blockIdx.x * kblocks + kb) * (kSpMetaBytes / 8)), fb);
+        ++issued;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1 && leader) {
+    if (lane == 0) {  // ---- MMA issuer (leader only) ----
+      const uint32_t tmem_e = tmem + 256u;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag)) break;
+        *(volatile int*)&sm.consumed = kb + 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
+        if constexpr (SPARSE) {
+          asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(tmem_e),
+                       "l"(smem_desc_meta(smem_u32(sm.E[s])))
+                       : "memory");
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t da = smem_desc(a0 + j * 32, 16, 1024);
+            const uint64_t db = smem_desc(b0 + j * 4096, BK * 128, 1024);
+            const uint32_t e_col = tmem_e + (uint32_t)j;
+            const uint32_t idesc = instr_desc_f16_sp(2 * kBM, BN, e_col & 1u);
+            const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %5, 0;\n\t"
+                "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(tmem),
+                "l"(da), "l"(db), "r"(e_col & ~1u), "r"(idesc), "r"(acc)
+                : "memory");
+          }
+        } else {
+          constexpr uint32_t idesc = instr_desc_f16(2 * kBM, BN);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = smem_desc(a0 + k * 32, 16, 1024);
+            const uint64_t db = smem_desc(b0 + k * 2048, BK * 128, 1024);
+            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                : "memory");
+          }
+        }
+        commit_pair(smem_u32(&sm.empty[s]));      // frees stage s in both CTAs
+      }
+      commit_pair(smem_u32(&sm.accum));
+    }
+    __syncwarp();
+  }
+
+  // ---- epilogue: each CTA its own 128 rows ----
+  const bool acc_done = drain_wait(smem_u32(&sm.accum), 0u);
+  __syncwarp();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const bool pair_ok =
+      !*abort_flag && ld_cluster_u32(map_to_rank(smem_u32(&sm.abort_flag), rank ^ 1u)) == 0u;
+  if (acc_done && pair_ok) {
+    const int row = m0 + warp * 32 + lane;
+    store_tile<BN>(tmem, warp, Y + (size_t)row * N + n0,
+                   shift != nullptr ? __ldg(shift + row) : 0.f,
+                   shift != nullptr ? colsum + n0 : nullptr);
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    if (leader)   // the stages this CTA posted: both CTAs' bytes land on these barriers
+      for (int kb = *(volatile int*)&sm.consumed; kb < issued; ++kb)
+        drain_wait(smem_u32(&sm.full[kb % S]), (uint32_t)(kb / S) & 1u);
+    const long long t0 = clock64();
+    while (clock64() - t0 < 40000) {
+    }
+  }
+  __syncthreads();
+  // the peer's tensor memory and shared memory stay until both CTAs are done
+  cluster_sync();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
                  : "memory");
   }
 }
@@ -494,6 +761,35 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+
+// 1-D tensor map over `bytes` of metadata as uint64 elements, box of one
+// 2048-byte tile (256 elements), no swizzle.
+bool make_map_meta(CUtensorMap* map, const void* base, uint64_t bytes) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[1] = {bytes / 8};
+  cuuint64_t strides[1] = {0};
+  cuuint32_t box[1] = {kSpMetaBytes / 8};
+  cuuint32_t estr[1] = {1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 1, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <bool SPARSE>
+cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me,
+                        uint16_t* Y, int M, int N, int K, const float* shift, const float* colsum,
+                        cudaStream_t stream) {
+  const size_t smem = sizeof(PairSmem<SPARSE>) + 1024;
+  auto fn = gemm_pair_kernel<SPARSE>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(M / kBM, N / PairCfg<SPARSE>::kBN);
+  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, me, Y, M, N, K, shift, colsum);
+  if (e != cudaSuccess) return e;
+  return cudaPeekAtLastError();
 }
 
 template <int BN>
@@ -532,6 +828,8 @@ cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kBK)) return cudaErrorInvalidValue;
+  if (M % 256 == 0 && N % 256 == 0)   // CTA pairs: 256 x 256 tiles, half of B per CTA
+    return launch_pair<false>(ma, mb, ma, Y, M, N, K, shift, colsum, stream);
   if (N % 256 == 0) return launch_bn<256>(ma, mb, Y, M, N, K, shift, colsum, stream);
   return launch_bn<128>(ma, mb, Y, M, N, K, shift, colsum, stream);
 }
@@ -548,8 +846,18 @@ cudaError_t launch_gemm_sp(const uint16_t* vals, const uint8_t* meta, const uint
   if (!make_map(&ma, vals, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, kBM))
     return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kSpBK)) return cudaErrorInvalidValue;
+  if (M % 256 == 0 && N % 256 == 0) {   // CTA pairs: 256 x 256 tiles, half of B per CTA
+    CUtensorMap me;
+    if (!make_map_meta(&me, meta, (uint64_t)M * (uint64_t)K / 8)) return cudaErrorInvalidValue;
+    return launch_pair<true>(ma, mb, me, Y, M, N, K, nullptr, nullptr, stream);
+  }
   if (N % 256 == 0) return launch_sp_bn<256>(ma, mb, meta, Y, M, N, K, stream);
   return launch_sp_bn<128>(ma, mb, meta, Y, M, N, K, stream);
+}
+
+cudaError_t set_wait_limit(long long cycles) {
+  const long long v = cycles > 0 ? cycles : kTimeoutCycles;
+  return cudaMemcpyToSymbol(g_wait_limit, &v, sizeof(v));
 }
 
 cudaError_t read_device_error(unsigned* out, cudaStream_t stream) {

@@ -6,13 +6,14 @@
 // memory through its own pool, a serving loop with a fixed memory budget
 // decided at start-up, or C code with no allocator of its own.  This entry
 // point takes only the inputs and outputs.  Its scratch (split-K partial sums
-// and arrival counters of the two products, and the fp16 hidden vector h when
+// with their epoch words for the two products, and the fp16 hidden vector h when
 // h_out is NULL) lives in one file-scope device array of
-// SIG_NOALLOC_SCRATCH_BYTES (2 MiB) that every GPU which loads the library
+// SIG_NOALLOC_SCRATCH_BYTES (4 MiB) that every GPU which loads the library
 // holds until the process exits.
 //
 // The array is shared by every call on a device and keeps the last call's
-// contents, so each call first clears the counters that must start at zero.
+// contents, so each call first clears what must start at zero: the epoch and
+// tagged partial-sum words of the two products.
 // Calls that overlap on the GPU (other streams, other host threads) race on
 // the array; serialise them.  A call whose scratch would exceed the array is
 // rejected with SIG_ERR_SHAPE before anything is enqueued.
@@ -84,12 +85,10 @@ extern "C" int gated_mlp_sparse_noalloc(const uint16_t* x, const uint16_t* WgT,
   char* base = static_cast<char*>(scratch);
   cudaStream_t st = (cudaStream_t)stream;
 
-  // arrival counters (if the products use any) must start at zero
-  if (g.up.counters > 0 && cudaMemsetAsync(base, 0, g.up.counters, st) != cudaSuccess)
-    return SIG_ERR_CUDA;
-  if (g.down.counters > 0 &&
-      cudaMemsetAsync(base + g.off_down, 0, g.down.counters, st) != cudaSuccess)
-    return SIG_ERR_CUDA;
+  // The split-K finish tags each partial sum with the tile's epoch; the array
+  // keeps the previous call's words, which may come from another shape, so
+  // every call starts from zeroed epochs and words (everything below h).
+  if (g.off_h > 0 && cudaMemsetAsync(base, 0, g.off_h, st) != cudaSuccess) return SIG_ERR_CUDA;
 
   uint16_t* h = h_out != nullptr ? h_out : reinterpret_cast<uint16_t*>(base + g.off_h);
   GemvLaunch up{};

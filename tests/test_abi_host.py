@@ -314,7 +314,7 @@ def test_noalloc_validation(lib):
 
 def test_noalloc_scratch_covers_every_accepted_shape(lib):
     """Every (d_model, d_ff) that gated_mlp_sparse accepts (multiples of 8 up
-    to SIG_MAX_D_IN) fits the allocation-free entry point's 2 MiB scratch.
+    to SIG_MAX_D_IN) fits the allocation-free entry point's 4 MiB scratch.
 
     The gated MLP's workspace is the sum of a term that depends only on d_ff
     (the gate/up product's counters and partials, and the hidden vector) and
@@ -323,7 +323,7 @@ def test_noalloc_scratch_covers_every_accepted_shape(lib):
     checked on a spread of pairs first, so that a change that couples the two
     terms fails here instead of hiding an oversize shape."""
     ws = lib.sig_workspace_bytes
-    OP_GATED_MLP, LIMIT, MAX_D = 3, 2 << 20, 131072
+    OP_GATED_MLP, LIMIT, MAX_D = 3, 4 << 20, 131072
     sizes = range(8, MAX_D + 1, 8)
     base = ws(OP_GATED_MLP, 8, 8, 0)
     f = {d: ws(OP_GATED_MLP, 8, d, 0) - base for d in sizes}      # d_ff term

@@ -69,6 +69,20 @@ def test_empty_and_full_masks(sig):
     assert np.all(y2.view(np.uint16) == 0)
 
 
+def test_wide_slice_path(sig):
+    """d_out above 296 column tiles: one slice per tile, so a slice owns all
+    257 input groups and the prologue takes the chunked path of mask words
+    and per-chunk placement (the one-group-per-thread path stops at 256)."""
+    p = workloads.projection("w", 2056, 76032, sigma=0.02, dist="laplace", seed=19,
+                             sparsities=(0.5,))
+    t = p.thresholds[0.5]
+    cols = np.concatenate([np.arange(16), np.random.default_rng(3).choice(76032, 240, replace=False),
+                           np.arange(76032 - 16, 76032)])
+    y = to_host(sig.sparse_gemv(to_dev(p.WT), to_dev(p.x), t=t))
+    ref = oracle.sparse_linear(p.WT, p.x, oracle.threshold_mask(p.x, t), cols=cols)
+    assert_within(y[cols], ref["y64"], ref["bound"], "wide slices")
+
+
 def test_index_path_and_fused_path_agree(sig):
     # the two paths split the kept rows differently (interleaved 8-input groups
     # under a threshold, equal runs of an index list), so they agree within the

@@ -95,8 +95,10 @@ def test_sparse_gemm_config(sig, n):
 
 
 @pytest.mark.parametrize("rows,K,N", [(128, 128, 128), (256, 256, 384), (384, 1024, 256),
-                                      (128, 4096, 512), (512, 640, 1280)])
+                                      (128, 4096, 512), (512, 640, 1280), (256, 128, 256),
+                                      (768, 2048, 512), (1280, 384, 256)])
 def test_sparse_gemm_shapes(sig, rows, K, N):
+    """One-CTA tiles (rows or N not a multiple of 256) and CTA-pair tiles."""
     WT, X = workloads.nm_tokens(rows + K + N, rows=rows, d=K, d_out=N)
     for n in (2, 1):
         Y = to_host(sig.nm_act_gemm(to_dev(X), to_dev(WT), n, 4))

@@ -38,6 +38,17 @@ def test_q8_extremes_and_degenerate_masks(sig):
     _check(sig, QT, scale, x, 0.0, "full mask")
 
 
+def test_q8_wide_slice_path(sig):
+    """More than 296 column tiles of 512: one slice per tile, 257 input groups
+    per slice, so the prologue takes the chunked path of mask words."""
+    QT, scale, x, ts = workloads.q8_projection(seed=18, d_in=2056, d_out=152576)
+    cols = np.concatenate([np.arange(16), np.random.default_rng(2).choice(152576, 240, replace=False),
+                           np.arange(152576 - 16, 152576)])
+    y = to_host(sig.sparse_gemv_q8(to_dev(QT), to_dev(scale), to_dev(x), ts[0.5]))
+    ref = oracle.q8_sparse_linear(QT, scale, x, oracle.threshold_mask(x, ts[0.5]), cols=cols)
+    assert_within(y[cols], ref["y64"], ref["bound"], "wide slices")
+
+
 def test_q8_deterministic(sig):
     QT, scale, x, ts = workloads.q8_projection(seed=4)
     dQ, ds, dx = to_dev(QT), to_dev(scale), to_dev(x)

@@ -775,3 +775,45 @@ def test_teal_mlp_reductions():
     g0, u0, h0 = oracle.rana_hidden(x0, WgT, WuT)
     assert np.array_equal(part["h16"].view(np.uint16), h0.view(np.uint16))
     assert np.array_equal(part["mask"], oracle.threshold_mask(h0, 0.3))
+
+
+def test_e4m3_decode_matches_the_library_format_and_closed_forms():
+    """Every one of the 256 e4m3 codes against torch's float8_e4m3fn (an
+    independent implementation of the same published format), plus values
+    worked out by hand from the definition."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_value(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    ok = ~np.isnan(ours)
+    assert np.array_equal(ours[ok], lib[ok])
+    assert np.array_equal(np.signbit(ours[ok]), np.signbit(lib[ok]))
+    v = oracle.e4m3_value
+    assert v(0x38) == 1.0 and v(0xB8) == -1.0          # exponent 7 = bias, mantissa 0
+    assert v(0x7E) == 448.0                             # largest finite: 2^8 * 1.75
+    assert v(0x01) == 2.0 ** -9 and v(0x08) == 2.0 ** -6   # smallest subnormal, smallest normal
+    assert v(0x07) == 7 * 2.0 ** -9                     # largest subnormal
+    assert np.isnan(v(0x7F)) and np.isnan(v(0xFF)) and np.signbit(v(0x80))
+    pos = ours[:0x7F]
+    assert (np.diff(pos) > 0).all()                    # codes 0 .. 0x7E increase
+
+
+def test_f8_product_is_the_fp16_product_on_exact_decoded_weights():
+    """With every scale 1 the fp8 product equals the plain masked product on
+    the decoded weights, and the per-column scale multiplies column j."""
+    rng = np.random.default_rng(12)
+    QT = rng.integers(0, 256, (40, 24), dtype=np.uint8)
+    QT[(QT & 0x7F) == 0x7F] = 0x38                      # no NaN codes
+    x = rng.laplace(0, 1, 40).astype(np.float16)
+    m = oracle.threshold_mask(x, 0.7)
+    W = oracle.e4m3_value(QT)
+    ref = oracle.masked_matvec(W, x, m)
+    out = oracle.f8_sparse_linear(QT, np.ones(24, np.float32), x, m)
+    assert np.allclose(out["y64"], ref[0], rtol=0, atol=0)
+    sc = rng.uniform(0.5, 2.0, 24).astype(np.float32)
+    out2 = oracle.f8_sparse_linear(QT, sc, x, m)
+    assert np.array_equal(out2["y64"], ref[0] * sc.astype(np.float64))
+    brute = np.array([sum(float(W[i, j]) * float(x[i]) for i in range(40) if m[i]) for j in range(24)])
+    assert np.allclose(out["y64"], brute, rtol=1e-12, atol=1e-12)
+

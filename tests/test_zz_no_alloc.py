@@ -64,12 +64,12 @@ def test_noalloc_matches_gated_mlp_twice_in_a_row(sig):
 
 
 def test_noalloc_rejects_sizes_beyond_its_maximum(sig):
-    """The largest accepted d_ff fits the 2 MiB array; one step beyond is
+    """The largest accepted d_ff fits the 4 MiB array; one step beyond is
     rejected with SIG_ERR_SHAPE.  Real (small) device buffers back every
     pointer, so nothing could fault even if the size checks did not stop it."""
     import torch
     d_model, d_ff = 8, 131072 + 8
-    assert sig.workspace_bytes(sig.OP_GATED_MLP, d_model, 131072) <= 2 << 20
+    assert sig.workspace_bytes(sig.OP_GATED_MLP, d_model, 131072) <= 4 << 20
     x = torch.zeros(d_model, dtype=torch.float16, device="cuda")
     Wg = torch.zeros((d_model, d_ff), dtype=torch.float16, device="cuda")
     Wu = torch.zeros_like(Wg)

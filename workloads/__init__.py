@@ -211,6 +211,28 @@ def q8_projection(seed: int = 0, d_in: int = 4096, d_out: int = 11008, q_sigma: 
     return QT, scale, x, {s: quantile_threshold(x, s) for s in sparsities}
 
 
+def f8_projection(seed: int = 0, d_in: int = 4096, d_out: int = 11008, q_sigma: float = 64.0,
+                  w_sigma: float = 0.02, sparsities=(0.5,)):
+    """An fp8 (e4m3) weight as a quantised checkpoint holds it, then x ~ Laplace(0, 1).
+
+    QT (d_in, d_out) uint8 e4m3 codes: N(0, q_sigma^2) clipped to the format's
+    range [-448, 448] and rounded to the nearest e4m3 value (torch's float8_e4m3fn
+    conversion); scale (d_out,) float32: w_sigma / q_sigma times U(0.9, 1.1).
+    Returns (QT, scale, x, {sparsity: t}).
+    """
+    import torch
+    rng = np.random.default_rng(seed)
+    QT = np.empty((d_in, d_out), dtype=np.uint8)
+    flat = QT.reshape(-1)
+    for lo in range(0, flat.size, _CHUNK):
+        hi = min(flat.size, lo + _CHUNK)
+        v = np.clip(rng.normal(0.0, q_sigma, hi - lo), -448.0, 448.0).astype(np.float32)
+        flat[lo:hi] = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    scale = (w_sigma / q_sigma * rng.uniform(0.9, 1.1, d_out)).astype(np.float32)
+    x = draw_vector(rng, d_in, "laplace")
+    return QT, scale, x, {s: quantile_threshold(x, s) for s in sparsities}
+
+
 @dataclass
 class RankAdapter:
     BT: np.ndarray    # (d_in, r) fp16: B transposed
