@@ -303,8 +303,9 @@ SIG_API int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out,
  *   QT [d_in x d_out] int8 (transposed: row i multiplies x_i), 16-byte aligned.
  *   scale [d_out] float32.  x [d_in] fp16.  y [d_out] fp16 out.
  *   ws sig_workspace_bytes(SIG_OP_SPARSE_GEMV_Q8, d_in, d_out, 0) bytes
- *      (0 means none is needed), 256-byte aligned, zeroed once before first use.
- * d_out % 16 == 0 (whole 16-byte lanes of a row), d_in <= SIG_MAX_D_IN.
+ *      (0 means none is needed), 256-byte aligned, zeroed before first use and
+ *      serving this shape only (see sig_workspace_init).
+ * d_out % 8 == 0 (whole 8-byte lanes of eight weights), d_in <= SIG_MAX_D_IN.
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE, SIG_ERR_ALIGN, SIG_ERR_WORKSPACE, SIG_ERR_CUDA.
  */
 SIG_API int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,

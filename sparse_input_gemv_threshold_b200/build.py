@@ -19,7 +19,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["api.cu", "gemv.cu", "gemv_batch.cu", "gemv_q8.cu", "mask.cu", "nm_gemm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "gemv.cu", "gemv_batch.cu", "mask.cu", "nm_gemm.cu", "noalloc.cu"]
 LIB = os.path.join(PKG, "libsig.so")
 
 NVCC_FLAGS = [

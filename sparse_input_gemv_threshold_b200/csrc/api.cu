@@ -4,7 +4,6 @@
 // returns at once.
 #include "../../include/sig.h"
 #include "internal.h"
-#include "gemv_q8.h"
 #include "nm_ex.h"
 
 #include <cuda_runtime.h>
@@ -78,8 +77,8 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
       return plan_gemv_batch(d_in, d_out, (int)rows).ws_bytes();
     case SIG_OP_SPARSE_GEMV_Q8:
     case SIG_OP_SPARSE_GEMV_F8:
-      if (check_gemv_shape(d_in, d_out) != SIG_OK || d_out % 16 != 0) return 0;
-      return plan_gemv_q8(d_in, d_out).ws_bytes();
+      if (check_gemv_shape(d_in, d_out) != SIG_OK) return 0;
+      return plan_gemv(d_in, d_out, false).ws_bytes();
     case SIG_OP_NM_GEMM:
       if (rows < 1 || d_in < 1) return 0;
       return round_up((size_t)rows * (size_t)d_in * 2, 256);   // the masked activation block
@@ -184,19 +183,20 @@ int sparse_gemv_batch(const uint16_t* WT, int64_t d_in, int64_t d_out, const uin
 
 namespace {
 
-int quantised_gemv(int fmt, const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+int quantised_gemv(int epi, const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
                    const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                    sig_stream_t stream) {
   if (QT == nullptr || scale == nullptr || x == nullptr || y == nullptr) return SIG_ERR_NULL;
   const int sh = check_gemv_shape(d_in, d_out);
   if (sh != SIG_OK) return sh;
-  if (d_out % 16 != 0) return SIG_ERR_SHAPE;
   if (!aligned16(QT) || !aligned16(x) || !aligned16(y) || !aligned4(scale)) return SIG_ERR_ALIGN;
-  const GemvPlan p = plan_gemv_q8(d_in, d_out);
+  const GemvPlan p = plan_gemv(d_in, d_out, false);
   if (p.ws_bytes() > 0 && (ws == nullptr || ws_bytes < p.ws_bytes())) return SIG_ERR_WORKSPACE;
   if (ws != nullptr && !aligned256(ws)) return SIG_ERR_ALIGN;
-  return cuda_status(launch_gemv_q8(p, fmt, QT, scale, x, t, y, (int)d_in, (int)d_out, ws,
-                                    (cudaStream_t)stream));
+  GemvLaunch a{};
+  a.QT = QT; a.col_scale = scale; a.y[0] = y; a.d_out[0] = (int)d_out;
+  a.x = x; a.t = t; a.d_in = (int)d_in; a.ws = ws;
+  return cuda_status(launch_gemv(MASK_THRESH, epi, p, a, (cudaStream_t)stream));
 }
 
 }  // namespace
@@ -204,14 +204,14 @@ int quantised_gemv(int fmt, const uint8_t* QT, const float* scale, int64_t d_in,
 int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
                    const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                    sig_stream_t stream) {
-  return quantised_gemv(kFmtInt8, reinterpret_cast<const uint8_t*>(QT), scale, d_in, d_out, x, t, y,
-                        ws, ws_bytes, stream);
+  return quantised_gemv(EPI_SCALE_I8, reinterpret_cast<const uint8_t*>(QT), scale, d_in, d_out, x,
+                        t, y, ws, ws_bytes, stream);
 }
 
 int sparse_gemv_f8(const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
                    const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                    sig_stream_t stream) {
-  return quantised_gemv(kFmtE4M3, QT, scale, d_in, d_out, x, t, y, ws, ws_bytes, stream);
+  return quantised_gemv(EPI_SCALE_E4M3, QT, scale, d_in, d_out, x, t, y, ws, ws_bytes, stream);
 }
 
 size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in) {

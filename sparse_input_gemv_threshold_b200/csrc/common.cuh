@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace sig {
@@ -80,6 +81,52 @@ __device__ __forceinline__ void fma8(float (&acc)[8], const uint4& v, float xv) 
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
     acc[2 * k] = fmaf(f.x, xv, acc[2 * k]);
     acc[2 * k + 1] = fmaf(f.y, xv, acc[2 * k + 1]);
+  }
+}
+
+// 8-byte streaming load of 8-bit weights (not kept in L1, evict-first in L2).
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p, uint64_t pol) {
+  uint2 r;
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.u32 {%0,%1}, [%2], %3;"
+      : "=r"(r.x), "=r"(r.y)
+      : "l"(p), "l"(pol));
+  return r;
+}
+
+// acc[k] += q_k * xv for the eight int8 weights packed in v: each becomes an
+// exact fp16 value (XOR 0x80 gives u = q + 128, a byte permute forms the
+// half 1024 + u, one half2 subtract of 1152 leaves q), then packed float32
+// FMAs (fma.rn.f32x2) two columns at a time.
+__device__ __forceinline__ void fma8_i8(float (&acc)[8], const uint2& v, float xv) {
+  const uint32_t w[2] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u};
+  const __half2 bias = __half2half2(__ushort_as_half((uint16_t)0x6480));   // 1152 = 1024 + 128
+  const float2 x2 = make_float2(xv, xv);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t lo = __byte_perm(w[k], 0x64646464u, 0x4140);   // halves 1024 + u0, 1024 + u1
+    const uint32_t hi = __byte_perm(w[k], 0x64646464u, 0x4342);   // halves 1024 + u2, 1024 + u3
+    const float2 a = __half22float2(__hsub2(*reinterpret_cast<const __half2*>(&lo), bias));
+    const float2 b = __half22float2(__hsub2(*reinterpret_cast<const __half2*>(&hi), bias));
+    const float2 r0 = __ffma2_rn(a, x2, make_float2(acc[4 * k], acc[4 * k + 1]));
+    const float2 r1 = __ffma2_rn(b, x2, make_float2(acc[4 * k + 2], acc[4 * k + 3]));
+    acc[4 * k] = r0.x; acc[4 * k + 1] = r0.y; acc[4 * k + 2] = r1.x; acc[4 * k + 3] = r1.y;
+  }
+}
+
+// The same for eight fp8 e4m3 weights: the hardware converts two codes to an
+// fp16 pair in one instruction (every e4m3 value is exact in fp16).
+__device__ __forceinline__ void fma8_e4m3(float (&acc)[8], const uint2& v, float xv) {
+  const uint32_t w[2] = {v.x, v.y};
+  const float2 x2 = make_float2(xv, xv);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xffffu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+    const float2 r0 = __ffma2_rn(a, x2, make_float2(acc[4 * k], acc[4 * k + 1]));
+    const float2 r1 = __ffma2_rn(b, x2, make_float2(acc[4 * k + 2], acc[4 * k + 3]));
+    acc[4 * k] = r0.x; acc[4 * k + 1] = r0.y; acc[4 * k + 2] = r1.x; acc[4 * k + 3] = r1.y;
   }
 }
 

@@ -1,4 +1,9 @@
-// Split-K sparse-input GEMV y = W (m . x) with the mask step fused ahead of it.
+// Split-K sparse-input GEMV y = W (m . x) with the mask step fused ahead of it,
+// for fp16 weights and for 8-bit (int8 or fp8 e4m3) weights with one float32
+// scale per output column.  The pages leave quantised sparse kernels open
+// (TEAL README, Limitations) and call weight quantisation orthogonal to
+// activation sparsity (Q-Sparse rebuttal, A1 on batched inference): an 8-bit
+// kept row moves d_out bytes instead of 2 d_out.
 //
 // The product reads only the weight rows of the kept inputs ("Adaptive Rank
 // Allocation ... RaNA Adapters", Q5.1: the columns of A that meet a zero mask
@@ -21,7 +26,10 @@
 //      of the lower bits);
 //   2. 8 warps stream the slice's rows of the tile, 8 rows in flight per warp:
 //      16-byte non-allocating loads with an L2 evict-first policy, the
-//      activation value riding along as a broadcast load, fp32 FMA;
+//      activation value riding along as a broadcast load, fp32 FMA (8-bit
+//      weights: 12 rows in flight, 8-byte lanes of eight weights, each made an
+//      exact fp16 value in registers, then packed float32 FMAs; the column
+//      scale multiplies the finished sum);
 //   3. the warps' sums meet in shared memory (fixed order) and the CTA
 //      stores one partial per column as a 64-bit word {value, tag} (tag = the
 //      tile's epoch + 1, read from the workspace at the start) with a relaxed
@@ -66,6 +74,8 @@ struct KArgs {
   const uint16_t* WT2;    // dual partner of WT[0] (gate/up)
   const uint16_t* x;
   const float* scale;
+  const float* col_scale; // 8-bit weights: one float32 per output column
+  const uint8_t* QT;      // 8-bit weights (d_in x d_out bytes), in place of WT[0]
   const int32_t* idx;
   const int32_t* nnz;
   float t;
@@ -282,13 +292,17 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   }
   const int col = (cg - t_first) * kTile + lane * 8;
   const bool col_ok = col < d_out;
+  constexpr bool Q8 = EPI == EPI_SCALE_I8 || EPI == EPI_SCALE_E4M3;   // 8-bit weights
   const uint16_t* wp = wsel + col;
+  const uint8_t* wq = Q8 ? a.QT + col : nullptr;     // 8 weights = 8 bytes per lane
   const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
   const uint64_t pol = l2_evict_first_policy();
   float acc[8], acc2[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) { acc[k] = 0.f; acc2[k] = 0.f; }
-  constexpr int U = DUAL ? 4 : 8;
+  // rows in flight per warp: 4 KB for fp16 (8 rows x 512 B),
+  // 8-bit weights 3 KB (12 rows x 256 B); 2 x 4 rows for the dual product
+  constexpr int U = DUAL ? 4 : (Q8 ? 12 : 8);
 
   for (int cb = 0; cb < n_rows; cb += a.chunk) {
     const int c_lo = lo + cb, c_hi = min(hi, c_lo + a.chunk), cn = c_hi - c_lo;
@@ -315,27 +329,49 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     }
     if (col_ok) {
       for (int j0 = warp; j0 < cn; j0 += kWarps * U) {
-        uint4 v[U], v2[U];
-        uint16_t xh[U];
+        if constexpr (Q8) {
+          uint2 q[U];
+          uint16_t xh[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int j = j0 + kWarps * u;
-          const int r = j < cn ? (MODE == MASK_DENSE ? c_lo + j : sidx[j]) : -1;
-          if (r >= 0) {
-            xh[u] = __ldg(a.x + r);
-            v[u] = ld_stream_v4(wp + (size_t)r * d_out, pol);
-            if (DUAL) v2[u] = ld_stream_v4(wp2 + (size_t)r * d_out, pol);
-          } else {
-            xh[u] = 0;
-            v[u] = make_uint4(0, 0, 0, 0);
-            if (DUAL) v2[u] = make_uint4(0, 0, 0, 0);
+          for (int u = 0; u < U; ++u) {
+            const int j = j0 + kWarps * u;
+            const int r = j < cn ? (MODE == MASK_DENSE ? c_lo + j : sidx[j]) : -1;
+            if (r >= 0) {
+              xh[u] = __ldg(a.x + r);
+              q[u] = ld_stream_v2(wq + (size_t)r * d_out, pol);
+            } else {
+              xh[u] = 0;
+              q[u] = make_uint2(0, 0);
+            }
           }
-        }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const float xv = h2f(xh[u]);
-          fma8(acc, v[u], xv);
-          if (DUAL) fma8(acc2, v2[u], xv);
+          for (int u = 0; u < U; ++u) {
+            if (EPI == EPI_SCALE_I8) fma8_i8(acc, q[u], h2f(xh[u]));
+            else fma8_e4m3(acc, q[u], h2f(xh[u]));
+          }
+        } else {
+          uint4 v[U], v2[U];
+          uint16_t xh[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int j = j0 + kWarps * u;
+            const int r = j < cn ? (MODE == MASK_DENSE ? c_lo + j : sidx[j]) : -1;
+            if (r >= 0) {
+              xh[u] = __ldg(a.x + r);
+              v[u] = ld_stream_v4(wp + (size_t)r * d_out, pol);
+              if (DUAL) v2[u] = ld_stream_v4(wp2 + (size_t)r * d_out, pol);
+            } else {
+              xh[u] = 0;
+              v[u] = make_uint4(0, 0, 0, 0);
+              if (DUAL) v2[u] = make_uint4(0, 0, 0, 0);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const float xv = h2f(xh[u]);
+            fma8(acc, v[u], xv);
+            if (DUAL) fma8(acc2, v2[u], xv);
+          }
         }
       }
     }
@@ -375,14 +411,18 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   const bool colr_ok = colr < e_dout;
   const int dtot = a.d_out_total;
 
-  auto finish = [&](float g, float u) {
-    if (EPI == EPI_STORE) {
-      Y[colr] = f2h_rn(g);
-    } else {
+  // the finished column: fp16(g), fp16(SiLU(g) u) or fp16(s_j g)
+  auto store_col = [&](int cc, float g, float u) {
+    if (EPI == EPI_SILU_MUL) {
       const float sg = g / (1.0f + expf(-g));
-      Y[colr] = f2h_rn(sg * u);
+      Y[cc] = f2h_rn(sg * u);
+    } else if (EPI == EPI_STORE) {
+      Y[cc] = f2h_rn(g);
+    } else {
+      Y[cc] = f2h_rn(g * __ldg(a.col_scale + cc));
     }
   };
+  auto finish = [&](float g, float u) { store_col(colr, g, u); };
 
   if (S == 1) {
     if (colr_ok) finish(p, p2);
@@ -478,12 +518,7 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   if (h == 0 && colc_ok) {
     const float gs = g + half_sum[tid];                      // slices [0, mid) then [mid, S)
     const float us = DUAL ? u + half_sum[kTile / 2 + tid] : 0.f;
-    if (EPI == EPI_STORE) {
-      Y[colc] = f2h_rn(gs);
-    } else {
-      const float sg = gs / (1.0f + expf(-gs));
-      Y[colc] = f2h_rn(sg * us);
-    }
+    store_col(colc, gs, us);
   }
   if (gave_up) atomicOr(&g_gemv_error, 2u);
   if (tid == 0) st_relaxed_u32(a.epochs + cg, tag);   // the next call tags with tag + 1
@@ -552,6 +587,7 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   k.d_out_total = cols;
   if (tiles != p.C) return cudaErrorInvalidValue;
   k.WT2 = a.WT2; k.x = a.x; k.scale = a.scale; k.idx = a.idx; k.nnz = a.nnz;
+  k.col_scale = a.col_scale; k.QT = a.QT;
   k.t = a.t; k.d_in = a.d_in; k.S = p.S; k.chunk = p.chunk;
   const size_t words = round_up((size_t)((a.d_in + 31) / 32) * 4, 16);
   const size_t red = (size_t)kWarps * kTile * 4 * (epi == EPI_SILU_MUL ? 2 : 1);
@@ -562,6 +598,11 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   k.slots = a.ws != nullptr
                 ? reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(a.ws) + p.counters)
                 : nullptr;
+  if (epi == EPI_SCALE_I8 || epi == EPI_SCALE_E4M3) {
+    if (mode != MASK_THRESH || a.n_mat != 1 || a.QT == nullptr) return cudaErrorInvalidValue;
+    if (epi == EPI_SCALE_I8) return launch_t<MASK_THRESH, false, EPI_SCALE_I8>(p, k, stream);
+    return launch_t<MASK_THRESH, false, EPI_SCALE_E4M3>(p, k, stream);
+  }
   if (epi == EPI_SILU_MUL) {
     if (mode == MASK_DENSE) return launch_t<MASK_DENSE, true, EPI_SILU_MUL>(p, k, stream);
     if (mode == MASK_THRESH) return launch_t<MASK_THRESH, true, EPI_SILU_MUL>(p, k, stream);

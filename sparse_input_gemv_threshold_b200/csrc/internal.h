@@ -28,10 +28,12 @@ enum MaskMode : int {
   MASK_SQUARE = 4          // x_i * x_i >= t (RaNA rank adapter masker, one float32 multiply)
 };
 
-// What happens to a finished output column.
+// What happens to a finished output column, and the weight format it implies.
 enum Epilogue : int {
-  EPI_STORE = 0,     // y_j = fp16(sum)
-  EPI_SILU_MUL = 1   // dual product (g, u): h_j = fp16(SiLU(g_j) * u_j)
+  EPI_STORE = 0,      // fp16 weights: y_j = fp16(sum)
+  EPI_SILU_MUL = 1,   // fp16 weights, dual product (g, u): h_j = fp16(SiLU(g_j) * u_j)
+  EPI_SCALE_I8 = 2,   // int8 weights: y_j = fp16(s_j * sum)
+  EPI_SCALE_E4M3 = 3  // fp8 e4m3 weights: y_j = fp16(s_j * sum)
 };
 
 // Launch `kernel` with programmatic stream serialization (see pdl_wait).
@@ -116,6 +118,8 @@ struct GemvLaunch {
   const uint16_t* WT2 = nullptr;         // second weight of the dual (gate, up) product
   const uint16_t* x = nullptr;
   const float* scale = nullptr;          // MASK_THRESH_SCALED
+  const float* col_scale = nullptr;      // EPI_SCALE_*: one float32 per output column
+  const uint8_t* QT = nullptr;           // EPI_SCALE_*: the 8-bit weight (d_in x d_out bytes)
   const int32_t* idx = nullptr;          // MASK_IDX
   const int32_t* nnz = nullptr;          // MASK_IDX
   float t = 0.f;

@@ -164,14 +164,15 @@ def test_q8_validation(lib):
     big = 1 << 30
     assert f(None, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == NULL
     assert f(FAKE, None, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == NULL
-    assert f(FAKE, FAKE, 64, 24, FAKE, 0.0, FAKE, FAKE, big, None) == SHAPE    # d_out % 16
+    assert f(FAKE, FAKE, 64, 20, FAKE, 0.0, FAKE, FAKE, big, None) == SHAPE    # d_out % 8
     assert f(FAKE, FAKE, 0, 64, FAKE, 0.0, FAKE, FAKE, big, None) == SHAPE
     assert f(FAKE_ODD, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == ALIGN
     assert f(FAKE, FAKE + 1, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == ALIGN   # scale alignment
     need = lib.sig_workspace_bytes(7, 64, 64, 0)
     assert need > 0
     assert f(FAKE, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, need - 1, None) == WORKSPACE
-    assert lib.sig_workspace_bytes(7, 64, 24, 0) == 0
+    assert lib.sig_workspace_bytes(7, 64, 20, 0) == 0
+    assert lib.sig_workspace_bytes(8, 64, 64, 0) == need      # fp8: the same plan
 
 
 def test_batch_validation(lib):
