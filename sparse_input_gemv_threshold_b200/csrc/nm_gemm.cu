@@ -127,12 +127,26 @@ __host__ __device__ constexpr uint32_t instr_desc_f16(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);
 }
 
-// Epilogue of one 128 x BN accumulator tile: warp w reads tensor-memory lanes
-// 32w .. 32w+31 (one output row per thread), 32 columns at a time, adds
-// mu * colsum[c] when colsum is given, rounds to fp16 and stores the row.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+// Epilogue of one 128 x BN accumulator tile.  Warp w owns tensor-memory lanes
+// 32w .. 32w+31, one output row per lane: it reads 32 columns at a time
+// (tcgen05.ld), adds mu * colsum[c] when colsum is given, rounds to fp16 and
+// writes its 32 rows into shared memory (`stage`, 32 x BN fp16 = BN/64 boxes
+// of 32 rows x 128 bytes in the 128-byte swizzled order, so that a quarter-warp
+// of 16-byte stores covers all banks), then one lane stores the boxes with TMA
+// (tensor map over Y, box 64 columns x 32 rows) and waits for the bulk stores
+// to complete.  The stores of a warp are contiguous 128-byte rows instead of
+// one 16-byte piece per row and lane.
 template <int BN>
-__device__ __forceinline__ void store_tile(uint32_t tmem, int warp, uint16_t* yrow, float mu,
-                                           const float* colsum) {
+__device__ __forceinline__ void store_tile_tma(uint32_t tmem, int warp, int lane, uint32_t stage,
+                                               const CUtensorMap* mapY, int m0, int n0, float mu,
+                                               const float* colsum) {
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     uint32_t r[32];
@@ -154,16 +168,34 @@ __device__ __forceinline__ void store_tile(uint32_t tmem, int warp, uint16_t* yr
     for (int q = 0; q < 16; ++q) {
       float v0 = __uint_as_float(r[2 * q]), v1 = __uint_as_float(r[2 * q + 1]);
       if (colsum != nullptr) {
-        v0 = fmaf(mu, __ldg(colsum + c + 2 * q), v0);
-        v1 = fmaf(mu, __ldg(colsum + c + 2 * q + 1), v1);
+        v0 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q), v0);
+        v1 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q + 1), v1);
       }
       const __half2 h = __floats2half2_rn(v0, v1);
       p[q] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+    // row `lane` of box c / 64; 16-byte chunk j of the row at (j ^ (row % 8)) * 16
+    const uint32_t row_base = stage + (uint32_t)(c / 64) * 4096u + (uint32_t)lane * 128u;
+    const int j0 = (c % 64) / 8;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t addr = row_base + (uint32_t)(((j0 + q) ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(p[4 * q]),
+                   "r"(p[4 * q + 1]), "r"(p[4 * q + 2]), "r"(p[4 * q + 3])
+                   : "memory");
+    }
   }
+  // the generic-proxy writes become visible to the bulk copy engine
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < BN / 64; ++b)
+      tma_store_2d(mapY, stage + (uint32_t)b * 4096u, n0 + b * 64, m0 + warp * 32);
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+  __syncwarp();
 }
 
 template <int BN>
@@ -181,7 +213,7 @@ struct __align__(1024) GemmSmem {
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                uint16_t* __restrict__ Y, int M, int N, int K, const float* __restrict__ shift,
+                const __grid_constant__ CUtensorMap mapY, int M, int N, int K, const float* __restrict__ shift,
                 const float* __restrict__ colsum) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the dynamic window starts 1024-aligned only by request; align by hand
@@ -284,9 +316,10 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (acc_done && !*abort_flag) {
     const int row = m0 + warp * 32 + lane;
-    store_tile<BN>(tmem, warp, Y + (size_t)row * N + n0,
-                   shift != nullptr ? __ldg(shift + row) : 0.f,   // the per-token shift added back
-                   shift != nullptr ? colsum + n0 : nullptr);
+    // the B stages are free once the accumulator is complete: 32 x BN fp16 per warp
+    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]) + (uint32_t)warp * (32u * BN * 2u), &mapY,
+                       m0, n0, shift != nullptr ? __ldg(shift + row) : 0.f,   // the shift added back
+                       shift != nullptr ? colsum : nullptr);
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -368,7 +401,8 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-               const uint8_t* __restrict__ meta, uint16_t* __restrict__ Y, int M, int N, int K) {
+               const uint8_t* __restrict__ meta, const __grid_constant__ CUtensorMap mapY, int M,
+               int N, int K) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SpSmem<BN>& sm = *reinterpret_cast<SpSmem<BN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -469,7 +503,8 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncwarp();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (acc_done && !*abort_flag)
-    store_tile<BN>(tmem, warp, Y + (size_t)(m0 + warp * 32 + lane) * N + n0, 0.f, nullptr);
+    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]) + (uint32_t)warp * (32u * BN * 2u), &mapY,
+                       m0, n0, 0.f, nullptr);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (tid == 0 && *abort_flag) {
@@ -590,7 +625,8 @@ struct __align__(1024) PairSmem {
 template <bool SPARSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                 const __grid_constant__ CUtensorMap mapE, uint16_t* __restrict__ Y, int M, int N,
+                 const __grid_constant__ CUtensorMap mapE, const __grid_constant__ CUtensorMap mapY,
+                 int M, int N,
                  int K, const float* __restrict__ shift, const float* __restrict__ colsum) {
   using C = PairCfg<SPARSE>;
   constexpr int BN = C::kBN, BK = C::kBK, S = C::kStages;
@@ -709,9 +745,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
       !*abort_flag && ld_cluster_u32(map_to_rank(smem_u32(&sm.abort_flag), rank ^ 1u)) == 0u;
   if (acc_done && pair_ok) {
     const int row = m0 + warp * 32 + lane;
-    store_tile<BN>(tmem, warp, Y + (size_t)row * N + n0,
-                   shift != nullptr ? __ldg(shift + row) : 0.f,
-                   shift != nullptr ? colsum + n0 : nullptr);
+    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]) + (uint32_t)warp * (32u * BN * 2u), &mapY,
+                       m0, n0, shift != nullptr ? __ldg(shift + row) : 0.f,
+                       shift != nullptr ? colsum : nullptr);
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -778,42 +814,50 @@ bool make_map_meta(CUtensorMap* map, const void* base, uint64_t bytes) {
          CUDA_SUCCESS;
 }
 
+// CTA pairs pay off once the weight tile is wide and deep enough that halving
+// its L2 reads matters (measured on B200: 4096 x 4096 x 4096 2:4 GEMM 97 us
+// with pairs against 115 us without; at 4096 x 1024 x 1024 10.9 against
+// 10.2 us).
+bool use_pair(int M, int N, int K) {
+  return M % 256 == 0 && N % 256 == 0 && N >= 2048 && K >= 2048;
+}
+
 template <bool SPARSE>
 cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me,
-                        uint16_t* Y, int M, int N, int K, const float* shift, const float* colsum,
-                        cudaStream_t stream) {
+                        const CUtensorMap& my, int M, int N, int K, const float* shift,
+                        const float* colsum, cudaStream_t stream) {
   const size_t smem = sizeof(PairSmem<SPARSE>) + 1024;
   auto fn = gemm_pair_kernel<SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(M / kBM, N / PairCfg<SPARSE>::kBN);
-  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, me, Y, M, N, K, shift, colsum);
+  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, me, my, M, N, K, shift, colsum);
   if (e != cudaSuccess) return e;
   return cudaPeekAtLastError();
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, uint16_t* Y, int M, int N,
-                      int K, const float* shift, const float* colsum, cudaStream_t stream) {
+cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my, int M,
+                      int N, int K, const float* shift, const float* colsum, cudaStream_t stream) {
   const size_t smem = sizeof(GemmSmem<BN>) + 1024;
   auto fn = gemm_f16_kernel<BN>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(N / BN, M / kBM);
-  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, Y, M, N, K, shift, colsum);
+  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, my, M, N, K, shift, colsum);
   if (e != cudaSuccess) return e;
   return cudaPeekAtLastError();
 }
 
 template <int BN>
 cudaError_t launch_sp_bn(const CUtensorMap& ma, const CUtensorMap& mb, const uint8_t* meta,
-                         uint16_t* Y, int M, int N, int K, cudaStream_t stream) {
+                         const CUtensorMap& my, int M, int N, int K, cudaStream_t stream) {
   const size_t smem = sizeof(SpSmem<BN>) + 1024;
   auto fn = gemm_sp_kernel<BN>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(N / BN, M / kBM);
-  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, meta, Y, M, N, K);
+  e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, meta, my, M, N, K);
   if (e != cudaSuccess) return e;
   return cudaPeekAtLastError();
 }
@@ -825,13 +869,14 @@ cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_
                                   cudaStream_t stream) {
   if (M % kBM != 0 || K % kBK != 0 || N % 128 != 0) return cudaErrorInvalidValue;
   if (shift != nullptr && colsum == nullptr) return cudaErrorInvalidValue;
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, my;
   if (!make_map(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kBK)) return cudaErrorInvalidValue;
-  if (M % 256 == 0 && N % 256 == 0)   // CTA pairs: 256 x 256 tiles, half of B per CTA
-    return launch_pair<false>(ma, mb, ma, Y, M, N, K, shift, colsum, stream);
-  if (N % 256 == 0) return launch_bn<256>(ma, mb, Y, M, N, K, shift, colsum, stream);
-  return launch_bn<128>(ma, mb, Y, M, N, K, shift, colsum, stream);
+  if (!make_map(&my, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N, 32)) return cudaErrorInvalidValue;
+  if (use_pair(M, N, K))   // CTA pairs: 256 x 256 tiles, half of B per CTA
+    return launch_pair<false>(ma, mb, ma, my, M, N, K, shift, colsum, stream);
+  if (N % 256 == 0) return launch_bn<256>(ma, mb, my, M, N, K, shift, colsum, stream);
+  return launch_bn<128>(ma, mb, my, M, N, K, shift, colsum, stream);
 }
 
 cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* WT, uint16_t* Y, int M, int N,
@@ -846,13 +891,15 @@ cudaError_t launch_gemm_sp(const uint16_t* vals, const uint8_t* meta, const uint
   if (!make_map(&ma, vals, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, kBM))
     return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kSpBK)) return cudaErrorInvalidValue;
-  if (M % 256 == 0 && N % 256 == 0) {   // CTA pairs: 256 x 256 tiles, half of B per CTA
+  CUtensorMap my;
+  if (!make_map(&my, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N, 32)) return cudaErrorInvalidValue;
+  if (use_pair(M, N, K)) {   // CTA pairs: 256 x 256 tiles, half of B per CTA
     CUtensorMap me;
     if (!make_map_meta(&me, meta, (uint64_t)M * (uint64_t)K / 8)) return cudaErrorInvalidValue;
-    return launch_pair<true>(ma, mb, me, Y, M, N, K, nullptr, nullptr, stream);
+    return launch_pair<true>(ma, mb, me, my, M, N, K, nullptr, nullptr, stream);
   }
-  if (N % 256 == 0) return launch_sp_bn<256>(ma, mb, meta, Y, M, N, K, stream);
-  return launch_sp_bn<128>(ma, mb, meta, Y, M, N, K, stream);
+  if (N % 256 == 0) return launch_sp_bn<256>(ma, mb, meta, my, M, N, K, stream);
+  return launch_sp_bn<128>(ma, mb, meta, my, M, N, K, stream);
 }
 
 cudaError_t set_wait_limit(long long cycles) {

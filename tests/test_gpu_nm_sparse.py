@@ -96,9 +96,11 @@ def test_sparse_gemm_config(sig, n):
 
 @pytest.mark.parametrize("rows,K,N", [(128, 128, 128), (256, 256, 384), (384, 1024, 256),
                                       (128, 4096, 512), (512, 640, 1280), (256, 128, 256),
-                                      (768, 2048, 512), (1280, 384, 256)])
+                                      (768, 2048, 512), (1280, 384, 256), (256, 2048, 2048),
+                                      (512, 4096, 2304)])
 def test_sparse_gemm_shapes(sig, rows, K, N):
-    """One-CTA tiles (rows or N not a multiple of 256) and CTA-pair tiles."""
+    """One-CTA tiles, and CTA-pair tiles (rows and N multiples of 256, N and K
+    at least 2048)."""
     WT, X = workloads.nm_tokens(rows + K + N, rows=rows, d=K, d_out=N)
     for n in (2, 1):
         Y = to_host(sig.nm_act_gemm(to_dev(X), to_dev(WT), n, 4))

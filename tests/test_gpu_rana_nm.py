@@ -135,7 +135,7 @@ def test_nm_gemm_config(sig, n, m):
 
 @pytest.mark.parametrize("rows,K,N", [(128, 64, 128), (256, 192, 384), (384, 1024, 256),
                                       (128, 4096, 512), (256, 64, 256), (512, 1024, 768),
-                                      (768, 2048, 512)])
+                                      (768, 2048, 512), (256, 2048, 2048), (512, 4096, 2304)])
 def test_nm_gemm_shapes(sig, rows, K, N):
     WT, X = workloads.nm_tokens(rows + K + N, rows=rows, d=K, d_out=N)
     for n, m in ((2, 4), (4, 4)):
