@@ -32,6 +32,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import tempfile
@@ -62,8 +63,9 @@ def parse():
                     help="for ncu: run only this kernel case eagerly and exit "
                          "(a Llama-2-7B projection name or launch group such as 'q|k|v' or "
                          "'gate|up' at 50%%, 'topk70b', 'batchB' (B tokens, 4096->11008), "
-                         "'q8up70b', 'nm2:4', 'nmsp2:4' (packed 2:4 operand, sparse GEMM) or "
-                         "'nmex2:4')")
+                         "'q8up70b' / 'f8up70b' (int8 / fp8 weights, 8192->28672), "
+                         "'nmN:M' (N:M mask + GEMM, e.g. 'nm8:16'), 'nmsp2:4' (packed 2:4 "
+                         "operand, sparse GEMM) or 'nmex2:4')")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     args = ap.parse_args()
     # at least three untimed warm-up steps; the JSON line reports the number run
@@ -1154,14 +1156,16 @@ def profile_case(args):
         union = int((np.abs(X.astype(np.float32)) >= t).any(axis=0).sum())
         info = {"case": case, "launches": args.launches, "copies": copies,
                 "algorithmic_bytes_per_launch": union * 2 * WT.shape[1] + B * 2 * sum(WT.shape)}
-    elif case == "q8up70b":
-        QT, scale, x, ts = workloads.q8_projection(seed=args.seed, d_in=8192, d_out=28672)
+    elif case in ("q8up70b", "f8up70b"):
+        make, run = ((workloads.q8_projection, sig.sparse_gemv_q8) if case == "q8up70b"
+                     else (workloads.f8_projection, sig.sparse_gemv_f8))
+        QT, scale, x, ts = make(seed=args.seed, d_in=8192, d_out=28672)
         copies = 3
         Qs = [torch.from_numpy(QT).cuda()]
         Qs += [Qs[0].clone() for _ in range(copies - 1)]
         sd, xd = torch.from_numpy(scale).cuda(), torch.from_numpy(x).cuda()
         for i in range(args.launches):
-            sig.sparse_gemv_q8(Qs[i % copies], sd, xd, ts[0.5])
+            run(Qs[i % copies], sd, xd, ts[0.5])
         nnz = int((np.abs(x.astype(np.float32)) >= ts[0.5]).sum())
         info = {"case": case, "launches": args.launches, "copies": copies,
                 "algorithmic_bytes_per_launch": nnz * 28672 + 2 * 8192 + 2 * 28672}
@@ -1184,11 +1188,12 @@ def profile_case(args):
             sig.sparsify_nm_packed(Xs[i % copies], n, out=pk[i % copies])
             sig.nm_act_gemm_packed(pk[i % copies], X.shape[0], X.shape[1], Wd)
         info = {"case": case, "launches": args.launches}
-    elif case == "nm2:4":
+    elif re.fullmatch(r"nm\d+:\d+", case):
+        n, m = (int(v) for v in case[2:].split(":"))
         WT, X = workloads.nm_tokens(args.seed)
         Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()
         for _ in range(args.launches):
-            Y = sig.nm_act_gemm(Xd, Wd, 2, 4)
+            Y = sig.nm_act_gemm(Xd, Wd, n, m)
         info = {"case": case, "launches": args.launches}
     elif case == "topk70b":
         (p,) = workloads.qsparse_70b(args.seed, names=("down",))
