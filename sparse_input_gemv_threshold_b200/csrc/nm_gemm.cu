@@ -3,15 +3,16 @@
 // block (tokens x K, K contiguous), B is the transposed weight WT (K x N,
 // N contiguous), Y is tokens x N in fp16 with float32 accumulation.
 //
-// sm_100a design: one CTA per 128 x BN output tile, 128 threads.
+// sm_100a design: one CTA per 128 x BN output tile, 256 threads.
 //   - thread 0 streams 64-wide K slices of A and B into a 4-stage shared
 //     ring with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast),
 //     signalling an mbarrier with the transaction byte count;
 //   - thread 32 issues tcgen05.mma (kind::f16, M = 128, N = BN, K = 16) from
 //     shared-memory descriptors into a float32 accumulator in tensor memory
 //     and frees each stage with tcgen05.commit;
-//   - all four warps then read their 32 accumulator lanes with tcgen05.ld,
-//     round to fp16 and store.
+//   - all eight warps then read the accumulator with tcgen05.ld (each its
+//     lane quarter and column half), round to fp16 and store through shared
+//     memory with TMA.
 // Launched with programmatic stream serialization: the launch, the mbarrier
 // setup and the tensor-memory allocation overlap the end of the kernel before
 // it; every thread then waits for that kernel (griddepcontrol.wait) before it
@@ -44,7 +45,15 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;          // one 128-byte swizzle row of fp16
 constexpr int kStages = 4;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;   // warp 0 loads, warp 1 issues MMAs, all eight store
+// Register cap of the GEMM kernels (64 per thread, the bound that four CTAs of
+// 256 threads per SM would impose; shared memory allows one).  A GEMM CTA
+// launched early behind the mask kernel before it (programmatic dependent
+// launch) sits on an SM while that kernel still runs; 16 K registers leave
+// the mask kernel six of its eight CTAs per SM, where the uncapped 90-128
+// registers halved them (measured on B200: 2:4 and 8:16 mask + GEMM at
+// 16384 x 4096 x 4096 slower by 85 us).
+constexpr int kMinBlocksForRegs = 4;
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -134,23 +143,28 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                : "memory");
 }
 
-// Epilogue of one 128 x BN accumulator tile.  Warp w owns tensor-memory lanes
-// 32w .. 32w+31, one output row per lane: it reads 32 columns at a time
-// (tcgen05.ld), adds mu * colsum[c] when colsum is given, rounds to fp16 and
-// writes its 32 rows into shared memory (`stage`, 32 x BN fp16 = BN/64 boxes
-// of 32 rows x 128 bytes in the 128-byte swizzled order, so that a quarter-warp
-// of 16-byte stores covers all banks), then one lane stores the boxes with TMA
-// (tensor map over Y, box 64 columns x 32 rows) and waits for the bulk stores
-// to complete.  The stores of a warp are contiguous 128-byte rows instead of
-// one 16-byte piece per row and lane.
+// Epilogue of one 128 x BN accumulator tile by the CTA's eight warps.  Warp w
+// reads tensor-memory lanes 32 (w % 4) .. 32 (w % 4) + 31 (one output row per
+// lane) and the columns of half w / 4 of the tile, 32 at a time (tcgen05.ld,
+// wait), adds mu * colsum[c] when colsum is given, rounds to fp16 and writes
+// the row's 64 bytes into the warp's staging area in shared memory
+// (`stage_base` + w x 32 x BN fp16) in the 128-byte swizzled order of the
+// output tensor map (box 64 columns x 32 rows), so that a quarter-warp of
+// 16-byte stores covers all banks.  After every 64 columns one lane stores
+// the block with TMA while the warp goes on to the next, and at the end waits
+// only until the bulk stores have read shared memory.
 template <int BN>
-__device__ __forceinline__ void store_tile_tma(uint32_t tmem, int warp, int lane, uint32_t stage,
+__device__ __forceinline__ void store_tile_tma(uint32_t tmem, int warp, int lane, uint32_t stage_base,
                                                const CUtensorMap* mapY, int m0, int n0, float mu,
                                                const float* colsum) {
+  constexpr int kCols = BN / 2;                       // columns per warp
+  const int q = warp & 3, c0 = (warp >> 2) * kCols;
+  const uint32_t stage = stage_base + (uint32_t)warp * (32u * kCols * 2u);
+  const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-  for (int c = 0; c < BN; c += 32) {
+  for (int cc = 0; cc < kCols; cc += 32) {
+    const int c = c0 + cc;
     uint32_t r[32];
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c;
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -161,40 +175,41 @@ __device__ __forceinline__ void store_tile_tma(uint32_t tmem, int warp, int lane
           "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
-        : "r"(taddr));
+        : "r"(lane_addr + (uint32_t)c));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
     uint32_t p[16];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      float v0 = __uint_as_float(r[2 * q]), v1 = __uint_as_float(r[2 * q + 1]);
+    for (int k = 0; k < 16; ++k) {
+      float v0 = __uint_as_float(r[2 * k]), v1 = __uint_as_float(r[2 * k + 1]);
       if (colsum != nullptr) {
-        v0 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q), v0);
-        v1 = fmaf(mu, __ldg(colsum + n0 + c + 2 * q + 1), v1);
+        v0 = fmaf(mu, __ldg(colsum + n0 + c + 2 * k), v0);
+        v1 = fmaf(mu, __ldg(colsum + n0 + c + 2 * k + 1), v1);
       }
       const __half2 h = __floats2half2_rn(v0, v1);
-      p[q] = *reinterpret_cast<const uint32_t*>(&h);
+      p[k] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    // row `lane` of box c / 64; 16-byte chunk j of the row at (j ^ (row % 8)) * 16
-    const uint32_t row_base = stage + (uint32_t)(c / 64) * 4096u + (uint32_t)lane * 128u;
-    const int j0 = (c % 64) / 8;
+    // row `lane` of block cc / 64; 16-byte chunk j of the row at (j ^ (row % 8)) * 16
+    const uint32_t row_base = stage + (uint32_t)(cc / 64) * 4096u + (uint32_t)lane * 128u;
+    const int j0 = (cc % 64) / 8;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t addr = row_base + (uint32_t)(((j0 + q) ^ (lane & 7)) << 4);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(p[4 * q]),
-                   "r"(p[4 * q + 1]), "r"(p[4 * q + 2]), "r"(p[4 * q + 3])
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t addr = row_base + (uint32_t)(((j0 + j) ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(p[4 * j]),
+                   "r"(p[4 * j + 1]), "r"(p[4 * j + 2]), "r"(p[4 * j + 3])
                    : "memory");
     }
+    if (cc % 64 == 32) {
+      // the generic-proxy writes become visible to the bulk copy engine
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(mapY, stage + (uint32_t)(cc / 64) * 4096u, n0 + c - 32, m0 + q * 32);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    }
   }
-  // the generic-proxy writes become visible to the bulk copy engine
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncwarp();
-  if (lane == 0) {
-#pragma unroll
-    for (int b = 0; b < BN / 64; ++b)
-      tma_store_2d(mapY, stage + (uint32_t)b * 4096u, n0 + b * 64, m0 + warp * 32);
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-  }
+  // shared memory may be reused or released once the stores have read it
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   __syncwarp();
 }
 
@@ -211,7 +226,7 @@ struct __align__(1024) GemmSmem {
 };
 
 template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kMinBlocksForRegs)
 gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                 const __grid_constant__ CUtensorMap mapY, int M, int N, int K, const float* __restrict__ shift,
                 const float* __restrict__ colsum) {
@@ -315,9 +330,9 @@ gemm_f16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   __syncwarp();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (acc_done && !*abort_flag) {
-    const int row = m0 + warp * 32 + lane;
+    const int row = m0 + (warp & 3) * 32 + lane;
     // the B stages are free once the accumulator is complete: 32 x BN fp16 per warp
-    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]) + (uint32_t)warp * (32u * BN * 2u), &mapY,
+    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]), &mapY,
                        m0, n0, shift != nullptr ? __ldg(shift + row) : 0.f,   // the shift added back
                        shift != nullptr ? colsum : nullptr);
   }
@@ -399,7 +414,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kMinBlocksForRegs)
 gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                const uint8_t* __restrict__ meta, const __grid_constant__ CUtensorMap mapY, int M,
                int N, int K) {
@@ -503,8 +518,7 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncwarp();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (acc_done && !*abort_flag)
-    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]) + (uint32_t)warp * (32u * BN * 2u), &mapY,
-                       m0, n0, 0.f, nullptr);
+    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]), &mapY, m0, n0, 0.f, nullptr);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (tid == 0 && *abort_flag) {
@@ -623,7 +637,7 @@ struct __align__(1024) PairSmem {
 };
 
 template <bool SPARSE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, kMinBlocksForRegs)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                  const __grid_constant__ CUtensorMap mapE, const __grid_constant__ CUtensorMap mapY,
                  int M, int N,
@@ -744,8 +758,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
   const bool pair_ok =
       !*abort_flag && ld_cluster_u32(map_to_rank(smem_u32(&sm.abort_flag), rank ^ 1u)) == 0u;
   if (acc_done && pair_ok) {
-    const int row = m0 + warp * 32 + lane;
-    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]) + (uint32_t)warp * (32u * BN * 2u), &mapY,
+    const int row = m0 + (warp & 3) * 32 + lane;
+    store_tile_tma<BN>(tmem, warp, lane, smem_u32(sm.B[0]), &mapY,
                        m0, n0, shift != nullptr ? __ldg(shift + row) : 0.f,
                        shift != nullptr ? colsum : nullptr);
   }
