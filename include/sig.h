@@ -81,7 +81,8 @@ typedef enum {
   SIG_OP_RANK_ADAPTER = 5, /* rank_adapter_sparse(d_in, d_out, rows = r) */
   SIG_OP_SPARSE_GEMV_BATCH = 6, /* sparse_gemv_batch(d_in, d_out, rows = tokens) */
   SIG_OP_SPARSE_GEMV_Q8 = 7,    /* sparse_gemv_q8(d_in, d_out)              */
-  SIG_OP_SPARSE_GEMV_F8 = 8     /* sparse_gemv_f8(d_in, d_out)              */
+  SIG_OP_SPARSE_GEMV_F8 = 8,    /* sparse_gemv_f8(d_in, d_out)              */
+  SIG_OP_SPARSE_GEMV_Q4 = 9     /* sparse_gemv_q4(d_in, d_out)              */
 } sig_op;
 
 /* Largest activation length the fused mask prologue accepts. */
@@ -323,6 +324,21 @@ SIG_API int sparse_gemv_q8(const int8_t* QT, const float* scale, int64_t d_in, i
  * and errors as sparse_gemv_q8.
  */
 SIG_API int sparse_gemv_f8(const uint8_t* QT, const float* scale, int64_t d_in, int64_t d_out,
+                           const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                           sig_stream_t stream);
+
+/*
+ * The same product with int4 weights, two to a byte: QT4 is d_in x d_out / 2
+ * bytes, row-major; byte b of row i holds q[i, 2b] in bits 0..3 and
+ * q[i, 2b + 1] in bits 4..7, each a two's-complement value in [-8, 7];
+ * W[j, i] = s_j q[i, j]:
+ *   y_j = fp16( s_j * sum_{i: m_i} q[i, j] x_i )      (float32 accumulation)
+ * A kept input costs d_out / 2 bytes.  Workspace
+ * (sig_workspace_bytes(SIG_OP_SPARSE_GEMV_Q4, d_in, d_out, 0)), shape rules
+ * (d_out % 8 == 0: whole 4-byte lanes of eight weights) and errors as
+ * sparse_gemv_q8; QT4 16-byte aligned.
+ */
+SIG_API int sparse_gemv_q4(const uint8_t* QT4, const float* scale, int64_t d_in, int64_t d_out,
                            const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                            sig_stream_t stream);
 

@@ -88,7 +88,7 @@ __all__ = [
     "rank_adapter_hidden", "rank_adapter_scores", "rank_adapter",
     "union_mask", "batched_sparse_linear", "q8_sparse_linear", "teal_mlp",
     "pts_shift", "wt_scores", "nm_mask_by_score", "var_gamma", "nm_variant", "nm_variant_gemm",
-    "nm_pack_2of4", "e4m3_value", "f8_sparse_linear",
+    "nm_pack_2of4", "e4m3_value", "f8_sparse_linear", "int4_values", "q4_sparse_linear",
 ]
 
 
@@ -488,6 +488,36 @@ def f8_sparse_linear(QT, scale, x, mask, cols=None) -> dict:
     if cols is not None:
         QT, s64 = QT[:, np.asarray(cols)], s64[np.asarray(cols)]
     Q64 = e4m3_value(QT)
+    xm = np.where(np.asarray(mask, dtype=bool), np.asarray(x, dtype=np.float64), 0.0)
+    y64 = (xm @ Q64) * s64
+    bound = (np.abs(xm) @ np.abs(Q64)) * np.abs(s64)
+    idx = compact(mask)
+    return {"mask": np.asarray(mask, dtype=bool), "idx": idx, "nnz": int(idx.size),
+            "y64": y64, "y16": fp16(y64), "bound": bound}
+
+
+def int4_values(packed) -> np.ndarray:
+    """The int4 weights held two to a byte: byte b of a row carries weight 2b
+    in bits 0..3 and weight 2b + 1 in bits 4..7, each a 4-bit two's-complement
+    integer in [-8, 7].  (d_in, d_out / 2) uint8 in, (d_in, d_out) int8 out."""
+    p = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    lo, hi = p & 0xF, p >> 4
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[..., 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return out.astype(np.int8)
+
+
+def q4_sparse_linear(QT4, scale, x, mask, cols=None) -> dict:
+    """y_j = s_j * sum_i q[i, j] * (m_i ? x_i : 0) in float64 with int4 weights
+    q (packed two to a byte, :func:`int4_values`) and one float32 scale per
+    output column: the weight-quantised product of :func:`q8_sparse_linear`
+    with 4-bit weights in place of 8-bit ones."""
+    Q = int4_values(QT4)
+    s64 = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    if cols is not None:
+        Q, s64 = Q[:, np.asarray(cols)], s64[np.asarray(cols)]
+    Q64 = Q.astype(np.float64)
     xm = np.where(np.asarray(mask, dtype=bool), np.asarray(x, dtype=np.float64), 0.0)
     y64 = (xm @ Q64) * s64
     bound = (np.abs(xm) @ np.abs(Q64)) * np.abs(s64)

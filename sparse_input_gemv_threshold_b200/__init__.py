@@ -26,7 +26,7 @@ __all__ = [
     "OP_SPARSE_GEMV_BATCH", "MAX_BATCH", "sparse_gemv_batch", "OP_SPARSE_GEMV_Q8",
     "sparse_gemv_q8", "sparsify_nm_ex", "nm_act_gemm_ex", "col_sums", "teal_mlp_sparse",
     "nm_packed_bytes", "sparsify_nm_packed", "nm_act_gemm_packed", "sparse_gemv_f8",
-    "OP_SPARSE_GEMV_F8", "set_wait_limit",
+    "OP_SPARSE_GEMV_F8", "set_wait_limit", "sparse_gemv_q4", "OP_SPARSE_GEMV_Q4",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsig.so")
@@ -35,6 +35,7 @@ OP_SPARSE_GEMV, OP_TOPK, OP_GATED_MLP, OP_NM_GEMM, OP_RANK_ADAPTER = 1, 2, 3, 4,
 OP_SPARSE_GEMV_BATCH = 6
 OP_SPARSE_GEMV_Q8 = 7
 OP_SPARSE_GEMV_F8 = 8
+OP_SPARSE_GEMV_Q4 = 9
 MAX_BATCH = 16
 MAX_D_IN = 131072
 
@@ -64,6 +65,7 @@ _SIGNATURES = {
     "sparse_gemv_batch": (_i32, [_p, _i64, _i64, _p, _i64, _f32, _p, _p, _sz, _p]),
     "sparse_gemv_q8": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
     "sparse_gemv_f8": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
+    "sparse_gemv_q4": (_i32, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _sz, _p]),
     "sparsify_nm_ex": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _p]),
     "nm_act_gemm_ex": (_i32, [_p, _i64, _i64, _p, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p, _sz,
                               _p]),
@@ -381,6 +383,27 @@ def sparse_gemv_f8(QT, scale, x, t: float, y=None, ws=None, stream=None):
         ws = workspace(OP_SPARSE_GEMV_F8, d_in, d_out, device=QT.device, stream=stream)
     _check("sparse_gemv_f8", _lib.sparse_gemv_f8(
         _ptr(QT), _ptr(scale), d_in, d_out, _ptr(x), float(t), _ptr(y), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return y
+
+
+def sparse_gemv_q4(QT4, scale, x, t: float, y=None, ws=None, stream=None):
+    """y = W (m . x) with int4 weights packed two to a byte (QT4: uint8,
+    d_in x d_out / 2; the even column in the low nibble) and float32 column
+    scales."""
+    _need(QT4, torch.uint8, "QT4")
+    _need(scale, torch.float32, "scale", QT4.device)
+    _need(x, torch.float16, "x", QT4.device)
+    d_in, half = QT4.shape
+    d_out = 2 * half
+    if x.numel() != d_in or scale.numel() != d_out:
+        raise ValueError("shapes: QT4 (d_in, d_out / 2), scale (d_out), x (d_in)")
+    if y is None:
+        y = torch.empty(d_out, dtype=torch.float16, device=QT4.device)
+    if ws is None:
+        ws = workspace(OP_SPARSE_GEMV_Q4, d_in, d_out, device=QT4.device, stream=stream)
+    _check("sparse_gemv_q4", _lib.sparse_gemv_q4(
+        _ptr(QT4), _ptr(scale), d_in, d_out, _ptr(x), float(t), _ptr(y), _ptr(ws), ws.numel(),
         _stream(stream)))
     return y
 

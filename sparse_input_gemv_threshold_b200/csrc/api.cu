@@ -77,6 +77,7 @@ size_t sig_workspace_bytes(int op, int64_t d_in, int64_t d_out, int64_t rows) {
       return plan_gemv_batch(d_in, d_out, (int)rows).ws_bytes();
     case SIG_OP_SPARSE_GEMV_Q8:
     case SIG_OP_SPARSE_GEMV_F8:
+    case SIG_OP_SPARSE_GEMV_Q4:
       if (check_gemv_shape(d_in, d_out) != SIG_OK) return 0;
       return plan_gemv(d_in, d_out, false).ws_bytes();
     case SIG_OP_NM_GEMM:
@@ -212,6 +213,12 @@ int sparse_gemv_f8(const uint8_t* QT, const float* scale, int64_t d_in, int64_t 
                    const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
                    sig_stream_t stream) {
   return quantised_gemv(EPI_SCALE_E4M3, QT, scale, d_in, d_out, x, t, y, ws, ws_bytes, stream);
+}
+
+int sparse_gemv_q4(const uint8_t* QT4, const float* scale, int64_t d_in, int64_t d_out,
+                   const uint16_t* x, float t, uint16_t* y, void* ws, size_t ws_bytes,
+                   sig_stream_t stream) {
+  return quantised_gemv(EPI_SCALE_I4, QT4, scale, d_in, d_out, x, t, y, ws, ws_bytes, stream);
 }
 
 size_t sig_workspace_bytes_multi(int n_mat, const int64_t* d_out, int64_t d_in) {

@@ -93,6 +93,24 @@ __device__ __forceinline__ uint2 ld_stream_v2(const void* p, uint64_t pol) {
   return r;
 }
 
+// 4-byte streaming load of eight int4 weights (not kept in L1, evict-first in L2).
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p, uint64_t pol) {
+  uint32_t r;
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.u32 %0, [%1], %2;" : "=r"(r) : "l"(p), "l"(pol));
+  return r;
+}
+
+// acc[k] += q_k * xv for the eight int4 weights of w (weight k in bits
+// 4k .. 4k+3, two's complement): each nibble is sign-extended by two shifts
+// and converted to float32 (exact), then one float32 FMA.
+__device__ __forceinline__ void fma8_i4(float (&acc)[8], uint32_t w, float xv) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int q = (int)(w << (28 - 4 * k)) >> 28;           // nibble k, sign-extended
+    acc[k] = fmaf(__int2float_rn(q), xv, acc[k]);
+  }
+}
+
 // acc[k] += q_k * xv for the eight int8 weights packed in v: each byte is
 // sign-extended by two shifts and converted to float32 (exact), then one
 // float32 FMA.  Measured on B200 against a byte-permute into fp16 1024 + u

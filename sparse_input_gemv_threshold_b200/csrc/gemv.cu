@@ -1,9 +1,9 @@
 // Split-K sparse-input GEMV y = W (m . x) with the mask step fused ahead of it,
-// for fp16 weights and for 8-bit (int8 or fp8 e4m3) weights with one float32
-// scale per output column.  The pages leave quantised sparse kernels open
-// (TEAL README, Limitations) and call weight quantisation orthogonal to
+// for fp16 weights and for 8-bit (int8 or fp8 e4m3) or int4 weights with one
+// float32 scale per output column.  The pages leave quantised sparse kernels
+// open (TEAL README, Limitations) and call weight quantisation orthogonal to
 // activation sparsity (Q-Sparse rebuttal, A1 on batched inference): an 8-bit
-// kept row moves d_out bytes instead of 2 d_out.
+// kept row moves d_out bytes instead of 2 d_out, an int4 row d_out / 2.
 //
 // The product reads only the weight rows of the kept inputs ("Adaptive Rank
 // Allocation ... RaNA Adapters", Q5.1: the columns of A that meet a zero mask
@@ -294,16 +294,19 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   const int col = (cg - t_first) * kTile + lane * 8;
   const bool col_ok = col < d_out;
   constexpr bool Q8 = EPI == EPI_SCALE_I8 || EPI == EPI_SCALE_E4M3;   // 8-bit weights
+  constexpr bool Q4 = EPI == EPI_SCALE_I4;                              // int4 weights
   const uint16_t* wp = wsel + col;
   const uint8_t* wq = Q8 ? a.QT + col : nullptr;     // 8 weights = 8 bytes per lane
+  const uint8_t* wq4 = Q4 ? a.QT + col / 2 : nullptr;  // 8 weights = 4 bytes per lane
   const uint16_t* wp2 = DUAL ? a.WT2 + col : nullptr;
   const uint64_t pol = l2_evict_first_policy();
   float acc[8], acc2[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) { acc[k] = 0.f; acc2[k] = 0.f; }
   // rows in flight per warp: 4 KB for fp16 (8 rows x 512 B),
-  // 8-bit weights 3 KB (12 rows x 256 B); 2 x 4 rows for the dual product
-  constexpr int U = DUAL ? 4 : (Q8 ? 12 : 8);
+  // 8-bit weights 3 KB (12 rows x 256 B), int4 weights 2 KB (16 rows x 128 B);
+  // 2 x 4 rows for the dual product
+  constexpr int U = DUAL ? 4 : (Q8 ? 12 : (Q4 ? 16 : 8));
 
   for (int cb = 0; cb < n_rows; cb += a.chunk) {
     const int c_lo = lo + cb, c_hi = min(hi, c_lo + a.chunk), cn = c_hi - c_lo;
@@ -330,7 +333,24 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     }
     if (col_ok) {
       for (int j0 = warp; j0 < cn; j0 += kWarps * U) {
-        if constexpr (Q8) {
+        if constexpr (Q4) {
+          uint32_t q[U];
+          uint16_t xh[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int j = j0 + kWarps * u;
+            const int r = j < cn ? sidx[j] : -1;
+            if (r >= 0) {
+              xh[u] = __ldg(a.x + r);
+              q[u] = ld_stream_u32(wq4 + (size_t)r * (size_t)(d_out / 2), pol);
+            } else {
+              xh[u] = 0;
+              q[u] = 0u;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) fma8_i4(acc, q[u], h2f(xh[u]));
+        } else if constexpr (Q8) {
           uint2 q[U];
           uint16_t xh[U];
 #pragma unroll
@@ -464,7 +484,9 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
   bool gave_up = false;
   float g = 0.f, u = 0.f;
   if (colc_ok) {
-    constexpr int B = DUAL ? 4 : 16;          // words of the column in flight together
+    // words of the column in flight together: a half of up to 20 slices
+    // (37 slices of a 16-tile launch) in one batch for the single product
+    constexpr int B = DUAL ? 4 : (MULTI ? 16 : 20);
     unsigned long long* sl = slots + pbase + c;
     unsigned long long* sl2 = slots2 + pbase + c;
     const long long t0 = clock64();
@@ -546,9 +568,11 @@ GemvPlan plan_gemv_multi(int64_t d_in, const int64_t* d_out, int n_mat, bool dua
     p.C += (int)((d_out[i] + kTile - 1) / kTile);
     total += d_out[i];
   }
-  // narrow launches (fewer than 16 column tiles) may cut the rows finer to
-  // fill the GPU; wider ones stop at 32 slices (one batch of partial loads)
-  const int cap = p.C >= 16 ? 32 : kMaxS;
+  // launches of up to 16 column tiles may cut the rows finer to fill every
+  // CTA slot (16 tiles: 37 slices, 592 CTAs; measured on B200 for 4096 x 4096
+  // at 50 %: 6.53 us against 7.12 us with 32 slices, whose 512 CTAs left some
+  // SMs with two or three); wider ones stop at 32 slices
+  const int cap = p.C > 16 ? 32 : kMaxS;
   p.S = std::max(1, std::min(cap, (kNumSMs * kGemvCtasPerSM) / std::max(1, p.C)));
   // rows per slice: at most ceil(d_in / S) for an index or dense slice, at
   // most 8 ceil(ceil(d_in / 8) / S) for a threshold slice's own groups
@@ -599,9 +623,10 @@ cudaError_t launch_gemv(int mode, int epi, const GemvPlan& p, const GemvLaunch& 
   k.slots = a.ws != nullptr
                 ? reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(a.ws) + p.counters)
                 : nullptr;
-  if (epi == EPI_SCALE_I8 || epi == EPI_SCALE_E4M3) {
+  if (epi == EPI_SCALE_I8 || epi == EPI_SCALE_E4M3 || epi == EPI_SCALE_I4) {
     if (mode != MASK_THRESH || a.n_mat != 1 || a.QT == nullptr) return cudaErrorInvalidValue;
     if (epi == EPI_SCALE_I8) return launch_t<MASK_THRESH, false, EPI_SCALE_I8>(p, k, stream);
+    if (epi == EPI_SCALE_I4) return launch_t<MASK_THRESH, false, EPI_SCALE_I4>(p, k, stream);
     return launch_t<MASK_THRESH, false, EPI_SCALE_E4M3>(p, k, stream);
   }
   if (epi == EPI_SILU_MUL) {

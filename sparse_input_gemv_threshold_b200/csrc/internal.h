@@ -33,7 +33,8 @@ enum Epilogue : int {
   EPI_STORE = 0,      // fp16 weights: y_j = fp16(sum)
   EPI_SILU_MUL = 1,   // fp16 weights, dual product (g, u): h_j = fp16(SiLU(g_j) * u_j)
   EPI_SCALE_I8 = 2,   // int8 weights: y_j = fp16(s_j * sum)
-  EPI_SCALE_E4M3 = 3  // fp8 e4m3 weights: y_j = fp16(s_j * sum)
+  EPI_SCALE_E4M3 = 3, // fp8 e4m3 weights: y_j = fp16(s_j * sum)
+  EPI_SCALE_I4 = 4    // int4 weights, two per byte: y_j = fp16(s_j * sum)
 };
 
 // Launch `kernel` with programmatic stream serialization (see pdl_wait).

@@ -173,6 +173,13 @@ def test_q8_validation(lib):
     assert f(FAKE, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, need - 1, None) == WORKSPACE
     assert lib.sig_workspace_bytes(7, 64, 20, 0) == 0
     assert lib.sig_workspace_bytes(8, 64, 64, 0) == need      # fp8: the same plan
+    assert lib.sig_workspace_bytes(9, 64, 64, 0) == need      # int4: the same plan
+    q4 = lib.sparse_gemv_q4
+    assert q4(None, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == NULL
+    assert q4(FAKE, FAKE, 64, 64, None, 0.0, FAKE, FAKE, big, None) == NULL
+    assert q4(FAKE, FAKE, 64, 20, FAKE, 0.0, FAKE, FAKE, big, None) == SHAPE    # d_out % 8
+    assert q4(FAKE_ODD, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, big, None) == ALIGN
+    assert q4(FAKE, FAKE, 64, 64, FAKE, 0.0, FAKE, FAKE, need - 1, None) == WORKSPACE
 
 
 def test_batch_validation(lib):

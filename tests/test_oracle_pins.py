@@ -777,6 +777,40 @@ def test_teal_mlp_reductions():
     assert np.array_equal(part["mask"], oracle.threshold_mask(h0, 0.3))
 
 
+def test_int4_decode_by_hand_and_by_arithmetic_shifts():
+    """Nibble decoding of the packed int4 weights: bytes worked out by hand
+    (low nibble first), then all 256 bytes against sign extension by an
+    arithmetic right shift of the nibble moved to the top of an int8."""
+    v = oracle.int4_values(np.array([[0x00, 0x7F, 0x80, 0x8F, 0x21, 0xF7]], np.uint8))
+    assert v.tolist() == [[0, 0, -1, 7, 0, -8, -1, -8, 1, 2, 7, -1]]
+    codes = np.arange(256, dtype=np.uint8)
+    lo = (codes << 4).astype(np.uint8).view(np.int8) >> 4
+    hi = codes.view(np.int8) >> 4
+    dec = oracle.int4_values(codes.reshape(1, 256))[0]
+    assert np.array_equal(dec[0::2], lo) and np.array_equal(dec[1::2], hi)
+    assert dec.min() == -8 and dec.max() == 7
+
+
+def test_q4_product_is_the_int8_product_on_the_decoded_weights():
+    """The int4 product equals the (golden-pinned) int8 product on the decoded
+    weights exactly, and a brute-force double loop."""
+    rng = np.random.default_rng(14)
+    QT4 = rng.integers(0, 256, (36, 12), dtype=np.uint8)
+    scale = rng.uniform(0.5, 2.0, 24).astype(np.float32)
+    x = rng.laplace(0, 1, 36).astype(np.float16)
+    m = oracle.threshold_mask(x, 0.6)
+    a = oracle.q4_sparse_linear(QT4, scale, x, m)
+    Q = oracle.int4_values(QT4)
+    b = oracle.q8_sparse_linear(Q, scale, x, m)
+    assert np.array_equal(a["y64"], b["y64"]) and np.array_equal(a["bound"], b["bound"])
+    brute = [float(scale[j]) * sum(int(Q[i, j]) * float(x[i]) for i in range(36) if m[i])
+             for j in range(24)]
+    assert np.allclose(a["y64"], brute, rtol=1e-12, atol=1e-12)
+    cols = np.array([1, 10, 23])
+    c = oracle.q4_sparse_linear(QT4, scale, x, m, cols=cols)
+    assert np.array_equal(c["y64"], a["y64"][cols])
+
+
 def test_e4m3_decode_matches_the_library_format_and_closed_forms():
     """Every one of the 256 e4m3 codes against torch's float8_e4m3fn (an
     independent implementation of the same published format), plus values

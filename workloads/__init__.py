@@ -211,6 +211,29 @@ def q8_projection(seed: int = 0, d_in: int = 4096, d_out: int = 11008, q_sigma: 
     return QT, scale, x, {s: quantile_threshold(x, s) for s in sparsities}
 
 
+def q4_projection(seed: int = 0, d_in: int = 4096, d_out: int = 11008, q_sigma: float = 2.5,
+                  w_sigma: float = 0.02, sparsities=(0.5,)):
+    """An int4 weight as a quantised checkpoint holds it, then x ~ Laplace(0, 1).
+
+    q (d_in, d_out): N(0, q_sigma^2) rounded to the nearest integer and clipped
+    to [-8, 7], packed two to a byte (even column in bits 0..3, odd column in
+    bits 4..7, two's complement) into QT4 (d_in, d_out / 2) uint8; scale
+    (d_out,) float32: w_sigma / q_sigma times U(0.9, 1.1).  Returns
+    (QT4, scale, x, {sparsity: t}).
+    """
+    rng = np.random.default_rng(seed)
+    QT4 = np.empty((d_in, d_out // 2), dtype=np.uint8)
+    rows = max(1, _CHUNK // max(1, d_out))
+    for lo in range(0, d_in, rows):
+        hi = min(d_in, lo + rows)
+        q = np.clip(np.rint(rng.normal(0.0, q_sigma, (hi - lo, d_out))), -8, 7).astype(np.int64)
+        nib = q & 0xF
+        QT4[lo:hi] = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    scale = (w_sigma / q_sigma * rng.uniform(0.9, 1.1, d_out)).astype(np.float32)
+    x = draw_vector(rng, d_in, "laplace")
+    return QT4, scale, x, {s: quantile_threshold(x, s) for s in sparsities}
+
+
 def f8_projection(seed: int = 0, d_in: int = 4096, d_out: int = 11008, q_sigma: float = 64.0,
                   w_sigma: float = 0.02, sparsities=(0.5,)):
     """An fp8 (e4m3) weight as a quantised checkpoint holds it, then x ~ Laplace(0, 1).
