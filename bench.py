@@ -66,7 +66,8 @@ def parse():
                          "'q8up70b' / 'f8up70b' / 'q4up70b' (int8 / fp8 / int4 weights, "
                          "8192->28672), "
                          "'nmN:M' (N:M mask + GEMM, e.g. 'nm8:16'), 'nmsp2:4' (packed 2:4 "
-                         "operand, sparse GEMM) or 'nmex2:4')")
+                         "operand, sparse GEMM), 'nmex2:4', 'gemm:MxKxN' (dense "
+                         "tensor-core GEMM) or 'gemmsp:MxKxN' (packed 2:4 GEMM)")
     ap.add_argument("--launches", type=int, default=8, help="launches in --profile-case mode")
     args = ap.parse_args()
     # at least three untimed warm-up steps; the JSON line reports the number run
@@ -1218,6 +1219,21 @@ def profile_case(args):
         Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(WT).cuda()
         for _ in range(args.launches):
             Y = sig.nm_act_gemm(Xd, Wd, n, m)
+        info = {"case": case, "launches": args.launches}
+    elif re.fullmatch(r"gemm(sp)?:\d+x\d+x\d+", case):
+        # one large tensor-core GEMM: dense on X ('gemm:MxKxN') or the packed
+        # 2:4 operand ('gemmsp:MxKxN'), for the CTA-pair kernels
+        M, K, N = (int(v) for v in case.split(":")[1].split("x"))
+        gen = torch.Generator(device="cpu").manual_seed(M + K + N)
+        Xd = torch.randn(M, K, generator=gen).half().cuda()
+        Wd = (torch.randn(K, N, generator=gen) * 0.02).half().cuda()
+        if case.startswith("gemmsp"):
+            pk = sig.sparsify_nm_packed(Xd, 2)
+            for _ in range(args.launches):
+                sig.nm_act_gemm_packed(pk, M, K, Wd)
+        else:
+            for _ in range(args.launches):
+                sig.nm_act_gemm(Xd, Wd, 4, 4)
         info = {"case": case, "launches": args.launches}
     elif case == "topk70b":
         (p,) = workloads.qsparse_70b(args.seed, names=("down",))
