@@ -610,23 +610,27 @@ __device__ __forceinline__ void commit_pair(uint32_t bar) {
       : "memory");
 }
 
-template <bool SPARSE>
+// WIDE (dense only): the pair computes a 256 x 512 tile as two M = 256,
+// N = 256 MMAs per K step into tensor-memory columns [0, 256) and [256, 512);
+// each CTA loads its 128 columns of each, so a stage brings 48 KB per CTA for
+// twice the work of a 32 KB stage of the 256 x 256 tile.
+template <bool SPARSE, bool WIDE = false>
 struct PairCfg {
-  static constexpr int kBN = 256;                        // N of the pair's MMA
+  static constexpr int kBN = WIDE ? 512 : 256;           // output columns of the pair's tile
   static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
-  static constexpr int kStages = SPARSE ? 4 : 6;
+  static constexpr int kStages = SPARSE ? 4 : (WIDE ? 4 : 6);
   static constexpr uint32_t kABytes = kBM * 64 * 2;      // 128 rows x 128 B
   static constexpr uint32_t kBBytes = kBK * (kBN / 2) * 2;
   static constexpr uint32_t kEBytes = SPARSE ? kSpMetaBytes : 0;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kEBytes;   // per CTA
-  static constexpr uint32_t kTmemCols = SPARSE ? 512u : 256u;
+  static constexpr uint32_t kTmemCols = (SPARSE || WIDE) ? 512u : 256u;
 };
 
-template <bool SPARSE>
+template <bool SPARSE, bool WIDE = false>
 struct __align__(1024) PairSmem {
-  using C = PairCfg<SPARSE>;
+  using C = PairCfg<SPARSE, WIDE>;
   uint16_t A[C::kStages][kBM * 64];
-  uint16_t B[C::kStages][C::kBK * (C::kBN / 2)];          // 2 blocks of 64 columns
+  uint16_t B[C::kStages][C::kBK * (C::kBN / 2)];          // kBN / 128 blocks of 64 columns
   uint8_t E[SPARSE ? C::kStages : 1][SPARSE ? kSpMetaBytes : 16];
   unsigned long long full[C::kStages];                    // used in the leader
   unsigned long long empty[C::kStages];
@@ -636,23 +640,25 @@ struct __align__(1024) PairSmem {
   int consumed;
 };
 
-template <bool SPARSE>
+template <bool SPARSE, bool WIDE = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, kMinBlocksForRegs)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                  const __grid_constant__ CUtensorMap mapE, const __grid_constant__ CUtensorMap mapY,
                  int M, int N,
                  int K, const float* __restrict__ shift, const float* __restrict__ colsum) {
-  using C = PairCfg<SPARSE>;
+  using C = PairCfg<SPARSE, WIDE>;
   constexpr int BN = C::kBN, BK = C::kBK, S = C::kStages;
+  constexpr int kMmas = BN / 256;                  // M = 256, N = 256 MMAs per K step
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  PairSmem<SPARSE>& sm = *reinterpret_cast<PairSmem<SPARSE>*>(
+  PairSmem<SPARSE, WIDE>& sm = *reinterpret_cast<PairSmem<SPARSE, WIDE>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const int m0 = blockIdx.x * kBM;                 // this CTA's rows
   const int n0 = blockIdx.y * BN;                  // the pair's columns
-  const int nb = n0 + (int)rank * (BN / 2);        // this CTA's half of B
+  // this CTA's half of each MMA's 256 columns: columns n0 + 256 h + 128 rank
+  const int nb = n0 + (int)rank * 128;
   const int kblocks = K / BK;
   volatile int* abort_flag = &sm.abort_flag;
   pdl_trigger();
@@ -692,8 +698,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
         if (leader) mbar_expect_tx(smem_u32(&sm.full[s]), 2 * C::kStageBytes);
         tma_load_2d_pair(smem_u32(sm.A[s]), &mapA, kb * 64, m0, fb);
 #pragma unroll
-        for (int j = 0; j < BN / 128; ++j)
-          tma_load_2d_pair(smem_u32(sm.B[s]) + j * (BK * 128), &mapB, nb + j * 64, kb * BK, fb);
+        for (int j = 0; j < BN / 128; ++j)   // block j: MMA j / 2, columns (j % 2) * 64 of its half
+          tma_load_2d_pair(smem_u32(sm.B[s]) + j * (BK * 128), &mapB,
+                           nb + (j >> 1) * 256 + (j & 1) * 64, kb * BK, fb);
         if constexpr (SPARSE)
           tma_load_1d_pair(smem_u32(sm.E[s]), &mapE,
                            (int)(((size_t)blockIdx.x * kblocks + kb) * (kSpMetaBytes / 8)), fb);
@@ -730,18 +737,22 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
                 : "memory");
           }
         } else {
-          constexpr uint32_t idesc = instr_desc_f16(2 * kBM, BN);
+          constexpr uint32_t idesc = instr_desc_f16(2 * kBM, 256);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t da = smem_desc(a0 + k * 32, 16, 1024);
-            const uint64_t db = smem_desc(b0 + k * 2048, BK * 128, 1024);
             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.ne.b32 p, %4, 0;\n\t"
-                "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-                "l"(da), "l"(db), "r"(idesc), "r"(acc)
-                : "memory");
+#pragma unroll
+            for (int h = 0; h < kMmas; ++h) {   // MMA h: its two 64-column blocks of B
+              const uint64_t db = smem_desc(b0 + h * 2 * (BK * 128) + k * 2048, BK * 128, 1024);
+              asm volatile(
+                  "{\n\t.reg .pred p;\n\t"
+                  "setp.ne.b32 p, %4, 0;\n\t"
+                  "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
+                      tmem + (uint32_t)(h * 256)),
+                  "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                  : "memory");
+            }
           }
         }
         commit_pair(smem_u32(&sm.empty[s]));      // frees stage s in both CTAs
@@ -836,15 +847,15 @@ bool use_pair(int M, int N, int K) {
   return M % 256 == 0 && N % 256 == 0 && N >= 2048 && K >= 2048;
 }
 
-template <bool SPARSE>
+template <bool SPARSE, bool WIDE = false>
 cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me,
                         const CUtensorMap& my, int M, int N, int K, const float* shift,
                         const float* colsum, cudaStream_t stream) {
-  const size_t smem = sizeof(PairSmem<SPARSE>) + 1024;
-  auto fn = gemm_pair_kernel<SPARSE>;
+  const size_t smem = sizeof(PairSmem<SPARSE, WIDE>) + 1024;
+  auto fn = gemm_pair_kernel<SPARSE, WIDE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(M / kBM, N / PairCfg<SPARSE>::kBN);
+  const dim3 grid(M / kBM, N / PairCfg<SPARSE, WIDE>::kBN);
   e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, ma, mb, me, my, M, N, K, shift, colsum);
   if (e != cudaSuccess) return e;
   return cudaPeekAtLastError();
@@ -887,8 +898,11 @@ cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_
   if (!make_map(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kBK)) return cudaErrorInvalidValue;
   if (!make_map(&my, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N, 32)) return cudaErrorInvalidValue;
-  if (use_pair(M, N, K))   // CTA pairs: 256 x 256 tiles, half of B per CTA
+  if (use_pair(M, N, K)) {   // CTA pairs: 256 x 512 (or 256 x 256) tiles, half of B per CTA
+    if (N % 512 == 0)
+      return launch_pair<false, true>(ma, mb, ma, my, M, N, K, shift, colsum, stream);
     return launch_pair<false>(ma, mb, ma, my, M, N, K, shift, colsum, stream);
+  }
   if (N % 256 == 0) return launch_bn<256>(ma, mb, my, M, N, K, shift, colsum, stream);
   return launch_bn<128>(ma, mb, my, M, N, K, shift, colsum, stream);
 }
