@@ -898,6 +898,11 @@ cudaError_t launch_gemm_f16_shift(const uint16_t* A, const uint16_t* WT, uint16_
   if (!make_map(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, kBM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, WT, (uint64_t)N, (uint64_t)K, (uint64_t)N, kBK)) return cudaErrorInvalidValue;
   if (!make_map(&my, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N, 32)) return cudaErrorInvalidValue;
+  // 256 x 512 pair tiles also for K >= 1024 when there are enough of them to
+  // fill the GPU's CTA pairs (A/B on B200, 16384 x 1024 x 1024: 35.0 against
+  // 50.0 us on 128 x 256 one-CTA tiles)
+  if (M % 256 == 0 && N % 512 == 0 && K >= 1024 && (M / 256) * (N / 512) >= kNumSMs / 2)
+    return launch_pair<false, true>(ma, mb, ma, my, M, N, K, shift, colsum, stream);
   if (use_pair(M, N, K)) {   // CTA pairs: 256 x 512 (or 256 x 256) tiles, half of B per CTA
     if (N % 512 == 0)
       return launch_pair<false, true>(ma, mb, ma, my, M, N, K, shift, colsum, stream);
@@ -926,7 +931,11 @@ cudaError_t launch_gemm_sp(const uint16_t* vals, const uint8_t* meta, const uint
     if (!make_map_meta(&me, meta, (uint64_t)M * (uint64_t)K / 8)) return cudaErrorInvalidValue;
     return launch_pair<true>(ma, mb, me, my, M, N, K, nullptr, nullptr, stream);
   }
-  if (N % 256 == 0) return launch_sp_bn<256>(ma, mb, meta, my, M, N, K, stream);
+  // 128-column tiles (two CTAs per SM) once 128 x 256 tiles would take two
+  // waves or more (A/B on B200, 16384 x 1024 x 1024: 34.8 against 38.1 us;
+  // at 4096 x 1024 x 1024 the wide tiles win, 9.2 against 9.8 us)
+  if (N % 256 == 0 && (M / kBM) * (N / 256) < 2 * kNumSMs)
+    return launch_sp_bn<256>(ma, mb, meta, my, M, N, K, stream);
   return launch_sp_bn<128>(ma, mb, meta, my, M, N, K, stream);
 }
 

@@ -109,6 +109,22 @@ def test_sparse_gemm_shapes(sig, rows, K, N):
     assert sig.take_device_error() == 0
 
 
+def test_gemm_paths_of_large_token_blocks(sig):
+    """9472 tokens x 1024 -> 1024: 296 one-CTA tiles of 128 x 256, so the 2:4
+    GEMM takes 128-column tiles, and 74 pair tiles of 256 x 512, so the dense
+    GEMM (8:16 on the masked block) takes the wide CTA-pair kernel at K = 1024.
+    Every output of 512 sampled token rows is checked."""
+    rows, K, N = 9472, 1024, 1024
+    WT, X = workloads.nm_tokens(7, rows=rows, d=K, d_out=N)
+    sample = np.sort(np.random.default_rng(5).choice(rows, 512, replace=False))
+    dX, dW = to_dev(X), to_dev(WT)
+    for n, m in ((2, 4), (8, 16)):
+        Y = to_host(sig.nm_act_gemm(dX, dW, n, m))
+        Y64, B = oracle.nm_gemm(X, WT, oracle.nm_mask(X, n, m), rows=sample)
+        assert_within(Y[sample], Y64, B, f"{rows}x{K}x{N} {n}:{m}")
+    assert sig.take_device_error() == 0
+
+
 def test_packed_entry_point_matches_the_fused_call(sig):
     """nm_act_gemm_packed on sparsify_nm's packed output is the product
     nm_act_gemm computes for 2:4 (bit for bit: same operand, same kernel)."""
