@@ -139,8 +139,9 @@ def workspace(op: int, d_in: int, d_out: int = 0, rows: int = 0, device=None,
               stream=None) -> torch.Tensor:
     """A zeroed workspace for ``op`` at these sizes, cached per (device, stream).
 
-    The kernels return their counters to zero, so a cached workspace can be
-    reused by later calls on the same stream.  Calls on different streams get
+    The kernels leave their counters ready for the next call (returned to
+    zero, or advanced to the next epoch), so a cached workspace can be reused
+    by later calls on the same stream.  Calls on different streams get
     different workspaces.
     """
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())

@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "nm_ex.h"
+#include "nm_pack.cuh"
 #include "nm_select.cuh"
 
 #include <cooperative_groups.h>
@@ -733,23 +734,10 @@ cudaError_t launch_topk(const uint16_t* x, int d, int k, uint32_t* mask_bits, in
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, x, d, k, chunk, mask_bits, idx, nnz);
 }
 
-// Packed 2:4 operand of the sparse tensor-core GEMM.  N = 2 keeps the two
-// largest |x| of every block of four (ties by lower position, NaN last); N = 1
-// keeps the largest and pads the second slot with +0 at the block's smallest
-// other position.  The two slots are written in ascending position order
-// (values to vals, positions as the metadata nibble p0 | p1 << 2).
-//
-// The metadata of a 128-row x 128-entry block is 128 lanes x 16 bytes in the
-// order a 128x128b tensor-memory copy hands it to the sparse MMA: lane
-// L = r % 8 + 8 h + 16 (r / 16) holds, for K group j (entries 32 j .. 32 j +
-// 31), the 16 bits of row r's half h (entries 32 j + 16 h .. + 15, four
-// nibbles, block q at bits 4 q) at bytes 4 j, 4 j + 1 when r % 16 < 8, else at
-// bytes 4 j + 2, 4 j + 3.  Rows 32 c .. 32 c + 31 own lanes 32 c .. 32 c + 31,
-// one contiguous quarter of the block's 2048 bytes.
-//
-// One CTA per 32 rows x 128 entries; thread t takes row t / 8 of them and
-// entries 16 (t % 8) .. + 15: four blocks, i.e. exactly one 16-bit metadata
-// field (group j = (t % 8) / 2, half h = t % 2).  The quarter is assembled in
+// Packed 2:4 operand of the sparse tensor-core GEMM (the selection and the
+// metadata layout are in nm_pack.cuh).  One CTA per 32 rows x 128 entries;
+// thread t takes row t / 8 of them and entries 16 (t % 8) .. + 15: four
+// blocks, i.e. exactly one 16-bit metadata field.  The quarter is assembled in
 // shared memory and stored as 512 contiguous bytes.
 template <int N>
 __global__ void __launch_bounds__(256)
@@ -764,33 +752,10 @@ nm_pack_kernel(const uint16_t* __restrict__ X, int d, int kblocks, uint16_t* __r
   pdl_wait();
   const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(src));
   const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
-  uint32_t out[4];
-  uint32_t nib = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    // the block's four entries, entry j at bits 16 j
-    const uint4& w = q < 2 ? v0 : v1;
-    const uint64_t ev = (q & 1) ? ((uint64_t)w.w << 32 | w.z) : ((uint64_t)w.y << 32 | w.x);
-    uint32_t comp[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)    // unique composites: position breaks ties
-      comp[j] = (mag_key((uint16_t)(ev >> (16 * j))) << 2) | (uint32_t)(3 - j);
-    const uint32_t top = select_top_n<4>(comp, N);            // the kept positions
-    // N = 1: the second slot is the smallest position not kept
-    const uint32_t slots = N == 2 ? top : top | ((top & 1u) ? 2u : 1u);
-    const uint32_t p0 = (uint32_t)(__ffs(slots) - 1);
-    const uint32_t p1 = (uint32_t)(31 - __clz(slots));
-    const uint32_t lo = ((top >> p0) & 1u) ? (uint32_t)(ev >> (16 * p0)) & 0xffffu : 0u;  // padding: +0
-    const uint32_t hi = ((top >> p1) & 1u) ? (uint32_t)(ev >> (16 * p1)) & 0xffffu : 0u;
-    out[q] = lo | (hi << 16);
-    nib |= (p0 | (p1 << 2)) << (4 * q);
-  }
-  *reinterpret_cast<uint4*>(vals + row * (d / 2) + kb * 64 + part * 8) =
-      make_uint4(out[0], out[1], out[2], out[3]);
-  const int j = part >> 1, h = part & 1;
-  const int r = (rq & 3) * 32 + r32;                          // row inside the 128-row block
-  const int L = (r & 7) + 8 * h + 16 * (r >> 4);              // in [32 (rq % 4), +32)
-  *reinterpret_cast<uint16_t*>(quarter + (L & 31) * 16 + 4 * j + 2 * ((r >> 3) & 1)) = (uint16_t)nib;
+  uint4 packed;
+  const uint32_t nib = pack_piece<N>(v0, v1, packed);
+  *reinterpret_cast<uint4*>(vals + row * (d / 2) + kb * 64 + part * 8) = packed;
+  *reinterpret_cast<uint16_t*>(quarter + meta_quarter_offset(rq * 32 + r32, part)) = (uint16_t)nib;
   __syncthreads();
   if (t < 32) {
     const size_t tile = (size_t)(rq >> 2) * kblocks + kb;
