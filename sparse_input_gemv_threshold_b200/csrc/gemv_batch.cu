@@ -123,7 +123,16 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
   const __half2 th2 = thresh_half2(a.t);
   const float th = __half2float(__low2half(th2));
   const int ngroups = (d_in + 7) >> 3;
-  const int K = s < ngroups ? (ngroups - 1 - s) / S + 1 : 0;
+  // the slice's groups: for 16 tokens the contiguous run [g_lo, g_lo + K),
+  // so that neighbouring threads load neighbouring 16-byte groups of each
+  // token; for fewer tokens every S-th group from s, g = s + k * S.
+  // Measured on B200 at 4096 -> 11008: 16 tokens 29.98 -> 27.99 us with the
+  // contiguous run; 2 and 8 tokens 0.3 us slower with it (not taken)
+  constexpr bool kContig = TOK == 16;
+  const int g_lo = kContig ? (int)(((long long)s * ngroups) / S) : s;
+  const int g_step = kContig ? 1 : S;
+  const int K = kContig ? (int)(((long long)(s + 1) * ngroups) / S) - g_lo
+                        : (s < ngroups ? (ngroups - 1 - s) / S + 1 : 0);
   const int nwords = (K + 3) >> 2;
   // one thread per group: every token's loads in flight together; for 16
   // tokens the groups are kept in shared memory for the staging
@@ -131,7 +140,7 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
   for (int k = tid; k < nwords * 4; k += kThreads) {
     uint32_t u = 0;
     if (k < K) {
-      const int e0 = (s + k * S) * 8;
+      const int e0 = (g_lo + k * g_step) * 8;
       uint4 v[TOK];
 #pragma unroll
       for (int b = 0; b < TOK; ++b)
@@ -220,7 +229,7 @@ batch_mma_kernel(const __grid_constant__ BArgs a) {
       const int rk = base + __popc(bits & ((1u << lane) - 1u));
       if (((bits >> lane) & 1u) && rk >= c_lo && rk < c_hi) {
         const int kg = w * 4 + (lane >> 3);              // the slice's group of this row
-        const int i = (s + kg * S) * 8 + (lane & 7);
+        const int i = (g_lo + kg * g_step) * 8 + (lane & 7);
         const int j = rk - c_lo;
         sidx[j] = i;
 #pragma unroll
