@@ -544,7 +544,13 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     store_col(colc, gs, us);
   }
   if (gave_up) atomicOr(&g_gemv_error, 2u);
-  if (tid == 0) st_relaxed_u32(a.epochs + cg, tag);   // the next call tags with tag + 1
+  // the next call tags with tag + 1.  Only a finisher that has seen every
+  // slice's word (its half holds a column) knows that every slice has read
+  // the epoch; the finisher of a tile's empty second half (a tile of at most
+  // 128 columns) must leave the epoch alone, or a slice that reads it late
+  // would tag with the next call's tag
+  const bool half_has_cols = (cg - e_first) * kTile + kdes * (kTile / 2) < e_dout;
+  if (tid == 0 && half_has_cols) st_relaxed_u32(a.epochs + cg, tag);
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

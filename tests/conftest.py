@@ -45,6 +45,24 @@ def sig():
     return mod
 
 
+@pytest.fixture(autouse=True)
+def _no_bounded_wait_gave_up(request):
+    """After every gpu test: no kernel may have given up a bounded wait (the
+    library's device error words are read and cleared).  A test that makes a
+    wait run out on purpose reads and clears the words itself."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    mod = sys.modules.get("sparse_input_gemv_threshold_b200")
+    if mod is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    code = mod.take_device_error()
+    assert code == 0, f"a kernel gave up a bounded wait (device error bits {code:#x})"
+
+
 def to_dev(a):
     import numpy as np
     import torch

@@ -53,8 +53,10 @@ def _check(sig, ra, t, what):
     return y, m
 
 
+# (64, 64, 76800): 300 output tiles, one slice each (no split-K partials)
 @pytest.mark.parametrize("d_in,r,d_out", [(64, 48, 24), (1000, 264, 520), (33, 8, 8),
-                                          (4096, 2048, 4096), (4096, 1024, 11008)])
+                                          (4096, 2048, 4096), (4096, 1024, 11008),
+                                          (64, 64, 76800)])
 def test_rank_adapter_shapes(sig, d_in, r, d_out):
     ra = workloads.rank_adapter(seed=d_in + r + d_out, d_in=d_in, r=r, d_out=d_out)
     t = _median_score_threshold(ra)
@@ -83,3 +85,39 @@ def test_rank_adapter_deterministic(sig):
     y, _, _ = _run(sig, ra, t)
     assert np.array_equal(first, y.view(np.uint16))
     del torch
+
+
+# (64, 48, 24) and (33, 8, 8): the output tile's second 128-column half is
+# empty, and the slice finishing it must not advance the tile's epoch before
+# every slice has read it
+@pytest.mark.parametrize("d_in,r,d_out", [(4096, 2048, 4096), (64, 48, 24), (33, 8, 8),
+                                          (1000, 264, 520)])
+def test_rank_adapter_repeated_calls_on_one_workspace(sig, d_in, r, d_out):
+    """One workspace through many calls: the split-K partial sums carry the
+    tile's epoch, which every call advances once; results equal those of a
+    fresh workspace bit for bit, and no bounded wait gives up."""
+    import torch
+    ra = workloads.rank_adapter(seed=7, d_in=d_in, r=r, d_out=d_out)
+    d_in, r = ra.BT.shape
+    d_out = ra.AT.shape[1]
+    t_mid = _median_score_threshold(ra)
+    ts = [t_mid, 0.5 * t_mid, 2.0 * t_mid]
+    dx, dB, dA = to_dev(ra.x), to_dev(ra.BT), to_dev(ra.AT)
+    n_ws = sig.workspace_bytes(sig.OP_RANK_ADAPTER, d_in, d_out, r)
+
+    def new_ws():
+        return torch.zeros(n_ws, dtype=torch.uint8, device="cuda")
+
+    fresh = {t: to_host(sig.rank_adapter_sparse(dx, dB, dA, t, ws=new_ws())).view(np.uint16).copy()
+             for t in ts}
+    ws = new_ws()
+    for k in range(12):
+        t = ts[k % 3]
+        y = to_host(sig.rank_adapter_sparse(dx, dB, dA, t, ws=ws)).view(np.uint16)
+        assert np.array_equal(y, fresh[t]), (k, t)
+    # a changed activation between calls on the same workspace
+    x2 = (ra.x.astype(np.float32) * -1.5).astype(np.float16)
+    y2 = to_host(sig.rank_adapter_sparse(to_dev(x2), dB, dA, t_mid, ws=ws)).view(np.uint16)
+    ref2 = to_host(sig.rank_adapter_sparse(to_dev(x2), dB, dA, t_mid, ws=new_ws())).view(np.uint16)
+    assert np.array_equal(y2, ref2)
+    assert sig.take_device_error() == 0
