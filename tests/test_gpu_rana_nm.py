@@ -110,13 +110,19 @@ def test_nm_mask_ragged_and_ties(sig):
         X[0, :3] = np.nan
         X[1, 1] = np.inf
         for m in ms:
-            for n in sorted({1, max(1, m // 2), m}):
+            for n in sorted({1, min(3, m), max(1, m // 2), max(1, m - 1), m}):
                 _check_nm(sig, X, n, m, f"d={d} {n}:{m}")
     _check_nm(sig, np.zeros((0, 64), np.float16), 2, 4, "zero rows")
     # several vectors per thread, rows whose last word is partial
     X = workloads.draw_vector(rng, (37, 1000), "laplace")
     for n, m in ((1, 1), (1, 2), (2, 4), (1, 4), (3, 8), (8, 8)):
         _check_nm(sig, X, n, m, f"37x1000 {n}:{m}")
+    # 16- and 32-entry blocks on rows of 1024 and 992 entries (31 words, the
+    # grid's last warp partly past the end), several n
+    for d in (1024, 992):
+        X = workloads.draw_vector(rng, (37, d), "laplace")
+        for n, m in ((5, 16), (8, 16), (15, 16), (1, 32), (11, 32), (16, 32), (32, 32)):
+            _check_nm(sig, X, n, m, f"37x{d} {n}:{m}")
 
 
 # ---------------------------------------------------------------------------
