@@ -99,7 +99,7 @@ SIG_API int sig_abi_version(void);
 /*
  * Bytes of device workspace an operation needs for the given sizes (0 when
  * the operation needs none).  Returns 0 and sets nothing for an unknown op.
- * It holds split-K partial sums and arrival counters; the gated MLP also
+ * It holds split-K partial sums and per-tile epoch or arrival counters; the gated MLP also
  * keeps its fp16 hidden vector there when h_out is NULL, and the N:M GEMM its
  * masked activation block.
  */
@@ -208,9 +208,10 @@ SIG_API size_t sig_nm_packed_bytes(int64_t rows, int64_t d);
  *        size is 0 (one slice per tile, which the planner chooses above 296
  *        tiles, i.e. d_out > 75776) ws may be NULL.
  * The split-K finish: every slice stores its partial sums and exits; the
- * tile's last slice waits (bounded, ~2 s; on expiry it sets bit 1 of the
- * device error word, see sig_take_device_error) until every slice's word
- * carries this call's tag, then adds them in slice order.
+ * tile's last two slices each finish one 128-column half: they wait (bounded,
+ * ~2 s; on expiry bit 1 of the device error word is set, see
+ * sig_take_device_error) until every slice's word carries this call's tag,
+ * then add them in slice order.
  * The result is bit-identical from run to run (fixed-order split-K reduction;
  * no floating-point atomics).  An empty mask writes y = 0.
  * Errors: SIG_ERR_NULL, SIG_ERR_SHAPE (d_in < 1, d_in > SIG_MAX_D_IN, d_out < 8,

@@ -18,28 +18,36 @@
 // equal runs.  Up to four weights that read the same input (q, k, v; gate, up)
 // share one launch and one mask: their column tiles are laid end to end.  One
 // launch does everything:
-//   1. the CTA loads its groups of the activation (from L2), ballots them into
-//      shared mask words with fp16 SIMD compares against the threshold rounded
-//      up to fp16 (exact for fp16 inputs), prefix-sums the words' popcounts
-//      (one barrier), and the warps place its kept rows in ascending order,
-//      one word per warp and one bit per lane (rank = word prefix + popcount
-//      of the lower bits);
+//   1. the CTA loads its groups of the activation (from L2) and takes their
+//      mask bits with fp16 SIMD compares against the threshold rounded up to
+//      fp16 (exact for fp16 inputs).  A slice of at most 256 groups (every
+//      Llama-2-7B and 70B launch) gives one group to each thread: one
+//      block-wide exclusive scan of the popcounts gives each thread the rank
+//      of its first kept row, and the thread places its rows itself.  Wider
+//      slices keep mask words in shared memory, prefix-sum their popcounts,
+//      and the warps place the rows one word per warp and one bit per lane
+//      (rank = word prefix + popcount of the lower bits);
 //   2. 8 warps stream the slice's rows of the tile, 8 rows in flight per warp:
 //      16-byte non-allocating loads with an L2 evict-first policy, the
 //      activation value riding along as a broadcast load, fp32 FMA (8-bit
 //      weights: 12 rows in flight, 8-byte lanes of eight weights, each made an
 //      exact float value in registers (int8: sign extension and an int-to-
 //      float conversion; e4m3: the hardware conversion to fp16 pairs, then
-//      packed float32 FMAs); the column scale multiplies the finished sum);
+//      packed float32 FMAs); int4 weights: 8 rows, 4-byte lanes of eight
+//      nibbles, sign-extended by shifts; the column scale multiplies the
+//      finished sum);
 //   3. the warps' sums meet in shared memory (fixed order) and the CTA
 //      stores one partial per column as a 64-bit word {value, tag} (tag = the
 //      tile's epoch + 1, read from the workspace at the start) with a relaxed
-//      store, and exits.  The tile's last slice, the CTA dispatched last,
-//      instead polls the tile's partial words in batches until every tag is
-//      current, adds them in slice order (its own last) and stores fp16; it
-//      then advances the tile's epoch.  The value and its tag travel in one
-//      single-copy-atomic 64-bit word, so no fence and no atomic stand
-//      between the last partial store and the sum.  The wait is bounded
+//      store, and exits.  The tile's last two slices, the CTAs dispatched
+//      last, instead finish one 128-column half each: two threads per column
+//      poll the partial words of half the slices each, in batches, until
+//      every tag is current, add them in slice order, and the two halves are
+//      added in a fixed order and stored as fp16.  A finisher whose half holds
+//      a column then advances the tile's epoch (it has seen every slice's
+//      word, so every slice has read the epoch).  The value and its tag
+//      travel in one single-copy-atomic 64-bit word, so no fence and no atomic
+//      stand between the last partial store and the sum.  The wait is bounded
 //      (~2 s of clock cycles; on expiry the kernel sets a bit in the device
 //      error word and stores what it has).
 // No floating-point atomics; y is bit-identical from run to run.
@@ -50,7 +58,7 @@
 
 namespace sig {
 
-// Device error word of the split-K finish (bit 1: a tile's last slice gave up
+// Device error word of the split-K finish (bit 1: a tile's finishing slice gave up
 // waiting for the other slices' partial sums); read with the GEMM's word.
 __device__ unsigned g_gemv_error = 0u;
 
@@ -399,7 +407,7 @@ sgemv_kernel(const __grid_constant__ KArgs a) {
     }
   }
 
-  // ---- 3. CTA partial, then the last arriver finishes the tile ---------
+  // ---- 3. CTA partial, then the last two slices finish the tile -------
   __syncthreads();   // the words / prefixes region becomes the warp-sum buffer
   float* red = reinterpret_cast<float*>(smem);
   {
