@@ -83,6 +83,52 @@ def test_wide_slice_path(sig):
     assert_within(y[cols], ref["y64"], ref["bound"], "wide slices")
 
 
+@pytest.mark.parametrize("sparsity", [0.0, 0.5, 0.99])
+def test_largest_input_width(sig, sparsity):
+    """d_in = SIG_MAX_D_IN (131072): one column tile, 64 slices of 256 input
+    groups each (the widest slice of the one-group-per-thread prologue); also
+    the index path over the same rows."""
+    p = workloads.projection("m", 131072, 64, sigma=0.02, dist="laplace", seed=23,
+                             sparsities=(sparsity,))
+    t = p.thresholds[sparsity]
+    dW, dx = to_dev(p.WT), to_dev(p.x)
+    ref = oracle.sparse_linear(p.WT, p.x, oracle.threshold_mask(p.x, t))
+    y = to_host(sig.sparse_gemv(dW, dx, t=t))
+    assert_within(y, ref["y64"], ref["bound"], f"d_in 131072 s={sparsity}")
+    mb, idx, nnz = sig.sparsify_threshold(dx, t)
+    assert int(to_host(nnz)[0]) == ref["nnz"]
+    y2 = to_host(sig.sparse_gemv(dW, dx, idx=idx, nnz=nnz))
+    assert_within(y2, ref["y64"], ref["bound"], f"d_in 131072 s={sparsity} index list")
+
+
+def test_slice_rows_in_several_chunks(sig):
+    """One slice per tile (d_out above 296 tiles) over 4200 kept inputs: the
+    chunked prologue places the slice's rows in two chunks (at most 4096 rows
+    of a slice are staged in shared memory at once)."""
+    p = workloads.projection("c", 4200, 76032, sigma=0.02, dist="laplace", seed=31,
+                             sparsities=(0.0,))
+    t = p.thresholds[0.0]
+    cols = np.concatenate([np.arange(16), np.random.default_rng(7).choice(76032, 240, replace=False),
+                           np.arange(76032 - 16, 76032)])
+    y = to_host(sig.sparse_gemv(to_dev(p.WT), to_dev(p.x), t=t))
+    ref = oracle.sparse_linear(p.WT, p.x, oracle.threshold_mask(p.x, t), cols=cols)
+    assert ref["nnz"] == 4200
+    assert_within(y[cols], ref["y64"], ref["bound"], "two chunks")
+
+
+def test_widest_output(sig):
+    """d_out = 2^20 (4096 column tiles, one slice each, no workspace)."""
+    p = workloads.projection("n", 8, 1 << 20, sigma=0.02, dist="laplace", seed=29,
+                             sparsities=(0.5,))
+    t = p.thresholds[0.5]
+    assert sig.workspace_bytes(sig.OP_SPARSE_GEMV, 8, 1 << 20) == 0
+    y = to_host(sig.sparse_gemv(to_dev(p.WT), to_dev(p.x), t=t))
+    cols = np.concatenate([np.arange(64), np.random.default_rng(5).choice(1 << 20, 448, replace=False),
+                           np.arange((1 << 20) - 64, 1 << 20)])
+    ref = oracle.sparse_linear(p.WT, p.x, oracle.threshold_mask(p.x, t), cols=cols)
+    assert_within(y[cols], ref["y64"], ref["bound"], "d_out 2^20")
+
+
 def test_index_path_and_fused_path_agree(sig):
     # the two paths split the kept rows differently (interleaved 8-input groups
     # under a threshold, equal runs of an index list), so they agree within the
