@@ -542,9 +542,10 @@ def cublas_dense(groups, copies, gx, stream, steps):
 
 
 def bench_topk(args, stream, sig, hbm_peak):
+    """Q-Sparse top-k then the index-list GEMV, both 70B MLP shapes, at the
+    keep fractions 0.6, 0.5 and 0.4 of d_in."""
     import torch
     projs = workloads.qsparse_70b(args.seed)
-    k_frac = 0.5
     W = [torch.from_numpy(p.WT).cuda() for p in projs]
     Wc = [w.clone() for w in W]
     X = [torch.from_numpy(p.x).cuda() for p in projs]
@@ -554,33 +555,38 @@ def bench_topk(args, stream, sig, hbm_peak):
     bufs = [(torch.empty((p.d_in + 31) // 32, dtype=torch.int32, device="cuda"),
              torch.empty(p.d_in, dtype=torch.int32, device="cuda"),
              torch.empty(1, dtype=torch.int32, device="cuda")) for p in projs]
-    ks = [workloads.topk_count(k_frac, p.d_in) for p in projs]
+    steps = 200
+    by_keep = {}
+    for k_frac in (0.6, 0.5, 0.4):
+        ks = [workloads.topk_count(k_frac, p.d_in) for p in projs]
 
-    def f(ws_w):
-        def g():
+        def f(ws_w, ks=ks):
+            def g():
+                for j, p in enumerate(projs):
+                    mb, idx, nnz = bufs[j]
+                    sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
+                    sig.sparse_gemv(ws_w[j], X[j], idx=idx, nnz=nnz, y=ys[j], ws=ws[j], stream=stream)
+            return g
+        sg = StepGraphs([f(W), f(Wc)], stream)
+        sec = time_steps(sg, steps, 8, stream)
+        us = sec / steps * 1e6
+        b = sum(k * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out for k, p in zip(ks, projs))
+
+        def h(ks=ks):   # top-k alone
             for j, p in enumerate(projs):
                 mb, idx, nnz = bufs[j]
                 sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
-                sig.sparse_gemv(ws_w[j], X[j], idx=idx, nnz=nnz, y=ys[j], ws=ws[j], stream=stream)
-        return g
-    sg = StepGraphs([f(W), f(Wc)], stream)
-    steps = 200
-    sec = time_steps(sg, steps, 8, stream)
-    us = sec / steps * 1e6
-    b = sum(k * 2 * p.d_out + 2 * p.d_in + 2 * p.d_out for k, p in zip(ks, projs))
-    # top-k alone
-    def h():
-        for j, p in enumerate(projs):
-            mb, idx, nnz = bufs[j]
-            sig.sparsify_topk(X[j], ks[j], mask_bits=mb, idx=idx, nnz=nnz, stream=stream)
-    st = StepGraphs([h], stream)
-    sec_t = time_steps(st, steps, 8, stream)
-    res = {"shapes": "8192->28672 and 28672->8192", "keep": k_frac,
-           "us_per_pair": round(us, 2), "GBps": round(b / (us * 1e-6) / 1e9, 1),
-           "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
-           "topk_select_us_per_pair": round(sec_t / steps * 1e6, 2),
+        st = StepGraphs([h], stream)
+        sec_t = time_steps(st, steps, 8, stream)
+        by_keep[k_frac] = {"keep": k_frac, "k": ks, "us_per_pair": round(us, 2),
+                           "GBps": round(b / (us * 1e-6) / 1e9, 1),
+                           "frac_of_peak": round(b / (us * 1e-6) / 1e9 / hbm_peak, 4),
+                           "topk_select_us_per_pair": round(sec_t / steps * 1e6, 2)}
+        del sg, st
+    res = {"shapes": "8192->28672 and 28672->8192", **by_keep[0.5],
+           "by_keep": [by_keep[k] for k in (0.6, 0.5, 0.4)],
            "l2": "2 rotating weight copies of 940 MB"}
-    del W, Wc, sg, st
+    del W, Wc
     torch.cuda.empty_cache()
     return res
 
