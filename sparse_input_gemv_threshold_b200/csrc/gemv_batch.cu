@@ -9,9 +9,9 @@
 // registers: a row that token b drops contributes x_b,i = 0 to y_b.
 //
 // Launch shape: C x S CTAs of 256 threads (three per SM for up to 8 tokens,
-// two for up to 16), a CTA owns a
-// 256-output column tile and the union rows of its interleaved 8-input
-// groups (slice s owns groups s, s+S, s+2S, ...):
+// two for up to 16), a CTA owns a 256-output column tile and the union rows
+// of its slice's 8-input groups (up to 8 tokens: slice s owns groups s, s+S,
+// s+2S, ...; 16 tokens: a contiguous run of about 1/S of the groups):
 //   1. one thread per group loads that group of every token's x (from L2,
 //      all tokens' loads in flight together) and ORs their fp16 threshold
 //      compares into a union byte; the popcounts are prefix-summed and the
